@@ -1,0 +1,178 @@
+/*
+ * moe_nvfp4.h -- C ABI of the NVFP4 weight-only routed-expert MoE layer for B200 (sm_100a).
+ *
+ * One call computes one routed-expert SwiGLU MoE layer of a large sparse model: for each
+ * token, the top-k of E router logits (ties to the lower expert index) with softmax
+ * weights over the k selected logits, then for every selected expert e
+ *     y = Wd_e (silu(Wg_e x) * (Wu_e x)),
+ * and out = sum over the k experts of weight * y, rounded to BF16.  Expert weights are
+ * NVFP4 (weight = e2m1(code) * e4m3(block scale) * global); activations are BF16.
+ *
+ * Sources (pages on Reflection's Beam-1.0-501B-A23B):
+ *  - "Beam 1.0 501B-A23B, streaming pack, NVFP4 experts / MLX 8-bit residents", section
+ *    "What this pack holds": the expert record (gate, up and down, each E2M1 codes in U32
+ *    words, one E4M3 block scale per 16 inputs and one F32 global scale), the MLX block
+ *    scale e4m3(s) x (g / 2688) in f32, 256 routed experts with 8 active per token,
+ *    activations in BF16.
+ *  - "Beam-1.0-501B-A23B VQ GGUF", section "What stays native": router logits and SwiGLU
+ *    are FP32 numerics; section "Kernel budget on GB10": hidden 5,120, intermediate 2,560,
+ *    mid values staged as BF16.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named *_dev are device memory of the current CUDA device, *_host are host
+ *    memory; the caller owns all of them and the library keeps none after the call.
+ *  - Tensors are dense row-major.  x [T, H] and out [T, H] are BF16 (uint16 bit patterns),
+ *    logits [T, E] are f32.  Device tensors must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Device work is only
+ *    enqueued: errors raised by a kernel at run time surface at the caller's next
+ *    synchronisation, or through moe_nvfp4_device_status().
+ *  - Arguments are validated on the host before anything is enqueued; on a negative return
+ *    nothing was enqueued (except MOE_NVFP4_ERR_CUDA from a launch) and
+ *    moe_nvfp4_last_error() gives a message for the calling thread.
+ *  - There is no CPU fallback: without an sm_100 device every compute entry point returns
+ *    MOE_NVFP4_ERR_UNSUPPORTED.
+ */
+#ifndef MOE_NVFP4_H_
+#define MOE_NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define MOE_NVFP4_OK               0
+#define MOE_NVFP4_ERR_INVALID_ARG (-1)  /* null pointer, bad k, T < 0, misaligned pointer   */
+#define MOE_NVFP4_ERR_UNSUPPORTED (-2)  /* shape outside the supported set, no sm_100 device */
+#define MOE_NVFP4_ERR_CUDA        (-3)  /* a CUDA runtime call or launch failed              */
+#define MOE_NVFP4_ERR_WORKSPACE   (-4)  /* caller workspace too small, or growth refused
+                                           during stream capture                             */
+#define MOE_NVFP4_ERR_TIMEOUT     (-5)  /* a bounded device-side wait gave up (device status) */
+
+/* Expert-GEMM path selection for moe_nvfp4_forward_ex. */
+#define MOE_NVFP4_PATH_AUTO    0
+#define MOE_NVFP4_PATH_DECODE  1   /* memory-bound grouped GEMV/GEMM, any number of tokens */
+#define MOE_NVFP4_PATH_PREFILL 2   /* tensor-core (tcgen05) grouped GEMM                     */
+
+/*
+ * Expert bank: E records in device memory, record e at base + e * record_stride.
+ * Inside a record, projection p (0 = gate [I, H], 1 = up [I, H], 2 = down [H, I]; shape
+ * [out, in], row-major) has
+ *   codes   at codes_off[p]:  [out, in/8] little-endian uint32 words; input i of a row is
+ *           the 4-bit E2M1 field at bits 4*(i%8) .. 4*(i%8)+3 of word i/8 (low nibble first);
+ *   scales  at scales_off[p]: [out, in/16] E4M3 (OCP "FN") bytes, scale b covering inputs
+ *           16b .. 16b+15 of its row;
+ *   global  at global_off[p]: one f32.
+ * global_mode 0: the weight is e2m1 * e4m3 * global.  global_mode 1: the stored f32 is the
+ * streaming pack's g and the multiplier is f32(g / 2688), as the pack page says MLX forms it.
+ * base, record_stride, codes_off and scales_off must be multiples of 16; global_off of 4.
+ * The bank is read only; several calls may share it.
+ */
+typedef struct moe_nvfp4_bank {
+  int32_t num_experts;    /* E, 1 .. 1024                                    */
+  int32_t hidden;         /* H, a multiple of 128                            */
+  int32_t intermediate;   /* I, a multiple of 128                            */
+  int32_t global_mode;    /* 0 or 1                                          */
+  const void* base_dev;   /* device pointer to record 0                      */
+  uint64_t record_stride; /* bytes between records                           */
+  uint64_t codes_off[3];
+  uint64_t scales_off[3];
+  uint64_t global_off[3];
+} moe_nvfp4_bank;
+
+/*
+ * The layer, out = MoE(x).  Inputs: x_dev [T, H] BF16, logits_dev [T, E] f32, T >= 0
+ * (T = 0 returns OK and enqueues nothing), 1 <= k <= min(E, 32).  Output: out_dev [T, H]
+ * BF16 (round to nearest even).  Scratch comes from a per-device workspace owned by the
+ * library that grows on demand (a growth synchronises the device; it is refused with
+ * MOE_NVFP4_ERR_WORKSPACE while `stream` is capturing -- call once outside capture first,
+ * or use moe_nvfp4_forward_ex with a caller workspace).  Not thread-safe per device when
+ * the internal workspace is used from several host threads on different streams.
+ */
+int moe_nvfp4_forward(const void* x_dev, const float* logits_dev, int64_t T,
+                      const moe_nvfp4_bank* bank, int32_t k, void* out_dev, void* stream);
+
+/*
+ * As moe_nvfp4_forward, plus:
+ *  x_next_dev     if not NULL, also writes x_next [T, H] = bf16(x + out) (the residual add of
+ *                 stacked layers; the sum of the two BF16 values rounded once);
+ *  workspace_dev  caller scratch of workspace_bytes >= moe_nvfp4_workspace_bytes(...), 256-byte
+ *                 aligned; if NULL the internal workspace is used;
+ *  path           MOE_NVFP4_PATH_*; AUTO picks the decode path when T*k <= 8*E.
+ * With a caller workspace nothing is allocated, so the call can be captured in a CUDA graph.
+ */
+int moe_nvfp4_forward_ex(const void* x_dev, const float* logits_dev, int64_t T,
+                         const moe_nvfp4_bank* bank, int32_t k, void* out_dev,
+                         void* x_next_dev, void* workspace_dev, size_t workspace_bytes,
+                         int32_t path, void* stream);
+
+/*
+ * End-to-end call with host tensors: copies x_host [T, H] BF16 and logits_host [T, E] f32 to
+ * the device, runs the layer on the resident bank, copies out [T, H] BF16 back to out_host and
+ * synchronises `stream` before returning.  Host buffers may be pageable or pinned (pinned
+ * copies are asynchronous and faster).  Uses the internal workspace and internal staging
+ * buffers for x, logits and out.
+ */
+int moe_nvfp4_forward_host(const void* x_host, const float* logits_host, int64_t T,
+                           const moe_nvfp4_bank* bank, int32_t k, void* out_host, void* stream);
+
+/*
+ * Routing only (router + permutation), for inspection:
+ *  ids_dev [T, k] int32 expert ids in rank order;   w_dev [T, k] f32 softmax weights;
+ *  counts_dev [E] int32;  offsets_dev [E+1] int32 exclusive prefix sum of counts;
+ *  perm_dev [T*k] int32: position p holds the routed row r = t*k + j, expert by expert,
+ *           ascending r inside an expert;   inv_dev [T*k] int32 with perm[inv[r]] = r.
+ * Ranking key: larger logit first, ties to the lower index, -0.0 equal to +0.0, NaN below
+ * -inf.  Scratch comes from the internal workspace.
+ */
+int moe_nvfp4_route(const float* logits_dev, int64_t T, int32_t E, int32_t k, int32_t* ids_dev,
+                    float* w_dev, int32_t* counts_dev, int32_t* offsets_dev, int32_t* perm_dev,
+                    int32_t* inv_dev, void* stream);
+
+/* Bytes of caller workspace moe_nvfp4_forward_ex needs for these sizes and path (AUTO
+ * gives the size of the path AUTO would take).  Returns 0 for invalid sizes. */
+size_t moe_nvfp4_workspace_bytes(int64_t T, int32_t E, int32_t k, int32_t H, int32_t I,
+                                 int32_t path);
+
+/* Message for the last non-OK status returned to the calling host thread ("" if none). */
+const char* moe_nvfp4_last_error(void);
+
+/*
+ * Reads and clears the current device's sticky kernel status (synchronises the device):
+ * MOE_NVFP4_OK, or MOE_NVFP4_ERR_TIMEOUT if a bounded wait inside a kernel gave up since the
+ * last call.  A timeout means the kernel returned early and its outputs are invalid.
+ */
+int moe_nvfp4_device_status(void);
+
+/* Number of kernels the last successful compute call on this host thread enqueued. */
+int moe_nvfp4_last_launch_count(void);
+
+/* Kernel kinds reported by moe_nvfp4_profile_end. */
+#define MOE_NVFP4_KERNEL_ROUTE          0  /* router + permutation (1 or 3 kernels)   */
+#define MOE_NVFP4_KERNEL_DECODE_GATEUP  1
+#define MOE_NVFP4_KERNEL_DECODE_DOWN    2
+#define MOE_NVFP4_KERNEL_COMBINE        3
+#define MOE_NVFP4_KERNEL_PREFILL_GATHER 4
+#define MOE_NVFP4_KERNEL_PREFILL_GATEUP 5
+#define MOE_NVFP4_KERNEL_PREFILL_DOWN   6
+#define MOE_NVFP4_KERNEL_KINDS          8
+
+/*
+ * Kernel timing for benchmarks.  Between moe_nvfp4_profile_begin() and
+ * moe_nvfp4_profile_end(), every kernel kind a compute call launches on the calling host
+ * thread is bracketed by two CUDA events recorded on the call's stream (also while the stream
+ * is capturing into a CUDA graph: the events become event-record nodes and hold the times of
+ * the graph's latest replay).  moe_nvfp4_profile_end() synchronises on the events and writes,
+ * for each kind, the summed milliseconds into ms[kind] and the number of bracketed launches
+ * into launches[kind], for kinds < n; both arrays are caller-owned host memory.
+ */
+int moe_nvfp4_profile_begin(void);
+int moe_nvfp4_profile_end(double* ms, int64_t* launches, int32_t n);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* MOE_NVFP4_H_ */

@@ -1,0 +1,60 @@
+// Internal launch interface between the C ABI (moe_nvfp4.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Routing outputs and scratch, all device pointers into one workspace.
+struct RouteBufs {
+  int32_t* ids;        // [T, k]
+  float* w;            // [T, k]
+  int32_t* counts;     // [E]
+  int32_t* offsets;    // [E + 1]
+  int32_t* perm;       // [T * k]
+  int32_t* inv;        // [T * k]
+  int4* groups;        // [max_groups]: (expert, first permuted row, rows, 0)
+  int32_t* ngroups;    // [1]
+  int32_t* chunk_counts;  // [nchunks, E] (multi-CTA routing only)
+  int group_rows;      // rows per group (decode token tile)
+};
+
+// Tokens per routing chunk in the multi-CTA router; one CTA routes T <= this on its own.
+constexpr int kRouteChunk = 64;
+
+inline int route_chunks(int64_t T) { return (int)((T + kRouteChunk - 1) / kRouteChunk); }
+inline int64_t max_groups(int64_t R, int E, int group_rows) {
+  int64_t g = (R + group_rows - 1) / group_rows + E;
+  return g < R ? g : R;
+}
+
+// Launches the router and the permutation; returns the number of kernels launched or a
+// negative cudaError_t.
+int launch_route(const float* logits, int64_t T, int E, int k, const RouteBufs& b,
+                 cudaStream_t s);
+
+struct BankView {
+  const uint8_t* base;
+  uint64_t stride;
+  uint64_t codes_off[3], scales_off[3], global_off[3];
+  int global_mode;
+  int E, H, I;
+};
+
+// Decode path: grouped NVFP4 GEMV/GEMM on mma.sync with TMA bulk staging.
+// gate/up: h [R, I] f32 = silu(x Wg^T gg) * (x Wu^T gu) for every routed row.
+int launch_decode_gateup(const BankView& bank, const uint16_t* x, int k, const RouteBufs& rb,
+                         int xrows, float* h, int num_sms, cudaStream_t s);
+// down: y [R, H] f32 = h Wd^T gd for every routed row.
+int launch_decode_down(const BankView& bank, const float* h, const RouteBufs& rb, int xrows,
+                       float* y, int num_sms, cudaStream_t s);
+
+// out [T, H] bf16 = sum_j w[t, j] * y[inv[t*k+j]]; optional x_next = bf16(x + out).
+int launch_combine(const float* y, const float* w, const int32_t* inv, int64_t T, int k, int H,
+                   const uint16_t* x, uint16_t* out, uint16_t* x_next, cudaStream_t s);
+
+size_t decode_smem_bytes(int K, int xrows, bool gateup);
+
+}  // namespace moe

@@ -1,0 +1,473 @@
+// C ABI of the NVFP4 weight-only routed-expert MoE layer: host-side validation, workspace
+// management and the launch sequence (route -> expert GEMMs -> combine).
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+#include "moe_nvfp4.h"
+
+namespace {
+
+thread_local std::string t_last_error;
+thread_local int t_last_launches = 0;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(MOE_NVFP4_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0;
+  int smem_optin = 0;
+};
+
+std::mutex g_mu;
+std::vector<DeviceInfo> g_info;
+
+struct Workspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+std::vector<Workspace> g_ws;
+
+struct HostStage {
+  void* x = nullptr;
+  void* logits = nullptr;
+  void* out = nullptr;
+  size_t x_bytes = 0, logits_bytes = 0, out_bytes = 0;
+};
+std::vector<HostStage> g_stage;
+
+int current_device(int* dev, DeviceInfo* info) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return fail(MOE_NVFP4_ERR_UNSUPPORTED, "no CUDA device: %s", cudaGetErrorString(e));
+  std::lock_guard<std::mutex> lk(g_mu);
+  if ((int)g_info.size() <= *dev) {
+    g_info.resize(*dev + 1);
+    g_ws.resize(*dev + 1);
+    g_stage.resize(*dev + 1);
+  }
+  DeviceInfo& d = g_info[*dev];
+  if (d.sms == 0) {
+    cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, *dev);
+    cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, *dev);
+    cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, *dev);
+  }
+  *info = d;
+  if (d.major != 10)
+    return fail(MOE_NVFP4_ERR_UNSUPPORTED, "device %d has compute capability %d.x; this library needs sm_100",
+                *dev, d.major);
+  return MOE_NVFP4_OK;
+}
+
+// Sizes of the workspace sub-buffers, each 256-byte aligned.
+struct WsLayout {
+  size_t ids, w, counts, offsets, perm, inv, groups, ngroups, chunk_counts, h, y, total;
+};
+
+size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+WsLayout ws_layout(int64_t T, int E, int k, int H, int I, int path) {
+  (void)path;
+  WsLayout L{};
+  const size_t R = (size_t)T * k;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o += up256(bytes);
+    return at;
+  };
+  L.ids = take(R * 4);
+  L.w = take(R * 4);
+  L.counts = take((size_t)E * 4);
+  L.offsets = take((size_t)(E + 1) * 4);
+  L.perm = take(R * 4);
+  L.inv = take(R * 4);
+  L.groups = take((size_t)moe::max_groups((int64_t)R, E, 8) * 16);
+  L.ngroups = take(4);
+  L.chunk_counts = take(T > moe::kRouteChunk ? (size_t)moe::route_chunks(T) * E * 4 : 0);
+  L.h = take(R * (size_t)I * 4);
+  L.y = take(R * (size_t)H * 4);
+  L.total = o;
+  return L;
+}
+
+int check_bank(const moe_nvfp4_bank* b) {
+  if (!b) return fail(MOE_NVFP4_ERR_INVALID_ARG, "bank is NULL");
+  if (!b->base_dev) return fail(MOE_NVFP4_ERR_INVALID_ARG, "bank->base_dev is NULL");
+  if (b->num_experts < 1 || b->num_experts > 1024)
+    return fail(MOE_NVFP4_ERR_UNSUPPORTED, "num_experts %d outside 1..1024", b->num_experts);
+  if (b->hidden < 128 || b->hidden % 128 || b->intermediate < 128 || b->intermediate % 128)
+    return fail(MOE_NVFP4_ERR_UNSUPPORTED, "hidden %d and intermediate %d must be positive multiples of 128",
+                b->hidden, b->intermediate);
+  if (b->hidden > 8192 || b->intermediate > 8192)
+    return fail(MOE_NVFP4_ERR_UNSUPPORTED, "hidden and intermediate are limited to 8192");
+  if (b->global_mode != 0 && b->global_mode != 1)
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "global_mode %d is not 0 or 1", b->global_mode);
+  if (!aligned(b->base_dev, 16) || b->record_stride % 16)
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "bank base and record_stride must be 16-byte aligned");
+  const uint64_t H = b->hidden, I = b->intermediate;
+  for (int p = 0; p < 3; ++p) {
+    if (b->codes_off[p] % 16 || b->scales_off[p] % 16 || b->global_off[p] % 4)
+      return fail(MOE_NVFP4_ERR_INVALID_ARG, "projection %d offsets misaligned (codes/scales 16 B, global 4 B)", p);
+    if (b->codes_off[p] + H * I / 2 > b->record_stride || b->scales_off[p] + H * I / 16 > b->record_stride ||
+        b->global_off[p] + 4 > b->record_stride)
+      return fail(MOE_NVFP4_ERR_INVALID_ARG, "projection %d does not fit in record_stride", p);
+  }
+  return MOE_NVFP4_OK;
+}
+
+moe::BankView view_of(const moe_nvfp4_bank* b) {
+  moe::BankView v;
+  v.base = static_cast<const uint8_t*>(b->base_dev);
+  v.stride = b->record_stride;
+  for (int p = 0; p < 3; ++p) {
+    v.codes_off[p] = b->codes_off[p];
+    v.scales_off[p] = b->scales_off[p];
+    v.global_off[p] = b->global_off[p];
+  }
+  v.global_mode = b->global_mode;
+  v.E = b->num_experts;
+  v.H = b->hidden;
+  v.I = b->intermediate;
+  return v;
+}
+
+bool sync_each_kernel() {
+  static const bool on = [] {
+    const char* s = getenv("MOE_NVFP4_SYNC");
+    return s && s[0] == '1';
+  }();
+  return on;
+}
+
+// Per-thread kernel timing (moe_nvfp4_profile_begin / _end).
+struct ProfPair {
+  int kind;
+  cudaEvent_t a, b;
+};
+thread_local bool t_prof_on = false;
+thread_local std::vector<ProfPair> t_prof;
+
+cudaEvent_t prof_event() {
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+void prof_before(int kind, cudaStream_t s) {
+  if (!t_prof_on) return;
+  ProfPair p{kind, prof_event(), prof_event()};
+  cudaEventRecord(p.a, s);
+  t_prof.push_back(p);
+}
+
+void prof_after(cudaStream_t s) {
+  if (!t_prof_on || t_prof.empty()) return;
+  cudaEventRecord(t_prof.back().b, s);
+}
+
+int after_launch(int rc, cudaStream_t s, const char* what, int* count) {
+  prof_after(s);
+  if (rc < 0) return cuda_fail((cudaError_t)(-rc), what);
+  *count += rc;
+  if (sync_each_kernel()) {
+    const cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+  }
+  return MOE_NVFP4_OK;
+}
+
+// Makes sure the internal workspace of `dev` holds `bytes`.
+int ensure_workspace(int dev, size_t bytes, cudaStream_t s, void** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_ws[dev];
+  if (w.bytes < bytes) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(s, &cs);
+    if (cs != cudaStreamCaptureStatusNone)
+      return fail(MOE_NVFP4_ERR_WORKSPACE,
+                  "internal workspace must grow to %zu bytes while the stream is capturing; run once "
+                  "outside capture or pass a workspace",
+                  bytes);
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "synchronise before workspace growth");
+    if (w.ptr) cudaFree(w.ptr);
+    w.ptr = nullptr;
+    w.bytes = 0;
+    e = cudaMalloc(&w.ptr, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "workspace allocation");
+    w.bytes = bytes;
+  }
+  *out = w.ptr;
+  return MOE_NVFP4_OK;
+}
+
+moe::RouteBufs route_bufs(uint8_t* ws, const WsLayout& L) {
+  moe::RouteBufs b;
+  b.ids = reinterpret_cast<int32_t*>(ws + L.ids);
+  b.w = reinterpret_cast<float*>(ws + L.w);
+  b.counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  b.offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  b.perm = reinterpret_cast<int32_t*>(ws + L.perm);
+  b.inv = reinterpret_cast<int32_t*>(ws + L.inv);
+  b.groups = reinterpret_cast<int4*>(ws + L.groups);
+  b.ngroups = reinterpret_cast<int32_t*>(ws + L.ngroups);
+  b.chunk_counts = reinterpret_cast<int32_t*>(ws + L.chunk_counts);
+  b.group_rows = 8;
+  return b;
+}
+
+int check_k_T(int64_t T, int E, int k) {
+  if (T < 0) return fail(MOE_NVFP4_ERR_INVALID_ARG, "T = %lld is negative", (long long)T);
+  if (k < 1 || k > 32 || k > E) return fail(MOE_NVFP4_ERR_INVALID_ARG, "k = %d outside 1..min(E=%d, 32)", k, E);
+  if (T > ((int64_t)1 << 31) / 32) return fail(MOE_NVFP4_ERR_UNSUPPORTED, "T = %lld too large", (long long)T);
+  return MOE_NVFP4_OK;
+}
+
+int resolve_path(int path, int64_t T, int k, int E) {
+  if (path == MOE_NVFP4_PATH_AUTO) return MOE_NVFP4_PATH_DECODE;
+  (void)T;
+  (void)k;
+  (void)E;
+  return path;
+}
+
+int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_bank* bank, int32_t k,
+                 void* out, void* x_next, void* workspace, size_t workspace_bytes, int32_t path,
+                 void* stream) {
+  t_last_launches = 0;
+  int rc = check_bank(bank);
+  if (rc) return rc;
+  const int E = bank->num_experts, H = bank->hidden, I = bank->intermediate;
+  if ((rc = check_k_T(T, E, k))) return rc;
+  if (path < MOE_NVFP4_PATH_AUTO || path > MOE_NVFP4_PATH_PREFILL)
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "path %d unknown", path);
+  int dev;
+  DeviceInfo info;
+  if ((rc = current_device(&dev, &info))) return rc;
+  if (T == 0) return MOE_NVFP4_OK;
+  if (!x || !logits || !out) return fail(MOE_NVFP4_ERR_INVALID_ARG, "x, logits and out must not be NULL");
+  if (!aligned(x, 16) || !aligned(logits, 16) || !aligned(out, 16) || (x_next && !aligned(x_next, 16)))
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "x, logits, out and x_next must be 16-byte aligned");
+  const int use = resolve_path(path, T, k, E);
+  if (use == MOE_NVFP4_PATH_PREFILL)
+    return fail(MOE_NVFP4_ERR_UNSUPPORTED, "prefill path not available in this build");
+  const int xrows = (int)(T < 8 ? T : 8);
+  if (moe::decode_smem_bytes(H, xrows, true) == 0 || moe::decode_smem_bytes(I, xrows, false) == 0 ||
+      (int)moe::decode_smem_bytes(H, xrows, true) > info.smem_optin)
+    return fail(MOE_NVFP4_ERR_UNSUPPORTED, "H=%d / I=%d exceed the decode kernel's shared memory", H, I);
+
+  const WsLayout L = ws_layout(T, E, k, H, I, use);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  if (ws) {
+    if (workspace_bytes < L.total)
+      return fail(MOE_NVFP4_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes,
+                  L.total);
+    if (!aligned(ws, 256)) return fail(MOE_NVFP4_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  } else if ((rc = ensure_workspace(dev, L.total, s, &ws))) {
+    return rc;
+  }
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  const moe::RouteBufs rb = route_bufs(w8, L);
+  const moe::BankView bv = view_of(bank);
+  float* h = reinterpret_cast<float*>(w8 + L.h);
+  float* y = reinterpret_cast<float*>(w8 + L.y);
+  int launches = 0;
+  prof_before(MOE_NVFP4_KERNEL_ROUTE, s);
+  if ((rc = after_launch(moe::launch_route(logits, T, E, k, rb, s), s, "route", &launches))) return rc;
+  prof_before(MOE_NVFP4_KERNEL_DECODE_GATEUP, s);
+  if ((rc = after_launch(moe::launch_decode_gateup(bv, static_cast<const uint16_t*>(x), k, rb, xrows, h,
+                                                   info.sms, s),
+                         s, "decode gate/up", &launches)))
+    return rc;
+  prof_before(MOE_NVFP4_KERNEL_DECODE_DOWN, s);
+  if ((rc = after_launch(moe::launch_decode_down(bv, h, rb, xrows, y, info.sms, s), s, "decode down",
+                         &launches)))
+    return rc;
+  prof_before(MOE_NVFP4_KERNEL_COMBINE, s);
+  if ((rc = after_launch(moe::launch_combine(y, rb.w, rb.inv, T, k, H, static_cast<const uint16_t*>(x),
+                                             static_cast<uint16_t*>(out), static_cast<uint16_t*>(x_next), s),
+                         s, "combine", &launches)))
+    return rc;
+  t_last_launches = launches;
+  return MOE_NVFP4_OK;
+}
+
+int ensure_stage(void** p, size_t* have, size_t need) {
+  if (*have >= need) return MOE_NVFP4_OK;
+  if (*p) cudaFree(*p);
+  *p = nullptr;
+  *have = 0;
+  const cudaError_t e = cudaMalloc(p, need);
+  if (e != cudaSuccess) return cuda_fail(e, "staging allocation");
+  *have = need;
+  return MOE_NVFP4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_nvfp4_forward(const void* x_dev, const float* logits_dev, int64_t T, const moe_nvfp4_bank* bank, int32_t k,
+                      void* out_dev, void* stream) {
+  return forward_impl(x_dev, logits_dev, T, bank, k, out_dev, nullptr, nullptr, 0, MOE_NVFP4_PATH_AUTO, stream);
+}
+
+int moe_nvfp4_forward_ex(const void* x_dev, const float* logits_dev, int64_t T, const moe_nvfp4_bank* bank,
+                         int32_t k, void* out_dev, void* x_next_dev, void* workspace_dev, size_t workspace_bytes,
+                         int32_t path, void* stream) {
+  return forward_impl(x_dev, logits_dev, T, bank, k, out_dev, x_next_dev, workspace_dev, workspace_bytes, path,
+                      stream);
+}
+
+int moe_nvfp4_forward_host(const void* x_host, const float* logits_host, int64_t T, const moe_nvfp4_bank* bank,
+                           int32_t k, void* out_host, void* stream) {
+  int rc = check_bank(bank);
+  if (rc) return rc;
+  if ((rc = check_k_T(T, bank->num_experts, k))) return rc;
+  int dev;
+  DeviceInfo info;
+  if ((rc = current_device(&dev, &info))) return rc;
+  if (T == 0) return MOE_NVFP4_OK;
+  if (!x_host || !logits_host || !out_host)
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "x_host, logits_host and out_host must not be NULL");
+  const size_t xb = (size_t)T * bank->hidden * 2, lb = (size_t)T * bank->num_experts * 4;
+  HostStage* st;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    st = &g_stage[dev];
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (xb > st->x_bytes || lb > st->logits_bytes || xb > st->out_bytes) {
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "synchronise before staging growth");
+    if ((rc = ensure_stage(&st->x, &st->x_bytes, xb))) return rc;
+    if ((rc = ensure_stage(&st->logits, &st->logits_bytes, lb))) return rc;
+    if ((rc = ensure_stage(&st->out, &st->out_bytes, xb))) return rc;
+  }
+  cudaError_t e = cudaMemcpyAsync(st->x, x_host, xb, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copy x to device");
+  e = cudaMemcpyAsync(st->logits, logits_host, lb, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copy logits to device");
+  rc = forward_impl(st->x, static_cast<const float*>(st->logits), T, bank, k, st->out, nullptr, nullptr, 0,
+                    MOE_NVFP4_PATH_AUTO, stream);
+  if (rc) return rc;
+  e = cudaMemcpyAsync(out_host, st->out, xb, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copy out to host");
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "synchronise");
+  return MOE_NVFP4_OK;
+}
+
+int moe_nvfp4_route(const float* logits_dev, int64_t T, int32_t E, int32_t k, int32_t* ids_dev, float* w_dev,
+                    int32_t* counts_dev, int32_t* offsets_dev, int32_t* perm_dev, int32_t* inv_dev, void* stream) {
+  t_last_launches = 0;
+  if (E < 1 || E > 1024) return fail(MOE_NVFP4_ERR_UNSUPPORTED, "E = %d outside 1..1024", E);
+  int rc = check_k_T(T, E, k);
+  if (rc) return rc;
+  int dev;
+  DeviceInfo info;
+  if ((rc = current_device(&dev, &info))) return rc;
+  if (!counts_dev || !offsets_dev) return fail(MOE_NVFP4_ERR_INVALID_ARG, "counts and offsets must not be NULL");
+  if (T > 0 && (!logits_dev || !ids_dev || !w_dev || !perm_dev || !inv_dev))
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "logits, ids, w, perm and inv must not be NULL");
+  const WsLayout L = ws_layout(T, E, k, 128, 128, MOE_NVFP4_PATH_DECODE);
+  const size_t need = L.h;  // routing part only
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws;
+  if ((rc = ensure_workspace(dev, need, s, &ws))) return rc;
+  moe::RouteBufs rb = route_bufs(static_cast<uint8_t*>(ws), L);
+  rb.ids = ids_dev;
+  rb.w = w_dev;
+  rb.counts = counts_dev;
+  rb.offsets = offsets_dev;
+  rb.perm = perm_dev;
+  rb.inv = inv_dev;
+  if (T == 0) {
+    cudaError_t e = cudaMemsetAsync(counts_dev, 0, (size_t)E * 4, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(offsets_dev, 0, (size_t)(E + 1) * 4, s);
+    return e == cudaSuccess ? MOE_NVFP4_OK : cuda_fail(e, "clear counts");
+  }
+  int launches = 0;
+  if ((rc = after_launch(moe::launch_route(logits_dev, T, E, k, rb, s), s, "route", &launches))) return rc;
+  t_last_launches = launches;
+  return MOE_NVFP4_OK;
+}
+
+size_t moe_nvfp4_workspace_bytes(int64_t T, int32_t E, int32_t k, int32_t H, int32_t I, int32_t path) {
+  if (T < 0 || E < 1 || E > 1024 || k < 1 || k > 32 || k > E || H < 128 || I < 128) return 0;
+  return ws_layout(T, E, k, H, I, resolve_path(path, T, k, E)).total;
+}
+
+const char* moe_nvfp4_last_error(void) { return t_last_error.c_str(); }
+
+int moe_nvfp4_device_status(void) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, moe::g_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read device status");
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(moe::g_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "clear device status");
+  if (v != 0) return fail(MOE_NVFP4_ERR_TIMEOUT, "a bounded device wait gave up (status %d)", v);
+  return MOE_NVFP4_OK;
+}
+
+int moe_nvfp4_last_launch_count(void) { return t_last_launches; }
+
+int moe_nvfp4_profile_begin(void) {
+  for (auto& p : t_prof) {
+    cudaEventDestroy(p.a);
+    cudaEventDestroy(p.b);
+  }
+  t_prof.clear();
+  t_prof_on = true;
+  return MOE_NVFP4_OK;
+}
+
+int moe_nvfp4_profile_end(double* ms, int64_t* launches, int32_t n) {
+  t_prof_on = false;
+  if ((!ms || !launches) && n > 0) return fail(MOE_NVFP4_ERR_INVALID_ARG, "ms and launches must not be NULL");
+  for (int i = 0; i < n; ++i) {
+    ms[i] = 0.0;
+    launches[i] = 0;
+  }
+  int rc = MOE_NVFP4_OK;
+  for (auto& p : t_prof) {
+    float t = 0.0f;
+    cudaError_t e = cudaEventSynchronize(p.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, p.a, p.b);
+    if (e != cudaSuccess && rc == MOE_NVFP4_OK) rc = cuda_fail(e, "profile event");
+    if (p.kind < n) {
+      ms[p.kind] += t;
+      launches[p.kind] += 1;
+    }
+    cudaEventDestroy(p.a);
+    cudaEventDestroy(p.b);
+  }
+  t_prof.clear();
+  return rc;
+}
+
+}  // extern "C"

@@ -1,0 +1,259 @@
+// Router (top-k + softmax over the selected logits) and token permutation.
+//
+// Method statement: top-k over the F32 router logits with warp-level selection, ties to the
+// lower expert index, softmax over the k selected logits; then a per-expert histogram, the
+// exclusive prefix sum of the counts, and a stable placement of the routed rows expert by
+// expert.  Page "Beam 1.0 501B-A23B, streaming pack, NVFP4 experts / MLX 8-bit residents",
+// section "What this pack holds" (256 routed experts, 8 active per token); page
+// "Beam-1.0-501B-A23B VQ GGUF", section "What stays native" (router logits in FP32).
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr unsigned kFull = 0xFFFFFFFFu;
+constexpr int kMaxE = 1024;
+constexpr int kMaxPerLane = kMaxE / 32;
+
+// Order-preserving key of a logit: larger logit -> larger key; -0.0 == +0.0; NaN lowest (0).
+__device__ __forceinline__ uint32_t rank_key(float v) {
+  uint32_t b = __float_as_uint(v);
+  if (v != v) return 0u;
+  if ((b << 1) == 0u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// One warp selects the top k (k <= 32) of a row of E (<= 1024) logits.  Lane j < k gets the
+// rank-j expert and its softmax weight.  Keys combine the logit key with the complemented
+// index so that a larger combined key is a higher rank (ties to the lower index).
+template <int PER_LANE>
+__device__ void warp_route_row(const float* __restrict__ row, int E, int k, int lane, int& id,
+                               float& weight) {
+  uint64_t key[PER_LANE];
+  uint64_t best = 0;
+#pragma unroll
+  for (int i = 0; i < PER_LANE; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = 0;
+    if (e < E) key[i] = ((uint64_t)rank_key(__ldg(row + e)) << 32) | (uint32_t)(0xFFFFFFFFu - e);
+    best = key[i] > best ? key[i] : best;
+  }
+  id = 0;
+  for (int r = 0; r < k; ++r) {
+    uint64_t m = best;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const uint64_t o = __shfl_xor_sync(kFull, m, off);
+      m = o > m ? o : m;
+    }
+    const int e = (int)(0xFFFFFFFFu - (uint32_t)m);
+    if (lane == r) id = e;
+    if (lane == (e & 31)) {
+      const int slot = e >> 5;
+      best = 0;
+#pragma unroll
+      for (int i = 0; i < PER_LANE; ++i) {
+        if (i == slot) key[i] = 0;
+        best = key[i] > best ? key[i] : best;
+      }
+    }
+  }
+  const float l = lane < k ? __ldg(row + id) : 0.0f;
+  const float lmax = __shfl_sync(kFull, l, 0);
+  float ex = lane < k ? expf(l - lmax) : 0.0f;
+  float sum = ex;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
+  weight = ex / sum;
+}
+
+__device__ void route_row(const float* row, int E, int k, int lane, int& id, float& w) {
+  if (E <= 32 * 8)
+    warp_route_row<8>(row, E, k, lane, id, w);
+  else
+    warp_route_row<kMaxPerLane>(row, E, k, lane, id, w);
+}
+
+// Exclusive scan of n ints in shared memory (in place) by the whole block; returns the total.
+__device__ int block_scan_excl(int* a, int n, int* warp_tmp) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int per = (n + nt - 1) / nt;
+  const int lo = tid * per, hi = min(n, lo + per);
+  int s = 0;
+  for (int i = lo; i < hi; ++i) s += a[i];
+  // inclusive warp scan of s
+  const int lane = tid & 31, wid = tid >> 5, nw = (nt + 31) >> 5;
+  int v = s;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(kFull, v, off);
+    if (lane >= off) v += o;
+  }
+  if (lane == 31) warp_tmp[wid] = v;
+  __syncthreads();
+  if (wid == 0) {
+    int t = lane < nw ? warp_tmp[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(kFull, t, off);
+      if (lane >= off) t += o;
+    }
+    if (lane < nw) warp_tmp[lane] = t;  // inclusive prefix over warps
+  }
+  __syncthreads();
+  int run = v - s + (wid > 0 ? warp_tmp[wid - 1] : 0);  // exclusive prefix of this thread
+  const int total = warp_tmp[nw - 1];
+  for (int i = lo; i < hi; ++i) {
+    const int c = a[i];
+    a[i] = run;
+    run += c;
+  }
+  __syncthreads();
+  return total;
+}
+
+// From per-expert counts in shared memory: offsets, group list and group count.
+__device__ void finish_counts(int* cnt, int* tmp, int* warp_tmp, int E, int group_rows,
+                              const RouteBufs& b) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    b.counts[e] = cnt[e];
+    tmp[e] = (cnt[e] + group_rows - 1) / group_rows;
+  }
+  __syncthreads();
+  const int ng = block_scan_excl(tmp, E, warp_tmp);         // tmp: first group of expert e
+  // cnt -> offsets (in place)
+  const int R = block_scan_excl(cnt, E, warp_tmp);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    b.offsets[e] = cnt[e];
+    const int c = b.counts[e];
+    for (int q = 0, g = tmp[e]; q * group_rows < c; ++q, ++g)
+      b.groups[g] = make_int4(e, cnt[e] + q * group_rows, min(group_rows, c - q * group_rows), 0);
+  }
+  if (threadIdx.x == 0) {
+    b.offsets[E] = R;
+    *b.ngroups = ng;
+  }
+}
+
+// Single-CTA routing for T <= kRouteChunk: router, histogram, scan, groups, stable scatter.
+__global__ void __launch_bounds__(512) route_small_kernel(const float* __restrict__ logits,
+                                                          int T, int E, int k, RouteBufs b) {
+  __shared__ int cnt[kMaxE], tmp[kMaxE], run[kMaxE], warp_tmp[32];
+  __shared__ int sids[kRouteChunk * 32];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int t = wid; t < T; t += nw) {
+    int id;
+    float w;
+    route_row(logits + (size_t)t * E, E, k, lane, id, w);
+    if (lane < k) {
+      b.ids[t * k + lane] = id;
+      b.w[t * k + lane] = w;
+      sids[t * k + lane] = id;
+      atomicAdd(&cnt[id], 1);
+    }
+  }
+  __syncthreads();
+  finish_counts(cnt, tmp, warp_tmp, E, b.group_rows, b);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) run[e] = cnt[e];   // cnt now = offsets
+  __syncthreads();
+  if (wid == 0) {
+    for (int t = 0; t < T; ++t) {
+      if (lane < k) {
+        const int r = t * k + lane, e = sids[r];
+        const int pos = run[e];
+        run[e] = pos + 1;
+        b.perm[pos] = r;
+        b.inv[r] = pos;
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// Multi-CTA routing, step 1: route the chunk's tokens and count its rows per expert.
+__global__ void __launch_bounds__(256) route_chunk_kernel(const float* __restrict__ logits,
+                                                          int64_t T, int E, int k, RouteBufs b) {
+  __shared__ int cnt[kMaxE];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int64_t t0 = (int64_t)blockIdx.x * kRouteChunk;
+  const int nt = (int)(T - t0 < kRouteChunk ? T - t0 : kRouteChunk);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int i = wid; i < nt; i += nw) {
+    const int64_t t = t0 + i;
+    int id;
+    float w;
+    route_row(logits + t * E, E, k, lane, id, w);
+    if (lane < k) {
+      b.ids[t * k + lane] = id;
+      b.w[t * k + lane] = w;
+      atomicAdd(&cnt[id], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    b.chunk_counts[(size_t)blockIdx.x * E + e] = cnt[e];
+}
+
+// Multi-CTA routing, step 2 (one CTA): per-expert prefix over chunks, counts, offsets, groups.
+__global__ void __launch_bounds__(1024) route_scan_kernel(int nchunks, int E, RouteBufs b) {
+  __shared__ int cnt[kMaxE], tmp[kMaxE], warp_tmp[32];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int c = 0; c < nchunks; ++c) {
+      int* p = b.chunk_counts + (size_t)c * E + e;
+      const int v = *p;
+      *p = run;
+      run += v;
+    }
+    cnt[e] = run;
+  }
+  __syncthreads();
+  finish_counts(cnt, tmp, warp_tmp, E, b.group_rows, b);
+}
+
+// Multi-CTA routing, step 3: stable placement of the chunk's rows.
+__global__ void __launch_bounds__(32) route_scatter_kernel(int64_t T, int E, int k, RouteBufs b) {
+  __shared__ int run[kMaxE];
+  const int lane = threadIdx.x;
+  const int64_t t0 = (int64_t)blockIdx.x * kRouteChunk;
+  const int nt = (int)(T - t0 < kRouteChunk ? T - t0 : kRouteChunk);
+  for (int e = lane; e < E; e += 32)
+    run[e] = b.offsets[e] + b.chunk_counts[(size_t)blockIdx.x * E + e];
+  __syncwarp();
+  for (int i = 0; i < nt; ++i) {
+    if (lane < k) {
+      const int64_t r = (t0 + i) * k + lane;
+      const int e = b.ids[r];
+      const int pos = run[e];
+      run[e] = pos + 1;
+      b.perm[pos] = (int32_t)r;
+      b.inv[r] = pos;
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace
+
+int launch_route(const float* logits, int64_t T, int E, int k, const RouteBufs& b,
+                 cudaStream_t s) {
+  if (T <= kRouteChunk) {
+    route_small_kernel<<<1, 512, 0, s>>>(logits, (int)T, E, k, b);
+    const cudaError_t err = cudaGetLastError();
+    return err == cudaSuccess ? 1 : -(int)err;
+  }
+  const int nch = route_chunks(T);
+  route_chunk_kernel<<<nch, 256, 0, s>>>(logits, T, E, k, b);
+  route_scan_kernel<<<1, 1024, 0, s>>>(nch, E, b);
+  route_scatter_kernel<<<nch, 32, 0, s>>>(T, E, k, b);
+  const cudaError_t err = cudaGetLastError();
+  return err == cudaSuccess ? 3 : -(int)err;
+}
+
+}  // namespace moe

@@ -43,3 +43,4 @@ from .moe import (  # noqa: F401
     round_to_bf16_bits,
     residual_add,
 )
+from .sources import GeneratedRecords  # noqa: F401

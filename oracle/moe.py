@@ -101,14 +101,22 @@ def residual_add(x_bits: np.ndarray, out_bits: np.ndarray) -> np.ndarray:
     return round_to_bf16_bits(bf16_bits_to_f64(x_bits) + bf16_bits_to_f64(out_bits))
 
 
+def _expert_job(job):
+    get_weights, e, X = job
+    Wg, Wu, Wd = get_weights(e)
+    return expert_forward(Wg, Wu, Wd, X)
+
+
 def layer_forward(x_bits: np.ndarray, logits: np.ndarray, k: int, get_weights,
-                  tokens=None, want_rows: bool = False):
+                  tokens=None, want_rows: bool = False, map_fn=map):
     """One MoE layer.
 
     x_bits [T, H] BF16 bit patterns, logits [T, E] f32, get_weights(e) -> (Wg, Wu, Wd) FP64.
     tokens: optional list of token indices to evaluate (routing is always computed for all).
     Returns a dict with ids, w, counts, offsets, perm, inv and out [len(tokens), H] (FP64);
     with want_rows also y [len(tokens), k, H], the expert outputs before the combine.
+    map_fn maps the per-expert work (decode the record, run the expert on its rows); a process
+    pool's map spreads it over host cores without changing any arithmetic.
     """
     T, E = np.asarray(logits).shape
     ids, w = route(logits, k)
@@ -121,11 +129,10 @@ def layer_forward(x_bits: np.ndarray, logits: np.ndarray, k: int, get_weights,
     for ti, t in enumerate(toks):
         for j in range(k):
             by_expert.setdefault(int(ids[t, j]), []).append((ti, int(t), j))
-    for e in sorted(by_expert):
-        rows = by_expert[e]
-        Wg, Wu, Wd = get_weights(e)
-        Y = expert_forward(Wg, Wu, Wd, x[[t for (_, t, _) in rows]])
-        for r, (ti, _, j) in enumerate(rows):
+    experts = sorted(by_expert)
+    jobs = [(get_weights, e, x[[t for (_, t, _) in by_expert[e]]]) for e in experts]
+    for e, Y in zip(experts, map_fn(_expert_job, jobs)):
+        for r, (ti, _, j) in enumerate(by_expert[e]):
             y[ti, j] = Y[r]
     out = np.zeros((len(toks), H))
     for j in range(k):

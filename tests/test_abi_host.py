@@ -1,0 +1,95 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel launched).
+
+The library must load, export every entry point the header declares, and reject invalid
+arguments on the host before touching a device.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import moe_inputs
+from moe_inputs import device as mdev
+import nvfp4_weight_only_top_b200 as moe
+from nvfp4_weight_only_top_b200 import _abi
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe_nvfp4.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_nvfp4_\w+)\s*\(", src)))
+
+
+def test_header_declares_expected_entry_points():
+    names = _declared()
+    assert "moe_nvfp4_forward" in names and "moe_nvfp4_route" in names
+    assert set(names) == set(_abi.SIGNATURES), "binding signatures must cover the header exactly"
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(_abi.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    moe.lib()       # typed load succeeds
+
+
+def test_bank_struct_layout_matches_header():
+    assert ctypes.sizeof(_abi.Bank) == 4 * 4 + 8 + 8 + 3 * 8 * 3
+    assert _abi.Bank.base_dev.offset == 16 and _abi.Bank.codes_off.offset == 32
+
+
+def _bank(**kw):
+    lay = moe_inputs.record_layout(16, 256, 128)
+    args = dict(base_ptr=0x10000, num_experts=16, hidden=256, intermediate=128,
+                record_stride=lay.record_stride, codes_off=lay.codes_off, scales_off=lay.scales_off,
+                global_off=lay.global_off, global_mode=0)
+    args.update(kw)
+    return moe.make_bank(**args)
+
+
+def _fwd(bank, T=4, k=2, x=0x20000, lg=0x30000, out=0x40000):
+    lib = moe.lib()
+    return lib.moe_nvfp4_forward(ctypes.c_void_p(x), ctypes.c_void_p(lg), T,
+                                 ctypes.byref(bank) if bank is not None else None, k, ctypes.c_void_p(out), None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(num_experts=0), _abi.ERR_UNSUPPORTED),
+    (dict(num_experts=2048), _abi.ERR_UNSUPPORTED),
+    (dict(hidden=200), _abi.ERR_UNSUPPORTED),
+    (dict(intermediate=64), _abi.ERR_UNSUPPORTED),
+    (dict(global_mode=2), _abi.ERR_INVALID_ARG),
+    (dict(base_ptr=0x10008), _abi.ERR_INVALID_ARG),
+    (dict(record_stride=1000), _abi.ERR_INVALID_ARG),
+])
+def test_bank_validation(kw, code):
+    assert _fwd(_bank(**kw)) == code
+    assert moe.moe_nvfp4_last_error() != ""
+
+
+def test_null_bank_and_bad_k_and_T():
+    assert _fwd(None) == _abi.ERR_INVALID_ARG
+    assert _fwd(_bank(), k=0) == _abi.ERR_INVALID_ARG
+    assert _fwd(_bank(), k=17) == _abi.ERR_INVALID_ARG        # k > E
+    assert _fwd(_bank(), k=33) == _abi.ERR_INVALID_ARG
+    assert _fwd(_bank(), T=-1) == _abi.ERR_INVALID_ARG
+    assert "T = -1" in moe.moe_nvfp4_last_error()
+
+
+def test_workspace_bytes_is_host_only():
+    a = moe.moe_nvfp4_workspace_bytes(1, 256, 8, 5120, 2560)
+    b = moe.moe_nvfp4_workspace_bytes(64, 256, 8, 5120, 2560)
+    assert 0 < a < b
+    assert moe.moe_nvfp4_workspace_bytes(-1, 256, 8, 5120, 2560) == 0
+    assert moe.moe_nvfp4_workspace_bytes(1, 256, 0, 5120, 2560) == 0
+    # the h and y buffers dominate: R*(H+I)*4
+    assert b >= 64 * 8 * (5120 + 2560) * 4
+
+
+def test_input_generator_key_matches_native():
+    for args in [(0, 0, 0, 0), (7, 3, 255, 1), (123456789, 23, 17, 0)]:
+        assert mdev.stream_key_native(*args) == moe_inputs.gen.stream_key(*args)
