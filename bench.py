@@ -213,7 +213,8 @@ def main():
     steps = args.steps if args.steps is not None else DEFAULT_STEPS[cfg.name]
     warm = args.warmup if args.warmup is not None else max(3, min(200, steps // 10))
     lay = cfg.layout
-    s = torch.cuda.current_stream()
+    s = torch.cuda.Stream()          # graphs are captured on a non-default stream
+    torch.cuda.set_stream(s)
 
     # ---- resident inputs: banks (one per layer), activations, rotating router logits
     banks, bufs = [], []

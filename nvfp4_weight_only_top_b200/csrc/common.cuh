@@ -155,6 +155,9 @@ __device__ __forceinline__ void mma_16816(float c[4], const uint32_t a[4], uint3
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// SwiGLU of one pair: silu(g) * u = g / (1 + e^-g) * u, in f32.
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
 // Multiplier of a projection's stored global: mode 0 the value itself, mode 1 f32(g / 2688).
 __device__ __forceinline__ float global_mult(float g, int mode) {
   return mode == 1 ? __fdiv_rn(g, 2688.0f) : g;

@@ -1,22 +1,22 @@
 // Decode path: memory-bound grouped NVFP4 expert GEMV/GEMM.
 //
 // Work item = (group, row tile): a group is <= 8 routed rows of one expert (in permuted
-// order), a row tile is 16 MMA rows x the full input width K.  For gate/up the 16 MMA rows
-// are 8 gate rows and the same 8 up rows, so SwiGLU is applied in-thread in the epilogue;
-// for down they are 16 rows of Wd.
+// order); a row tile is 16 weight rows x the full input width K, one MMA M-tile.  For gate/up
+// the 16 rows are 8 gate rows and the same 8 up rows, so SwiGLU is applied in-thread in the
+// epilogue; for down they are 16 rows of Wd.
 //
-// One CTA per SM walks a contiguous range of items.  Warp kNW (the producer) streams each
-// tile's codes and scales into a ring of shared-memory stages with 1-D bulk copies (TMA),
-// one copy per weight row so that rows land at a padded pitch (conflict-free reads).  The
-// kNW consumer warps split K: warp w takes 128-wide K units w, w + kNW, ...  Each thread
-// dequantizes its codes in registers (E2M1 -> f16 by cvt, times the E4M3 block scale in
-// f16, both exact), and feeds mma.sync m16n8k16 with the weights as A (16 rows) and the
-// group's activations as B (N = 8 token slots, f32 accumulators).  Partial sums of the
-// warps are added through shared memory; the global scale and SwiGLU are applied in f32.
+// Two CTAs per SM, each walking a contiguous range of items.  The kNW warps of a CTA split K
+// into 128-wide units (warp w takes units w, w + kNW, ...).  A thread streams its share of
+// every unit straight from HBM with 128-bit loads into a 3-slot register ring (two units in
+// flight while it computes a third), dequantizes 2 rows x 32 codes in registers (E2M1 -> f16
+// by cvt, times the E4M3 block scale in f16: both exact) and issues 8 mma.sync m16n8k16 with
+// the weights as A and the group's activations (N = 8 token slots, staged once per group in
+// shared memory) as B, alternating between two accumulators.  The warps' partial sums are
+// added through shared memory in a fixed order; the global scale and SwiGLU follow in f32.
 //
-// Within one MMA the 16 logical k of a row come from four threads; thread tid4 supplies
-// K offsets 32*tid4 + 4*s .. +3 of the unit for k-step s, and the activations are staged
-// in shared memory in the matching order, so no data is shuffled between threads.
+// The MMA's 16 logical k of a row come from four threads: thread tid4 supplies 4 K values of
+// its own 32-wide slice of the unit per k-step, and the activations are staged in the same
+// order, so no data moves between threads.
 //
 // Weight layout: page "Beam 1.0 501B-A23B, streaming pack, NVFP4 experts / MLX 8-bit
 // residents", section "What this pack holds"; SwiGLU in FP32: page "Beam-1.0-501B-A23B VQ
@@ -30,11 +30,10 @@ __device__ int g_status = 0;
 
 namespace {
 
-constexpr int kNW = 10;                    // consumer warps
-constexpr int kThreads = 32 * (kNW + 1);   // + one producer warp
-constexpr int kTileRows = 16;
-constexpr int kMaxStages = 8;
-constexpr int kSmemLimit = 232448;         // 227 KB opt-in per block on sm_100
+constexpr int kNW = 10;                  // warps per CTA
+constexpr int kThreads = 32 * kNW;
+constexpr int kCtasPerSm = 2;
+constexpr int kSmemLimit = 113 * 1024;   // per CTA, two CTAs per SM
 
 struct DecodeParams {
   const uint8_t* bank;
@@ -43,44 +42,28 @@ struct DecodeParams {
   int global_mode;
   int K, N;       // inputs per weight row, output rows per matrix
   int k;          // routing top-k: routed row r belongs to token r / k
-  int stages;
   int xrows;      // activation rows staged per group (1 .. 8)
   const int4* groups;
   const int32_t* ngroups;
   const int32_t* perm;
   const void* xin;  // gate/up: bf16 x [T, K]; down: f32 h [R, K] (permuted rows)
-  float* out;       // [R, N] (permuted rows)
+  float* out;       // gate/up: h [R, N] = silu(G) * U; down: y [R, N] (permuted rows)
 };
 
-struct Layout {
-  int code_pitch, stage_codes, stage_bytes, xs_pitch, off_xs, off_red, off_bar, total;
-};
+__host__ __device__ inline int xs_pitch(int K) { return K * 2 + 64; }   // = 64 (mod 128)
+__host__ __device__ inline int off_red(int K, int xrows) { return (xrows * xs_pitch(K) + 127) & ~127; }
+__host__ __device__ inline int smem_total(int K, int xrows) { return off_red(K, xrows) + 2 * kNW * 32 * 16; }
 
-__host__ __device__ inline Layout make_layout(int K, int stages, int xrows) {
-  Layout L;
-  const int rowb = K / 2;
-  L.code_pitch = rowb + ((rowb % 128) == 0 ? 64 : 0);   // pitch = 64 (mod 128)
-  L.stage_codes = kTileRows * L.code_pitch;
-  L.stage_bytes = (L.stage_codes + kTileRows * (K / 16) + 127) & ~127;
-  L.xs_pitch = K * 2 + 64;                              // = 64 (mod 128)
-  L.off_xs = stages * L.stage_bytes;
-  L.off_red = L.off_xs + ((xrows * L.xs_pitch + 127) & ~127);
-  L.off_bar = L.off_red + 2 * kNW * 32 * 16;
-  L.total = L.off_bar + 2 * stages * 8;
-  return L;
-}
-
-// Stage the group's activations as f16 in the fragment order: inside each 128-wide K unit,
-// the 8 values K0 .. K0+7 with K0 = 32*t + 8*i go to 16-byte chunk 4*i + t.
+// Stage the group's activations as f16 in fragment order: inside each 128-wide K unit the 8
+// values K0 .. K0+7 with K0 = 32*t + 8*i go to 16-byte chunk 4*i + t.
 template <bool GATEUP>
-__device__ void fill_xs(const DecodeParams& p, const Layout& L, uint8_t* xs, int row0, int nrows,
-                        int ctid) {
+__device__ void fill_xs(const DecodeParams& p, uint8_t* xs, int row0, int nrows) {
   const int cpr = p.K / 8;  // chunks of 8 values per row
-  for (int c = ctid; c < p.xrows * cpr; c += kNW * 32) {
+  const int pitch = xs_pitch(p.K);
+  for (int c = threadIdx.x; c < p.xrows * cpr; c += kThreads) {
     const int n = c / cpr, kk = (c - n * cpr) * 8;
     const int u = kk >> 7, q = kk & 127;
-    uint4* dst = reinterpret_cast<uint4*>(xs + n * L.xs_pitch + u * 256 +
-                                          (((q & 31) >> 3) * 4 + (q >> 5)) * 16);
+    uint4* dst = reinterpret_cast<uint4*>(xs + n * pitch + u * 256 + (((q & 31) >> 3) * 4 + (q >> 5)) * 16);
     uint4 v = make_uint4(0, 0, 0, 0);
     if (n < nrows) {
       if (GATEUP) {
@@ -95,192 +78,208 @@ __device__ void fill_xs(const DecodeParams& p, const Layout& L, uint8_t* xs, int
         const float4* src = reinterpret_cast<const float4*>(
             static_cast<const float*>(p.xin) + (size_t)(row0 + n) * p.K + kk);
         const float4 a = src[0], b = src[1];
-        v.x = pack_f16x2(a.x, a.y);
-        v.y = pack_f16x2(a.z, a.w);
-        v.z = pack_f16x2(b.x, b.y);
-        v.w = pack_f16x2(b.z, b.w);
+        v = make_uint4(pack_f16x2(a.x, a.y), pack_f16x2(a.z, a.w), pack_f16x2(b.x, b.y), pack_f16x2(b.z, b.w));
       }
     }
     *dst = v;
   }
 }
 
+// One thread's share of one unit of one item: 16 code bytes and 2 scale bytes of each of the
+// MMA rows gid and gid + 8.
+struct Frag {
+  uint4 c0, c1;
+  uint32_t s0, s1;
+};
+
+// Walks the (item, unit) steps of one warp.  All warps take the same number of steps per
+// item (units beyond K are empty steps), so item boundaries line up across the CTA.
+struct Cursor {
+  int item, q, g, tile;
+  const uint8_t* rec;
+};
+
+__device__ __forceinline__ uint32_t ld_u16_nc(const uint8_t* p) {
+  uint16_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint4 ld_v4_stream(const uint8_t* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
 template <bool GATEUP>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  const Layout L = make_layout(p.K, p.stages, p.xrows);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.off_bar);
-  uint64_t* empty = full + p.stages;
+  uint8_t* xs = smem;
+  float4* red = reinterpret_cast<float4*>(smem + off_red(p.K, p.xrows));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tiles = GATEUP ? p.N / 8 : p.N / kTileRows;
+  const int gid = lane >> 2, tid4 = lane & 3;
+  const int tiles = GATEUP ? p.N / 8 : p.N / 16;
   const int items = *p.ngroups * tiles;
   const int per = items / (int)gridDim.x, rem = items % (int)gridDim.x;
   const int i0 = (int)blockIdx.x * per + min((int)blockIdx.x, rem);
   const int i1 = i0 + per + ((int)blockIdx.x < rem ? 1 : 0);
-  const uint32_t rowb = p.K / 2, scb = p.K / 16;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < p.stages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kNW);
-    }
-    fence_barrier_init();
-  }
-  __syncthreads();
-
-  if (warp == kNW) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      int issued = 0;
-      for (int it = i0; it < i1; ++it, ++issued) {
-        const int j = it - i0, s = j % p.stages;
-        const uint32_t ph = (j / p.stages) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1)) break;
-        const int g = it / tiles, tile = it - g * tiles;
-        const uint8_t* rec = p.bank + (uint64_t)p.groups[g].x * p.stride;
-        uint8_t* st = smem + s * L.stage_bytes;
-        mbar_arrive_expect_tx(&full[s], kTileRows * (rowb + scb));
-        if (GATEUP) {
-          const int n0 = tile * 8;
-          const uint8_t* gc = rec + p.codes_off[0] + (size_t)n0 * rowb;
-          const uint8_t* uc = rec + p.codes_off[1] + (size_t)n0 * rowb;
-#pragma unroll 1
-          for (int r = 0; r < 8; ++r) {
-            bulk_g2s(st + r * L.code_pitch, gc + (size_t)r * rowb, rowb, &full[s], pol);
-            bulk_g2s(st + (8 + r) * L.code_pitch, uc + (size_t)r * rowb, rowb, &full[s], pol);
-          }
-          bulk_g2s(st + L.stage_codes, rec + p.scales_off[0] + (size_t)n0 * scb, 8 * scb, &full[s], pol);
-          bulk_g2s(st + L.stage_codes + 8 * scb, rec + p.scales_off[1] + (size_t)n0 * scb, 8 * scb,
-                   &full[s], pol);
-        } else {
-          const int n0 = tile * kTileRows;
-          const uint8_t* dc = rec + p.codes_off[0] + (size_t)n0 * rowb;
-#pragma unroll 1
-          for (int r = 0; r < kTileRows; ++r)
-            bulk_g2s(st + r * L.code_pitch, dc + (size_t)r * rowb, rowb, &full[s], pol);
-          bulk_g2s(st + L.stage_codes, rec + p.scales_off[0] + (size_t)n0 * scb, kTileRows * scb,
-                   &full[s], pol);
-        }
-      }
-      // Do not leave while copies may still be landing (matters only on the error path).
-      for (int j = max(0, issued - p.stages); j < issued; ++j)
-        mbar_wait(&full[j % p.stages], (j / p.stages) & 1);
-    }
-    return;
-  }
-
-  // ---------------------------------------------------------------- consumers
-  const int gid = lane >> 2, tid4 = lane & 3;
+  if (i0 >= i1) return;
   const int units = p.K / 128;
-  uint8_t* xs = smem + L.off_xs;
-  float4* red = reinterpret_cast<float4*>(smem + L.off_red);
-  int cur_g = -1, row0 = 0, nrows = 0;
-  float gm0 = 0.0f, gm1 = 0.0f;
-  const bool has_x = gid < p.xrows;
-  const uint8_t* xrow = xs + (has_x ? gid : 0) * L.xs_pitch + tid4 * 16;
+  const int U = (units + kNW - 1) / kNW;           // steps per item
+  const uint32_t rowb = p.K / 2, scb = p.K / 16;
+  const uint64_t pol = policy_evict_first();
 
-  for (int it = i0; it < i1; ++it) {
-    const int j = it - i0, s = j % p.stages;
-    const uint32_t ph = (j / p.stages) & 1;
-    const int g = it / tiles, tile = it - g * tiles;
-    if (g != cur_g) {
-      named_bar_sync(1, kNW * 32);
-      const int4 grp = p.groups[g];
-      row0 = grp.y;
-      nrows = grp.z;
-      const uint8_t* rec = p.bank + (uint64_t)grp.x * p.stride;
-      gm0 = global_mult(*reinterpret_cast<const float*>(rec + p.global_off[0]), p.global_mode);
-      gm1 = GATEUP ? global_mult(*reinterpret_cast<const float*>(rec + p.global_off[1]), p.global_mode)
-                   : 0.0f;
-      fill_xs<GATEUP>(p, L, xs, row0, nrows, threadIdx.x);
-      named_bar_sync(1, kNW * 32);
-      cur_g = g;
+  // Per-thread byte offsets (inside a record) of rows gid and gid + 8 of tile 0.
+  const uint64_t c0_off = p.codes_off[0] + (uint64_t)gid * rowb + tid4 * 16;
+  const uint64_t s0_off = p.scales_off[0] + (uint64_t)gid * scb + tid4 * 2;
+  const uint64_t c1_off = GATEUP ? p.codes_off[1] + (uint64_t)gid * rowb + tid4 * 16 : c0_off + 8 * rowb;
+  const uint64_t s1_off = GATEUP ? p.scales_off[1] + (uint64_t)gid * scb + tid4 * 2 : s0_off + 8 * scb;
+  const int tile_rows = GATEUP ? 8 : 16;
+
+  auto start = [&](Cursor& c, int item) {
+    c.item = item;
+    c.q = 0;
+    c.g = item / tiles;
+    c.tile = item - c.g * tiles;
+    c.rec = p.bank + (uint64_t)__ldg(&p.groups[c.g].x) * p.stride;
+  };
+  auto advance = [&](Cursor& c) {
+    if (++c.q == U) {
+      c.q = 0;
+      ++c.item;
+      if (++c.tile == tiles && c.item < i1) {
+        c.tile = 0;
+        ++c.g;
+        c.rec = p.bank + (uint64_t)__ldg(&p.groups[c.g].x) * p.stride;
+      }
     }
-    if (!mbar_wait(&full[s], ph)) break;
+  };
+  auto load = [&](const Cursor& c, Frag& f) {
+    const int u = warp + kNW * c.q;
+    if (c.item < i1 && u < units) {
+      const uint64_t row = (uint64_t)c.tile * tile_rows;
+      const uint8_t* b = c.rec + u * 64;
+      f.c0 = ld_v4_stream(b + c0_off + row * rowb, pol);
+      f.c1 = ld_v4_stream(b + c1_off + row * rowb, pol);
+      const uint8_t* sb = c.rec + u * 8;
+      f.s0 = ld_u16_nc(sb + s0_off + row * scb);
+      f.s1 = ld_u16_nc(sb + s1_off + row * scb);
+    }
+  };
 
-    const uint8_t* st = smem + s * L.stage_bytes;
-    const uint8_t* rowA = st + gid * L.code_pitch + tid4 * 16;
-    const uint8_t* rowB = rowA + 8 * L.code_pitch;
-    const uint8_t* scA = st + L.stage_codes + gid * scb + tid4 * 2;
-    const uint8_t* scB = scA + 8 * scb;
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll 1
-    for (int u = warp; u < units; u += kNW) {
-      const uint4 qa = *reinterpret_cast<const uint4*>(rowA + u * 64);
-      const uint4 qb = *reinterpret_cast<const uint4*>(rowB + u * 64);
-      const uint32_t hsa = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(scA + u * 8));
-      const uint32_t hsb = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(scB + u * 8));
+  const bool has_x = gid < p.xrows;
+  const uint8_t* xrow = xs + (has_x ? gid : 0) * xs_pitch(p.K) + tid4 * 16;
+  int cur_g = -1, row0 = 0, nrows = 0, j = 0;
+  float gm0 = 0.0f, gm1 = 0.0f;
+  float acc[2][4];
+
+  auto compute = [&](const Cursor& c, const Frag& f) {
+    if (c.q == 0) {
+      if (c.g != cur_g) {
+        named_bar_sync(1, kThreads);
+        const int4 grp = p.groups[c.g];
+        row0 = grp.y;
+        nrows = grp.z;
+        gm0 = global_mult(*reinterpret_cast<const float*>(c.rec + p.global_off[0]), p.global_mode);
+        gm1 = GATEUP ? global_mult(*reinterpret_cast<const float*>(c.rec + p.global_off[1]), p.global_mode) : 0.0f;
+        fill_xs<GATEUP>(p, xs, row0, nrows);
+        named_bar_sync(1, kThreads);
+        cur_g = c.g;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[0][i] = acc[1][i] = 0.0f;
+    }
+    const int u = warp + kNW * c.q;
+    if (u < units) {
       uint4 xq[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        xq[i] = has_x ? *reinterpret_cast<const uint4*>(xrow + u * 256 + i * 64)
-                      : make_uint4(0, 0, 0, 0);
-      const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
-      const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
+        xq[i] = has_x ? *reinterpret_cast<const uint4*>(xrow + u * 256 + i * 64) : make_uint4(0, 0, 0, 0);
+      const uint32_t hs0 = e4m3x2_to_f16x2((uint16_t)f.s0);
+      const uint32_t hs1 = e4m3x2_to_f16x2((uint16_t)f.s1);
+      const uint32_t w0[4] = {f.c0.x, f.c0.y, f.c0.z, f.c0.w};
+      const uint32_t w1[4] = {f.c1.x, f.c1.y, f.c1.z, f.c1.w};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t sA = bcast_half(hsa, q >= 2), sB = bcast_half(hsb, q >= 2);
+      for (int w = 0; w < 4; ++w) {
+        const uint32_t sA = bcast_half(hs0, w >= 2), sB = bcast_half(hs1, w >= 2);
         uint32_t fa[4], fb[4];
-        e2m1x8_to_f16x8(wa[q], fa);
-        e2m1x8_to_f16x8(wb[q], fb);
+        e2m1x8_to_f16x8(w0[w], fa);
+        e2m1x8_to_f16x8(w1[w], fb);
         const uint32_t a0[4] = {hmul2(fa[0], sA), hmul2(fb[0], sB), hmul2(fa[1], sA), hmul2(fb[1], sB)};
-        mma_16816(acc, a0, xq[q].x, xq[q].y);
+        mma_16816(acc[0], a0, xq[w].x, xq[w].y);
         const uint32_t a1[4] = {hmul2(fa[2], sA), hmul2(fb[2], sB), hmul2(fa[3], sA), hmul2(fb[3], sB)};
-        mma_16816(acc, a1, xq[q].z, xq[q].w);
+        mma_16816(acc[1], a1, xq[w].z, xq[w].w);
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
-
-    const int buf = j & 1;
-    red[(buf * kNW + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    named_bar_sync(1, kNW * 32);
-    if (warp == j % kNW) {
-      float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (c.q == U - 1) {
+      const int buf = j & 1;
+      red[(buf * kNW + warp) * 32 + lane] =
+          make_float4(acc[0][0] + acc[1][0], acc[0][1] + acc[1][1], acc[0][2] + acc[1][2], acc[0][3] + acc[1][3]);
+      named_bar_sync(1, kThreads);
+      if (warp == j % kNW) {
+        float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-      for (int w = 0; w < kNW; ++w) {
-        const float4 v = red[(buf * kNW + w) * 32 + lane];
-        c[0] += v.x;
-        c[1] += v.y;
-        c[2] += v.z;
-        c[3] += v.w;
-      }
-      // c[0], c[1]: MMA row gid, token slots 2*tid4, 2*tid4+1; c[2], c[3]: MMA row gid + 8.
+        for (int w = 0; w < kNW; ++w) {
+          const float4 v = red[(buf * kNW + w) * 32 + lane];
+          cs[0] += v.x, cs[1] += v.y, cs[2] += v.z, cs[3] += v.w;
+        }
+        // cs[0..1]: MMA row gid, token slots 2*tid4, 2*tid4+1; cs[2..3]: MMA row gid + 8.
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int n = 2 * tid4 + cc;
-        if (n < nrows) {
-          float* o = p.out + (size_t)(row0 + n) * p.N;
-          if (GATEUP) {
-            const float gv = c[cc] * gm0, uv = c[2 + cc] * gm1;
-            o[tile * 8 + gid] = gv / (1.0f + expf(-gv)) * uv;
-          } else {
-            o[tile * kTileRows + gid] = c[cc] * gm0;
-            o[tile * kTileRows + gid + 8] = c[2 + cc] * gm0;
+        for (int cc = 0; cc < 2; ++cc) {
+          const int n = 2 * tid4 + cc;
+          if (n < nrows) {
+            if (GATEUP) {
+              p.out[(size_t)(row0 + n) * p.N + c.tile * 8 + gid] = silu_mul(cs[cc] * gm0, cs[2 + cc] * gm1);
+            } else {
+              float* o = p.out + (size_t)(row0 + n) * p.N;
+              o[c.tile * 16 + gid] = cs[cc] * gm0;
+              o[c.tile * 16 + gid + 8] = cs[2 + cc] * gm0;
+            }
           }
         }
       }
+      ++j;
     }
+  };
+
+  // Three-slot ring: loads run two steps ahead of the step being computed.
+  const int S = (i1 - i0) * U;
+  Cursor lc, cc;
+  start(lc, i0);
+  start(cc, i0);
+  Frag fA, fB, fC;
+  load(lc, fA);
+  advance(lc);
+  load(lc, fB);
+  advance(lc);
+  for (int s = 0; s < S; s += 3) {
+    load(lc, fC);
+    advance(lc);
+    compute(cc, fA);
+    advance(cc);
+    if (s + 1 >= S) break;
+    load(lc, fA);
+    advance(lc);
+    compute(cc, fB);
+    advance(cc);
+    if (s + 2 >= S) break;
+    load(lc, fB);
+    advance(lc);
+    compute(cc, fC);
+    advance(cc);
   }
 }
 
-int pick_stages(int K, int xrows, int stage_cap) {
-  for (int s = stage_cap; s >= 2; --s)
-    if (make_layout(K, s, xrows).total <= kSmemLimit) return s;
-  return 0;
-}
-
 template <bool GATEUP>
-int launch(const DecodeParams& p0, int num_sms, cudaStream_t s) {
-  DecodeParams p = p0;
-  p.stages = pick_stages(p.K, p.xrows, kMaxStages);
-  if (p.stages == 0) return -(int)cudaErrorInvalidValue;
-  const int bytes = make_layout(p.K, p.stages, p.xrows).total;
+int launch(const DecodeParams& p, int num_sms, cudaStream_t s) {
+  const int bytes = smem_total(p.K, p.xrows);
+  if (bytes > kSmemLimit) return -(int)cudaErrorInvalidValue;
   cudaError_t err = cudaFuncSetAttribute(decode_kernel<GATEUP>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (err != cudaSuccess) return -(int)err;
-  decode_kernel<GATEUP><<<num_sms, kThreads, bytes, s>>>(p);
+  decode_kernel<GATEUP><<<num_sms * kCtasPerSm, kThreads, bytes, s>>>(p);
   err = cudaGetLastError();
   return err == cudaSuccess ? 1 : -(int)err;
 }
@@ -289,8 +288,8 @@ int launch(const DecodeParams& p0, int num_sms, cudaStream_t s) {
 
 size_t decode_smem_bytes(int K, int xrows, bool gateup) {
   (void)gateup;
-  const int st = pick_stages(K, xrows, kMaxStages);
-  return st ? (size_t)make_layout(K, st, xrows).total : 0;
+  const int b = smem_total(K, xrows);
+  return b <= kSmemLimit ? (size_t)b : 0;
 }
 
 int launch_decode_gateup(const BankView& bank, const uint16_t* x, int k, const RouteBufs& rb,
@@ -323,8 +322,11 @@ int launch_decode_down(const BankView& bank, const float* h, const RouteBufs& rb
   p.bank = bank.base;
   p.stride = bank.stride;
   p.codes_off[0] = bank.codes_off[2];
+  p.codes_off[1] = bank.codes_off[2];
   p.scales_off[0] = bank.scales_off[2];
+  p.scales_off[1] = bank.scales_off[2];
   p.global_off[0] = bank.global_off[2];
+  p.global_off[1] = bank.global_off[2];
   p.global_mode = bank.global_mode;
   p.K = bank.I;
   p.N = bank.H;

@@ -15,10 +15,13 @@ struct RouteBufs {
   int32_t* offsets;    // [E + 1]
   int32_t* perm;       // [T * k]
   int32_t* inv;        // [T * k]
-  int4* groups;        // [max_groups]: (expert, first permuted row, rows, 0)
+  int4* groups;        // [max_groups]: (expert, first permuted row, rows, 0), rows >= 2
   int32_t* ngroups;    // [1]
+  int4* singles;       // [max_groups]: (expert, permuted row, 1, 0): one-row groups
+  int32_t* nsingles;   // [1]
   int32_t* chunk_counts;  // [nchunks, E] (multi-CTA routing only)
   int group_rows;      // rows per group (decode token tile)
+  int split_singles;   // 1: one-row groups go to `singles`; 0: they stay in `groups`
 };
 
 // Tokens per routing chunk in the multi-CTA router; one CTA routes T <= this on its own.
@@ -43,13 +46,20 @@ struct BankView {
   int E, H, I;
 };
 
-// Decode path: grouped NVFP4 GEMV/GEMM on mma.sync with TMA bulk staging.
+// Decode path, groups of 2..8 rows: grouped NVFP4 GEMM on mma.sync.
 // gate/up: h [R, I] f32 = silu(x Wg^T gg) * (x Wu^T gu) for every routed row.
 int launch_decode_gateup(const BankView& bank, const uint16_t* x, int k, const RouteBufs& rb,
                          int xrows, float* h, int num_sms, cudaStream_t s);
 // down: y [R, H] f32 = h Wd^T gd for every routed row.
 int launch_decode_down(const BankView& bank, const float* h, const RouteBufs& rb, int xrows,
                        float* y, int num_sms, cudaStream_t s);
+
+// Decode path, one-row groups: warp-per-row NVFP4 GEMV on CUDA cores (same outputs).
+bool rows_supported(int K, bool gateup);
+int launch_rows_gateup(const BankView& bank, const uint16_t* x, int k, const RouteBufs& rb,
+                       float* h, int num_sms, cudaStream_t s);
+int launch_rows_down(const BankView& bank, const float* h, const RouteBufs& rb, float* y,
+                     int num_sms, cudaStream_t s);
 
 // out [T, H] bf16 = sum_j w[t, j] * y[inv[t*k+j]]; optional x_next = bf16(x + out).
 int launch_combine(const float* y, const float* w, const int32_t* inv, int64_t T, int k, int H,

@@ -82,7 +82,7 @@ int current_device(int* dev, DeviceInfo* info) {
 
 // Sizes of the workspace sub-buffers, each 256-byte aligned.
 struct WsLayout {
-  size_t ids, w, counts, offsets, perm, inv, groups, ngroups, chunk_counts, h, y, total;
+  size_t ids, w, counts, offsets, perm, inv, groups, ngroups, singles, nsingles, chunk_counts, h, y, total;
 };
 
 size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -105,6 +105,8 @@ WsLayout ws_layout(int64_t T, int E, int k, int H, int I, int path) {
   L.inv = take(R * 4);
   L.groups = take((size_t)moe::max_groups((int64_t)R, E, 8) * 16);
   L.ngroups = take(4);
+  L.singles = take((size_t)E * 16);
+  L.nsingles = take(4);
   L.chunk_counts = take(T > moe::kRouteChunk ? (size_t)moe::route_chunks(T) * E * 4 : 0);
   L.h = take(R * (size_t)I * 4);
   L.y = take(R * (size_t)H * 4);
@@ -175,16 +177,27 @@ cudaEvent_t prof_event() {
   return e;
 }
 
+// While a stream captures, an event record only becomes a timing node of the graph when it
+// is recorded as an external event.
+void prof_record(cudaEvent_t e, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(s, &cs);
+  if (cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+  else
+    cudaEventRecord(e, s);
+}
+
 void prof_before(int kind, cudaStream_t s) {
   if (!t_prof_on) return;
   ProfPair p{kind, prof_event(), prof_event()};
-  cudaEventRecord(p.a, s);
+  prof_record(p.a, s);
   t_prof.push_back(p);
 }
 
 void prof_after(cudaStream_t s) {
   if (!t_prof_on || t_prof.empty()) return;
-  cudaEventRecord(t_prof.back().b, s);
+  prof_record(t_prof.back().b, s);
 }
 
 int after_launch(int rc, cudaStream_t s, const char* what, int* count) {
@@ -233,8 +246,11 @@ moe::RouteBufs route_bufs(uint8_t* ws, const WsLayout& L) {
   b.inv = reinterpret_cast<int32_t*>(ws + L.inv);
   b.groups = reinterpret_cast<int4*>(ws + L.groups);
   b.ngroups = reinterpret_cast<int32_t*>(ws + L.ngroups);
+  b.singles = reinterpret_cast<int4*>(ws + L.singles);
+  b.nsingles = reinterpret_cast<int32_t*>(ws + L.nsingles);
   b.chunk_counts = reinterpret_cast<int32_t*>(ws + L.chunk_counts);
   b.group_rows = 8;
+  b.split_singles = 0;
   return b;
 }
 
@@ -290,21 +306,31 @@ int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
     return rc;
   }
   uint8_t* w8 = static_cast<uint8_t*>(ws);
-  const moe::RouteBufs rb = route_bufs(w8, L);
+  moe::RouteBufs rb = route_bufs(w8, L);
+  // One-row groups take the CUDA-core row kernels when both widths allow; groups of two or
+  // more rows (none when T == 1) take the mma.sync kernels.
+  const bool rows = moe::rows_supported(H, true) && moe::rows_supported(I, false);
+  const bool multi = !rows || T > 1;
+  rb.split_singles = rows ? 1 : 0;
   const moe::BankView bv = view_of(bank);
   float* h = reinterpret_cast<float*>(w8 + L.h);
   float* y = reinterpret_cast<float*>(w8 + L.y);
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
   int launches = 0;
   prof_before(MOE_NVFP4_KERNEL_ROUTE, s);
   if ((rc = after_launch(moe::launch_route(logits, T, E, k, rb, s), s, "route", &launches))) return rc;
   prof_before(MOE_NVFP4_KERNEL_DECODE_GATEUP, s);
-  if ((rc = after_launch(moe::launch_decode_gateup(bv, static_cast<const uint16_t*>(x), k, rb, xrows, h,
-                                                   info.sms, s),
-                         s, "decode gate/up", &launches)))
+  if (rows && (rc = after_launch(moe::launch_rows_gateup(bv, xb, k, rb, h, info.sms, s), s, "rows gate/up",
+                                 &launches)))
+    return rc;
+  if (multi && (rc = after_launch(moe::launch_decode_gateup(bv, xb, k, rb, xrows, h, info.sms, s), s,
+                                  "decode gate/up", &launches)))
     return rc;
   prof_before(MOE_NVFP4_KERNEL_DECODE_DOWN, s);
-  if ((rc = after_launch(moe::launch_decode_down(bv, h, rb, xrows, y, info.sms, s), s, "decode down",
-                         &launches)))
+  if (rows && (rc = after_launch(moe::launch_rows_down(bv, h, rb, y, info.sms, s), s, "rows down", &launches)))
+    return rc;
+  if (multi && (rc = after_launch(moe::launch_decode_down(bv, h, rb, xrows, y, info.sms, s), s, "decode down",
+                                  &launches)))
     return rc;
   prof_before(MOE_NVFP4_KERNEL_COMBINE, s);
   if ((rc = after_launch(moe::launch_combine(y, rb.w, rb.inv, T, k, H, static_cast<const uint16_t*>(x),
