@@ -119,6 +119,27 @@ int moe_nvfp4_forward_host(const void* x_host, const float* logits_host, int64_t
                            const moe_nvfp4_bank* bank, int32_t k, void* out_host, void* stream);
 
 /*
+ * As moe_nvfp4_forward, but allocating nothing: the scratch comes from one fixed array of
+ * MOE_NVFP4_NOALLOC_MAX_BYTES that the library places in device memory when it is loaded
+ * (every device the process uses holds it until exit).  The pages this library follows have
+ * no counterpart for this call; it exists for callers that cannot call cudaMalloc: runtimes
+ * that reserve all device memory up front and forbid later allocations, and latency-critical
+ * loops that must not pay for the device-wide synchronisation an allocation can cause.
+ *  - Inputs and outputs are the caller's, as for moe_nvfp4_forward.
+ *  - Calls needing more scratch than the array holds (about T*k*(H+I)*4 bytes plus routing
+ *    tables; T <= 64 at E=256, k=8, H=5120, I=2560) return MOE_NVFP4_ERR_WORKSPACE and enqueue
+ *    nothing.
+ *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *    that device current; make that first call before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents; nothing in it needs
+ *    to start at zero (each call writes every entry it reads).  Calls whose GPU work overlaps
+ *    -- different streams, or several host threads -- race on it: order them on one stream.
+ */
+#define MOE_NVFP4_NOALLOC_MAX_BYTES ((size_t)16 << 20)
+int moe_nvfp4_forward_noalloc(const void* x_dev, const float* logits_dev, int64_t T,
+                              const moe_nvfp4_bank* bank, int32_t k, void* out_dev, void* stream);
+
+/*
  * Routing only (router + permutation), for inspection:
  *  ids_dev [T, k] int32 expert ids in rank order;   w_dev [T, k] f32 softmax weights;
  *  counts_dev [E] int32;  offsets_dev [E+1] int32 exclusive prefix sum of counts;

@@ -76,6 +76,20 @@ def moe_nvfp4_forward_ex(x, logits, bank: Bank, k: int, out=None, x_next=None, w
     return out
 
 
+def moe_nvfp4_forward_noalloc(x, logits, bank: Bank, k: int, out=None, stream=None):
+    """As moe_nvfp4_forward, with scratch from the library's fixed device array (no allocation).
+
+    For callers that cannot allocate device memory during a call; `out` may be passed in so
+    that the call itself allocates nothing on the Python side either.
+    """
+    import torch
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().moe_nvfp4_forward_noalloc(_ptr(x), _ptr(logits), x.shape[0], ctypes.byref(bank), k, _ptr(out),
+                                           _stream(stream)))
+    return out
+
+
 def moe_nvfp4_forward_host(x_host: np.ndarray, logits_host: np.ndarray, bank: Bank, k: int,
                            out_host: np.ndarray | None = None, stream=None) -> np.ndarray:
     """End-to-end call on host arrays: x [T, H] BF16 bit patterns (uint16), logits [T, E] f32.

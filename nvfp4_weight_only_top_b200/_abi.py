@@ -46,6 +46,7 @@ SIGNATURES = {
     "moe_nvfp4_forward": (ctypes.c_int, [_vp, _vp, _i64, _BANKP, _i32, _vp, _vp]),
     "moe_nvfp4_forward_ex": (ctypes.c_int, [_vp, _vp, _i64, _BANKP, _i32, _vp, _vp, _vp, _sz, _i32, _vp]),
     "moe_nvfp4_forward_host": (ctypes.c_int, [_vp, _vp, _i64, _BANKP, _i32, _vp, _vp]),
+    "moe_nvfp4_forward_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _BANKP, _i32, _vp, _vp]),
     "moe_nvfp4_route": (ctypes.c_int, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_nvfp4_workspace_bytes": (ctypes.c_size_t, [_i64, _i32, _i32, _i32, _i32, _i32]),
     "moe_nvfp4_last_error": (ctypes.c_char_p, []),

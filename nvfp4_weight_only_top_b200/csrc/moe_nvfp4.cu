@@ -352,6 +352,27 @@ int ensure_stage(void** p, size_t* have, size_t need) {
   return MOE_NVFP4_OK;
 }
 
+// Fixed scratch for moe_nvfp4_forward_noalloc: a file-scope device array, so the entry point
+// never allocates.  Every device that loads the library holds it until the process exits.
+constexpr size_t kNoAllocBytes = (size_t)16 << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+// Device address of g_noalloc_scratch per device (host code only sees a stand-in for it).
+std::vector<void*> g_noalloc_addr;
+
+int noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if ((int)g_noalloc_addr.size() <= dev) g_noalloc_addr.resize(dev + 1, nullptr);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);   // current device = dev
+    if (e != cudaSuccess) return cuda_fail(e, "resolve the fixed scratch array");
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return MOE_NVFP4_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -458,6 +479,27 @@ int moe_nvfp4_device_status(void) {
   if (e != cudaSuccess) return cuda_fail(e, "clear device status");
   if (v != 0) return fail(MOE_NVFP4_ERR_TIMEOUT, "a bounded device wait gave up (status %d)", v);
   return MOE_NVFP4_OK;
+}
+
+int moe_nvfp4_forward_noalloc(const void* x_dev, const float* logits_dev, int64_t T, const moe_nvfp4_bank* bank,
+                              int32_t k, void* out_dev, void* stream) {
+  t_last_launches = 0;
+  int rc = check_bank(bank);
+  if (rc) return rc;
+  if ((rc = check_k_T(T, bank->num_experts, k))) return rc;
+  const size_t need = ws_layout(T, bank->num_experts, k, bank->hidden, bank->intermediate, MOE_NVFP4_PATH_AUTO).total;
+  if (need > kNoAllocBytes)
+    return fail(MOE_NVFP4_ERR_WORKSPACE,
+                "this call needs %zu bytes of scratch; the fixed array of moe_nvfp4_forward_noalloc holds %zu "
+                "(MOE_NVFP4_NOALLOC_MAX_BYTES); use moe_nvfp4_forward_ex with a caller workspace",
+                need, kNoAllocBytes);
+  int dev;
+  DeviceInfo info;
+  if ((rc = current_device(&dev, &info))) return rc;
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(dev, &scratch))) return rc;
+  return forward_impl(x_dev, logits_dev, T, bank, k, out_dev, nullptr, scratch, kNoAllocBytes,
+                      MOE_NVFP4_PATH_AUTO, stream);
 }
 
 int moe_nvfp4_last_launch_count(void) { return t_last_launches; }

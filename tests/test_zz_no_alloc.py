@@ -1,0 +1,56 @@
+"""moe_nvfp4_forward_noalloc: the entry point for callers that cannot allocate device memory
+(runtimes that reserve all device memory up front, latency-critical loops that cannot afford
+an allocation's synchronisation).  It must give the same layer output as moe_nvfp4_forward,
+call after call, although every call reuses one fixed scratch array inside the library.
+
+This file is collected last on purpose: it must pass both on its own in a fresh process and
+after every other test has run in the same process.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import moe_inputs
+import oracle
+from conftest import assert_layer_close
+from gpu_helpers import bf16_tensor, bits_of, device_bank
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode_t1", "decode_t64_zipf"])
+def test_noalloc_matches_forward_on_two_calls_in_a_row(name):
+    import torch
+    import nvfp4_weight_only_top_b200 as moe
+    cfg = moe_inputs.CONFIGS[name]
+    buf, bank = device_bank(cfg)
+    lib = moe.lib()
+    for call in range(2):                      # different inputs on each call
+        x = bf16_tensor(moe_inputs.make_x(cfg, seed=cfg.seed + call))
+        lg = torch.from_numpy(moe_inputs.make_logits(cfg, seed=cfg.seed + call)).cuda()
+        ref = moe.moe_nvfp4_forward(x, lg, bank, cfg.k)
+        out = torch.empty_like(x)
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        rc = lib.moe_nvfp4_forward_noalloc(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(lg.data_ptr()),
+                                           x.shape[0], ctypes.byref(bank), cfg.k,
+                                           ctypes.c_void_p(out.data_ptr()), stream)
+        assert rc == 0, moe.moe_nvfp4_last_error()
+        torch.cuda.synchronize()
+        assert moe.moe_nvfp4_device_status() == 0
+        assert_layer_close(oracle.bf16_bits_to_f64(bits_of(out)), oracle.bf16_bits_to_f64(bits_of(ref)),
+                           f"{name} call {call}")
+
+
+def test_noalloc_rejects_scratch_beyond_its_array():
+    import torch
+    import nvfp4_weight_only_top_b200 as moe
+    cfg = moe_inputs.CONFIGS["decode_t1"]
+    buf, bank = device_bank(cfg)
+    T = 4096                                    # needs far more than the fixed array holds
+    x = torch.zeros((T, cfg.H), dtype=torch.bfloat16, device="cuda")
+    lg = torch.zeros((T, cfg.E), dtype=torch.float32, device="cuda")
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_nvfp4_forward_noalloc(x, lg, bank, cfg.k)
+    assert ei.value.code == -4 and "fixed array" in str(ei.value)
+    assert moe.moe_nvfp4_last_launch_count() == 0
