@@ -67,4 +67,16 @@ int launch_combine(const float* y, const float* w, const int32_t* inv, int64_t T
 
 size_t decode_smem_bytes(int K, int xrows, bool gateup);
 
+// Prefill path: grouped NVFP4 GEMM on tcgen05 tensor cores, groups of up to kPrefillRows rows.
+constexpr int kPrefillRows = 256;
+bool prefill_supported(int H, int I);
+// xp [R, H] f16 = x[perm[r] / k] for every routed row r (expert order).
+int launch_gather(const uint16_t* x, const int32_t* perm, int k, int64_t R, int H, void* xp, cudaStream_t s);
+// h16 [R, I] f16 = silu(xp Wg^T gg) * (xp Wu^T gu).
+int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const RouteBufs& rb, void* h16,
+                          int num_sms, cudaStream_t s);
+// y [R, H] f32 = h16 Wd^T gd.
+int launch_prefill_down(const BankView& bank, const void* h16, int64_t R, const RouteBufs& rb, float* y,
+                        int num_sms, cudaStream_t s);
+
 }  // namespace moe

@@ -261,12 +261,63 @@ int check_k_T(int64_t T, int E, int k) {
   return MOE_NVFP4_OK;
 }
 
-int resolve_path(int path, int64_t T, int k, int E) {
-  if (path == MOE_NVFP4_PATH_AUTO) return MOE_NVFP4_PATH_DECODE;
-  (void)T;
-  (void)k;
-  (void)E;
-  return path;
+// AUTO takes the tensor-core path once experts average more than 8 routed rows and the
+// shapes allow it (H a multiple of 256, I of 128).
+int resolve_path(int path, int64_t T, int k, int E, int H, int I) {
+  if (path != MOE_NVFP4_PATH_AUTO) return path;
+  return (T * k > (int64_t)8 * E && moe::prefill_supported(H, I)) ? MOE_NVFP4_PATH_PREFILL
+                                                                  : MOE_NVFP4_PATH_DECODE;
+}
+
+// Prefill path: route (groups of up to 256 rows) -> gather -> tcgen05 gate/up -> tcgen05 down
+// -> combine.  The f16 gathered rows live in the y region and the f16 intermediate in the h
+// region, so the workspace is the decode path's.
+int prefill_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_bank* bank, int32_t k, void* out,
+                 void* x_next, void* workspace, size_t workspace_bytes, void* stream, int dev,
+                 const DeviceInfo& info) {
+  const int E = bank->num_experts, H = bank->hidden, I = bank->intermediate;
+  const WsLayout L = ws_layout(T, E, k, H, I, MOE_NVFP4_PATH_PREFILL);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  int rc;
+  if (ws) {
+    if (workspace_bytes < L.total)
+      return fail(MOE_NVFP4_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes,
+                  L.total);
+    if (!aligned(ws, 256)) return fail(MOE_NVFP4_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  } else if ((rc = ensure_workspace(dev, L.total, s, &ws))) {
+    return rc;
+  }
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  moe::RouteBufs rb = route_bufs(w8, L);
+  rb.group_rows = moe::kPrefillRows;
+  rb.split_singles = 0;
+  const moe::BankView bv = view_of(bank);
+  const int64_t R = T * k;
+  void* h16 = w8 + L.h;
+  void* xp = w8 + L.y;
+  float* y = reinterpret_cast<float*>(w8 + L.y);
+  int launches = 0;
+  prof_before(MOE_NVFP4_KERNEL_ROUTE, s);
+  if ((rc = after_launch(moe::launch_route(logits, T, E, k, rb, s), s, "route", &launches))) return rc;
+  prof_before(MOE_NVFP4_KERNEL_PREFILL_GATHER, s);
+  if ((rc = after_launch(moe::launch_gather(static_cast<const uint16_t*>(x), rb.perm, k, R, H, xp, s), s, "gather",
+                         &launches)))
+    return rc;
+  prof_before(MOE_NVFP4_KERNEL_PREFILL_GATEUP, s);
+  if ((rc = after_launch(moe::launch_prefill_gateup(bv, xp, R, rb, h16, info.sms, s), s, "prefill gate/up",
+                         &launches)))
+    return rc;
+  prof_before(MOE_NVFP4_KERNEL_PREFILL_DOWN, s);
+  if ((rc = after_launch(moe::launch_prefill_down(bv, h16, R, rb, y, info.sms, s), s, "prefill down", &launches)))
+    return rc;
+  prof_before(MOE_NVFP4_KERNEL_COMBINE, s);
+  if ((rc = after_launch(moe::launch_combine(y, rb.w, rb.inv, T, k, H, static_cast<const uint16_t*>(x),
+                                             static_cast<uint16_t*>(out), static_cast<uint16_t*>(x_next), s),
+                         s, "combine", &launches)))
+    return rc;
+  t_last_launches = launches;
+  return MOE_NVFP4_OK;
 }
 
 int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_bank* bank, int32_t k,
@@ -286,9 +337,13 @@ int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
   if (!x || !logits || !out) return fail(MOE_NVFP4_ERR_INVALID_ARG, "x, logits and out must not be NULL");
   if (!aligned(x, 16) || !aligned(logits, 16) || !aligned(out, 16) || (x_next && !aligned(x_next, 16)))
     return fail(MOE_NVFP4_ERR_INVALID_ARG, "x, logits, out and x_next must be 16-byte aligned");
-  const int use = resolve_path(path, T, k, E);
-  if (use == MOE_NVFP4_PATH_PREFILL)
-    return fail(MOE_NVFP4_ERR_UNSUPPORTED, "prefill path not available in this build");
+  const int use = resolve_path(path, T, k, E, H, I);
+  if (use == MOE_NVFP4_PATH_PREFILL) {
+    if (!moe::prefill_supported(H, I))
+      return fail(MOE_NVFP4_ERR_UNSUPPORTED, "prefill path needs H %% 256 == 0 and I %% 128 == 0 (H=%d, I=%d)", H,
+                  I);
+    return prefill_impl(x, logits, T, bank, k, out, x_next, workspace, workspace_bytes, stream, dev, info);
+  }
   const int xrows = (int)(T < 8 ? T : 8);
   if (moe::decode_smem_bytes(H, xrows, true) == 0 || moe::decode_smem_bytes(I, xrows, false) == 0 ||
       (int)moe::decode_smem_bytes(H, xrows, true) > info.smem_optin)
@@ -465,7 +520,7 @@ int moe_nvfp4_route(const float* logits_dev, int64_t T, int32_t E, int32_t k, in
 
 size_t moe_nvfp4_workspace_bytes(int64_t T, int32_t E, int32_t k, int32_t H, int32_t I, int32_t path) {
   if (T < 0 || E < 1 || E > 1024 || k < 1 || k > 32 || k > E || H < 128 || I < 128) return 0;
-  return ws_layout(T, E, k, H, I, resolve_path(path, T, k, E)).total;
+  return ws_layout(T, E, k, H, I, resolve_path(path, T, k, E, H, I)).total;
 }
 
 const char* moe_nvfp4_last_error(void) { return t_last_error.c_str(); }

@@ -1,0 +1,407 @@
+// Prefill path: grouped NVFP4 expert GEMM on the 5th-generation tensor cores (tcgen05, TMEM).
+//
+// Work item (tile) = one group of up to 256 routed rows of one expert x 2 MMA M-tiles of 128
+// weight rows: for gate/up the gate rows r0 .. r0+127 and the same up rows (SwiGLU is applied
+// in the epilogue), for down 256 consecutive rows of Wd.  The two M-tiles share every tile of
+// activations, halving activation traffic per FLOP.
+//
+// Per CTA (one per SM, persistent over tiles): warps 0-3 dequantize -- each thread owns one
+// weight row of each M-tile, streams its codes and scales from HBM with 128-bit loads two
+// stages ahead, converts E2M1 with cvt and multiplies by the E4M3 block scale in f16 (exact),
+// and stores the f16 row chunk into a 128-byte-swizzled K-major shared-memory stage; warp 4
+// loads the group's activation rows (f16, expert-permuted) with 2-D TMA into swizzled stages;
+// warp 5 issues tcgen05.mma kind::f16 (M = 128, N = rows of the group rounded up to 16,
+// K = 16) into two f32 accumulators in tensor memory and releases each stage with
+// tcgen05.commit.  After a tile's last K stage, warps 0-3 read the accumulators back with
+// tcgen05.ld and apply the global scale (and SwiGLU for gate/up).
+//
+// Weight layout: page "Beam 1.0 501B-A23B, streaming pack, NVFP4 experts / MLX 8-bit
+// residents", section "What this pack holds"; SwiGLU in FP32: page "Beam-1.0-501B-A23B VQ
+// GGUF", section "What stays native".  The pages' prefill kernels ("decode-once prefill MoE
+// GEMM" on sm_120) dequantize each weight tile once for all of a group's tokens; so does this
+// one, on sm_100a tensor cores.
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kBM = 128;                       // rows per MMA M-tile
+constexpr int kKC = 64;                        // K per stage: one 128-byte swizzle row of f16
+constexpr int kStages = 3;
+constexpr int kMaxN = 256;
+constexpr int kBoxRows = 64;                   // activation rows per TMA box
+constexpr int kThreads = 32 * 6;               // 4 dequant/epilogue warps, TMA warp, MMA warp
+constexpr int kABytes = kBM * kKC * 2;         // 16 KB: one M-tile of one stage
+constexpr int kBBytes = kMaxN * kKC * 2;       // 32 KB: activations of one stage
+constexpr int kTmemCols = 512;                 // two 256-column f32 accumulators
+constexpr int kSmemBytes = kStages * (2 * kABytes + kBBytes) + 1024 /*barriers*/ + 1024 /*align*/;
+
+struct PrefillParams {
+  const uint8_t* bank;
+  uint64_t stride;
+  uint64_t codes_off[2], scales_off[2], global_off[2];  // matrix of M-tile 0 / M-tile 1
+  int global_mode;
+  int K;                 // inputs per weight row
+  int tiles_per_group;   // output-row tiles per group
+  int gateup;            // 1: M-tile 0 = gate rows, M-tile 1 = same up rows; 0: 256 consecutive rows
+  const int4* groups;    // (expert, first permuted row, rows <= 256, 0)
+  const int32_t* ngroups;
+  void* out;             // gate/up: h f16 [R, out_stride]; down: y f32 [R, out_stride]
+  int out_stride;
+};
+
+__device__ __forceinline__ uint4 ld_v4_nc(const uint8_t* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_u32_nc(const uint8_t* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// One thread's share of one stage: 64 codes and 4 scale bytes of each of its two rows.
+struct StageFrag {
+  uint4 c[2][2];
+  uint32_t s[2];
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap xmap, const PrefillParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = smem;                                   // [stage][m-tile] 16 KB each
+  uint8_t* sB = smem + kStages * 2 * kABytes;           // [stage] 32 KB each
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * kBBytes);
+  uint64_t* a_full = bars;
+  uint64_t* b_full = bars + kStages;
+  uint64_t* empty = bars + 2 * kStages;
+  uint64_t* d_full = bars + 3 * kStages;
+  uint64_t* d_empty = d_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_empty + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntiles = *p.ngroups * p.tiles_per_group;
+  const int nst = p.K / kKC;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&a_full[s], 4 * 32);
+      mbar_init(&b_full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(d_full, 1);
+    mbar_init(d_empty, 4 * 32);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 4) {
+    // ------------------------------------------------------------ dequant + epilogue
+    const int t = threadIdx.x;                      // weight row within each M-tile
+    const uint32_t rowb = p.K / 2, scb = p.K / 16;
+    const int total = ((ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x);  // tiles of this CTA
+    // Load cursor (two stages ahead of the stage being stored).
+    int ltile = 0, lc = 0;
+    auto tile_of = [&](int i) { return (int)blockIdx.x + i * (int)gridDim.x; };
+    auto load = [&](int i, int c, StageFrag& f) {
+      if (i >= total) return;
+      const int tt = tile_of(i), g = tt / p.tiles_per_group, m = tt - g * p.tiles_per_group;
+      const uint8_t* rec = p.bank + (uint64_t)__ldg(&p.groups[g].x) * p.stride;
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const uint64_t row = p.gateup ? (uint64_t)m * kBM + t : (uint64_t)m * 2 * kBM + mt * kBM + t;
+        const uint8_t* cp = rec + p.codes_off[mt] + row * rowb + c * (kKC / 2);
+        f.c[mt][0] = ld_v4_nc(cp);
+        f.c[mt][1] = ld_v4_nc(cp + 16);
+        f.s[mt] = ld_u32_nc(rec + p.scales_off[mt] + row * scb + c * (kKC / 16));
+      }
+    };
+    auto advance = [&](int& i, int& c) {
+      if (++c == nst) {
+        c = 0;
+        ++i;
+      }
+    };
+    auto store = [&](int s, const StageFrag& f) {
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const uint32_t base = smem_addr(sA + (s * 2 + mt) * kABytes) + t * 128;
+        const uint32_t h01 = e4m3x2_to_f16x2((uint16_t)(f.s[mt] & 0xFFFF));
+        const uint32_t h23 = e4m3x2_to_f16x2((uint16_t)(f.s[mt] >> 16));
+        const uint32_t sc[4] = {bcast_half(h01, false), bcast_half(h01, true), bcast_half(h23, false),
+                                bcast_half(h23, true)};
+        const uint32_t w[8] = {f.c[mt][0].x, f.c[mt][0].y, f.c[mt][0].z, f.c[mt][0].w,
+                               f.c[mt][1].x, f.c[mt][1].y, f.c[mt][1].z, f.c[mt][1].w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {                  // word j = K 8j .. 8j+7 = 16-byte chunk j
+          uint32_t e[4];
+          e2m1x8_to_f16x8(w[j], e);
+          const uint32_t s2 = sc[j >> 1];
+          st_shared_v4(base + ((j ^ (t & 7)) << 4), hmul2(e[0], s2), hmul2(e[1], s2), hmul2(e[2], s2),
+                       hmul2(e[3], s2));
+        }
+      }
+    };
+    auto epilogue = [&](int i) {
+      const int tt = tile_of(i), g = tt / p.tiles_per_group, m = tt - g * p.tiles_per_group;
+      const int4 grp = __ldg(&p.groups[g]);
+      const uint8_t* rec = p.bank + (uint64_t)grp.x * p.stride;
+      const float gm0 = global_mult(__ldg(reinterpret_cast<const float*>(rec + p.global_off[0])), p.global_mode);
+      const float gm1 = global_mult(__ldg(reinterpret_cast<const float*>(rec + p.global_off[1])), p.global_mode);
+      if (!__all_sync(0xffffffffu, mbar_wait(d_full, i & 1))) return;   // tcgen05.ld needs the whole warp
+      tc_fence_after();
+      const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+      for (int n0 = 0; n0 < grp.z; n0 += 32) {
+        uint32_t d0[32], d1[32];
+        tmem_ld32(lane_base + n0, d0);
+        tmem_ld32(lane_base + 256 + n0, d1);
+        tmem_wait_ld();
+        const int nn = min(32, grp.z - n0);
+        if (p.gateup) {
+          __half* o = static_cast<__half*>(p.out) + (size_t)(grp.y + n0) * p.out_stride + m * kBM + t;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < nn)
+              o[(size_t)j * p.out_stride] =
+                __float2half_rn(silu_mul(__uint_as_float(d0[j]) * gm0, __uint_as_float(d1[j]) * gm1));
+        } else {
+          float* o = static_cast<float*>(p.out) + (size_t)(grp.y + n0) * p.out_stride + m * 2 * kBM + t;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (j < nn) {
+              o[(size_t)j * p.out_stride] = __uint_as_float(d0[j]) * gm0;
+              o[(size_t)j * p.out_stride + kBM] = __uint_as_float(d1[j]) * gm1;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(d_empty);
+    };
+
+    StageFrag fa, fb;                                // stages q and q + 1, loaded ahead
+    load(ltile, lc, fa);
+    advance(ltile, lc);
+    load(ltile, lc, fb);
+    advance(ltile, lc);
+    int q = 0;
+    bool ok = true;
+    const int first = nst < kStages ? nst : kStages;   // stages of a tile stored before the previous epilogue
+    for (int i = 0; i < total && ok; ++i) {
+      for (int c = 0; c < nst; ++c, ++q) {
+        const int s = q % kStages;
+        if (!mbar_wait(&empty[s], ((q / kStages) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+        StageFrag nxt;
+        load(ltile, lc, nxt);                          // stage q + 2
+        advance(ltile, lc);
+        store(s, fa);
+        fa = fb;
+        fb = nxt;
+        fence_proxy_async_smem();
+        mbar_arrive(&a_full[s]);
+        if (i > 0 && c == first - 1) epilogue(i - 1);
+      }
+    }
+    if (ok && total > 0) epilogue(total - 1);
+  } else if (warp == 4) {
+    // ------------------------------------------------------------ activation TMA
+    if (lane == 0) {
+      int q = 0;
+      bool ok = true;
+      for (int tt = blockIdx.x; tt < ntiles && ok; tt += gridDim.x) {
+        const int4 grp = __ldg(&p.groups[tt / p.tiles_per_group]);
+        const int nbox = (grp.z + kBoxRows - 1) / kBoxRows;
+        for (int c = 0; c < nst; ++c, ++q) {
+          const int s = q % kStages;
+          if (!mbar_wait(&empty[s], ((q / kStages) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&b_full[s], nbox * kBoxRows * kKC * 2);
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d(sB + s * kBBytes + b * kBoxRows * kKC * 2, &xmap, c * kKC, grp.y + b * kBoxRows, &b_full[s]);
+        }
+      }
+      for (int j = max(0, q - kStages); j < q; ++j) mbar_wait(&b_full[j % kStages], (j / kStages) & 1);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      int q = 0, i = 0;
+      bool ok = true;
+      for (int tt = blockIdx.x; tt < ntiles && ok; tt += gridDim.x, ++i) {
+        const int4 grp = __ldg(&p.groups[tt / p.tiles_per_group]);
+        const int N = (grp.z + 15) & ~15;
+        const uint32_t idesc = idesc_f16(kBM, N);
+        if (i > 0 && !mbar_wait(d_empty, (i - 1) & 1)) break;
+        tc_fence_after();
+        for (int c = 0; c < nst; ++c, ++q) {
+          const int s = q % kStages;
+          const uint32_t ph = (q / kStages) & 1;
+          if (!mbar_wait(&a_full[s], ph) || !mbar_wait(&b_full[s], ph)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b0 = smem_addr(sB + s * kBBytes);
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            const uint32_t a0 = smem_addr(sA + (s * 2 + mt) * kABytes);
+#pragma unroll
+            for (int k = 0; k < kKC / 16; ++k)
+              tc_mma_f16(tmem + mt * 256, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), idesc,
+                         (c | k) != 0);
+          }
+          tc_commit(&empty[s]);
+        }
+        if (ok) tc_commit(d_full);
+      }
+      // Do not free tensor memory while MMAs may still run (matters only on the error path).
+      if (q > 0) mbar_wait(&empty[(q - 1) % kStages], ((q - 1) / kStages) & 1);
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Gathers the routed rows of x (bf16 [T, H]) in expert order into f16 [R, H].
+__global__ void gather_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int k, int64_t R,
+                              int H, __half* __restrict__ xp) {
+  const int per = H / 8;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= R * per) return;
+  const int64_t r = i / per;
+  const int c = (int)(i - r * per) * 8;
+  const int t = perm[r] / k;
+  const uint4 b = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + c));
+  uint4 o;
+  o.x = pack_f16x2(bf16_bits_to_f32(b.x & 0xFFFF), bf16_bits_to_f32(b.x >> 16));
+  o.y = pack_f16x2(bf16_bits_to_f32(b.y & 0xFFFF), bf16_bits_to_f32(b.y >> 16));
+  o.z = pack_f16x2(bf16_bits_to_f32(b.z & 0xFFFF), bf16_bits_to_f32(b.z >> 16));
+  o.w = pack_f16x2(bf16_bits_to_f32(b.w & 0xFFFF), bf16_bits_to_f32(b.w >> 16));
+  *reinterpret_cast<uint4*>(xp + r * H + c) = o;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (EncodeTiledFn) nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// Tensor map over a row-major f16 matrix [rows, cols]: boxes of 64 columns x 64 rows, 128B swizzle.
+int make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return -(int)cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {kKC, kBoxRows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -(int)cudaErrorInvalidValue;
+}
+
+int launch_prefill(const PrefillParams& p, const CUtensorMap& map, int num_sms, cudaStream_t s) {
+  cudaError_t err = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (err != cudaSuccess) return -(int)err;
+  prefill_kernel<<<num_sms, kThreads, kSmemBytes, s>>>(map, p);
+  err = cudaGetLastError();
+  return err == cudaSuccess ? 1 : -(int)err;
+}
+
+}  // namespace
+
+bool prefill_supported(int H, int I) { return H % 256 == 0 && I % 128 == 0 && H % kKC == 0 && I % kKC == 0; }
+
+int launch_gather(const uint16_t* x, const int32_t* perm, int k, int64_t R, int H, void* xp, cudaStream_t s) {
+  const int64_t n = R * (H / 8);
+  gather_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(x, perm, k, R, H, static_cast<__half*>(xp));
+  const cudaError_t err = cudaGetLastError();
+  return err == cudaSuccess ? 1 : -(int)err;
+}
+
+int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const RouteBufs& rb, void* h16,
+                          int num_sms, cudaStream_t s) {
+  CUtensorMap map;
+  int rc = make_rows_map(&map, xp, R, bank.H);
+  if (rc) return rc;
+  PrefillParams p{};
+  p.bank = bank.base;
+  p.stride = bank.stride;
+  for (int m = 0; m < 2; ++m) {
+    p.codes_off[m] = bank.codes_off[m];
+    p.scales_off[m] = bank.scales_off[m];
+    p.global_off[m] = bank.global_off[m];
+  }
+  p.global_mode = bank.global_mode;
+  p.K = bank.H;
+  p.tiles_per_group = bank.I / kBM;
+  p.gateup = 1;
+  p.groups = rb.groups;
+  p.ngroups = rb.ngroups;
+  p.out = h16;
+  p.out_stride = bank.I;
+  return launch_prefill(p, map, num_sms, s);
+}
+
+int launch_prefill_down(const BankView& bank, const void* h16, int64_t R, const RouteBufs& rb, float* y,
+                        int num_sms, cudaStream_t s) {
+  CUtensorMap map;
+  int rc = make_rows_map(&map, h16, R, bank.I);
+  if (rc) return rc;
+  PrefillParams p{};
+  p.bank = bank.base;
+  p.stride = bank.stride;
+  for (int m = 0; m < 2; ++m) {
+    p.codes_off[m] = bank.codes_off[2];
+    p.scales_off[m] = bank.scales_off[2];
+    p.global_off[m] = bank.global_off[2];
+  }
+  p.global_mode = bank.global_mode;
+  p.K = bank.I;
+  p.tiles_per_group = bank.H / (2 * kBM);
+  p.gateup = 0;
+  p.groups = rb.groups;
+  p.ngroups = rb.ngroups;
+  p.out = y;
+  p.out_stride = bank.H;
+  return launch_prefill(p, map, num_sms, s);
+}
+
+}  // namespace moe

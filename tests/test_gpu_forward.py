@@ -11,7 +11,8 @@ from gpu_helpers import bf16_tensor, bits_of, device_bank, pool_map
 
 pytestmark = pytest.mark.gpu
 
-PATHS = ["auto", "decode"]
+PATHS = ["auto", "decode", "prefill"]
+_ORACLE_CACHE = {}
 
 
 def _run(cfg, bank, xb, lg, path="auto", x_next=False):
@@ -36,42 +37,69 @@ def _oracle(cfg, xb, lg, layer=0, tokens=None, global_mode=0, seed=None):
 @pytest.mark.parametrize("name", ["tiny", "decode_t1", "decode_t64_zipf", "prefill_t8192"])
 def test_layer_matches_oracle(name, path):
     cfg = moe_inputs.CONFIGS[name]
-    if name == "prefill_t8192" and path == "decode":
-        pytest.skip("auto covers the large-T decode launch here")
     buf, bank = device_bank(cfg)
     xb, lg = moe_inputs.make_x(cfg), moe_inputs.make_logits(cfg)
     out, _ = _run(cfg, bank, xb, lg, path)
     tokens = moe_inputs.sample_tokens(cfg.T, 512, cfg.seed)
-    ref = _oracle(cfg, xb, lg, tokens=tokens)
-    assert_layer_close(oracle.bf16_bits_to_f64(out[tokens]), ref["out"], f"{name}/{path}")
+    if name not in _ORACLE_CACHE:
+        _ORACLE_CACHE[name] = _oracle(cfg, xb, lg, tokens=tokens)["out"]
+    assert_layer_close(oracle.bf16_bits_to_f64(out[tokens]), _ORACLE_CACHE[name], f"{name}/{path}")
 
 
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("T", [1, 2, 3, 8, 9, 13, 64, 65, 100])
-def test_tiny_ragged_T(T):
+def test_tiny_ragged_T(T, path):
     base = moe_inputs.CONFIGS["tiny"]
     cfg = moe_inputs.LayerConfig("tiny_T", base.E, base.k, base.H, base.I, T, 1, "distinct", seed=T)
     buf, bank = device_bank(cfg)
     xb, lg = moe_inputs.make_x(cfg), moe_inputs.make_logits(cfg)
-    out, _ = _run(cfg, bank, xb, lg)
-    assert_layer_close(oracle.bf16_bits_to_f64(out), _oracle(cfg, xb, lg)["out"], f"T={T}")
+    out, _ = _run(cfg, bank, xb, lg, path)
+    assert_layer_close(oracle.bf16_bits_to_f64(out), _oracle(cfg, xb, lg)["out"], f"T={T}/{path}")
 
 
+def _prefill_shape_ok(H, I):
+    return H % 256 == 0 and I % 128 == 0
+
+
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("E,k,H,I,T", [(16, 1, 256, 128, 5), (16, 16, 256, 128, 6), (64, 4, 384, 256, 40),
                                        (8, 2, 128, 128, 3), (32, 8, 1024, 512, 20)])
-def test_shapes(E, k, H, I, T):
+def test_shapes(E, k, H, I, T, path):
+    import nvfp4_weight_only_top_b200 as moe
     cfg = moe_inputs.LayerConfig("shape", E, k, H, I, T, 1, "normal", seed=E + H)
     buf, bank = device_bank(cfg)
     xb, lg = moe_inputs.make_x(cfg), moe_inputs.make_logits(cfg)
-    out, _ = _run(cfg, bank, xb, lg)
-    assert_layer_close(oracle.bf16_bits_to_f64(out), _oracle(cfg, xb, lg)["out"], f"{E},{k},{H},{I},{T}")
+    if path == "prefill" and not _prefill_shape_ok(H, I):
+        with pytest.raises(moe.MoeError) as ei:
+            _run(cfg, bank, xb, lg, path)
+        assert ei.value.code == -2 and "prefill" in str(ei.value)
+        return
+    out, _ = _run(cfg, bank, xb, lg, path)
+    assert_layer_close(oracle.bf16_bits_to_f64(out), _oracle(cfg, xb, lg)["out"], f"{E},{k},{H},{I},{T}/{path}")
 
 
-def test_global_mode_1():
+@pytest.mark.parametrize("E,k,H,I,T,dist", [
+    (8, 2, 256, 128, 1100, "normal"),      # about 275 rows per expert: groups of 256 plus a ragged group
+    (4, 4, 512, 256, 600, "normal"),       # every expert takes 600 rows: 256 + 256 + 88
+    (16, 2, 768, 384, 300, "zipf"),        # skewed counts, K = 768 / 384: many stages, 3 M-tile pairs
+    (2, 1, 256, 128, 520, "normal")])      # two experts, groups of 1..256 rows
+def test_prefill_groups_beyond_one_tile(E, k, H, I, T, dist):
+    cfg = moe_inputs.LayerConfig("prefill_groups", E, k, H, I, T, 1, dist, seed=T + H)
+    buf, bank = device_bank(cfg)
+    xb, lg = moe_inputs.make_x(cfg), moe_inputs.make_logits(cfg)
+    ref = _oracle(cfg, xb, lg)["out"]
+    for path in ("prefill", "decode"):
+        out, _ = _run(cfg, bank, xb, lg, path)
+        assert_layer_close(oracle.bf16_bits_to_f64(out), ref, f"{E},{k},{H},{I},{T}/{path}")
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_global_mode_1(path):
     cfg = moe_inputs.CONFIGS["tiny"]
     buf, bank = device_bank(cfg, global_mode=1)
     xb, lg = moe_inputs.make_x(cfg), moe_inputs.make_logits(cfg)
-    out, _ = _run(cfg, bank, xb, lg)
-    assert_layer_close(oracle.bf16_bits_to_f64(out), _oracle(cfg, xb, lg, global_mode=1)["out"], "mode1")
+    out, _ = _run(cfg, bank, xb, lg, path)
+    assert_layer_close(oracle.bf16_bits_to_f64(out), _oracle(cfg, xb, lg, global_mode=1)["out"], f"mode1/{path}")
 
 
 def test_T0_enqueues_nothing():
