@@ -337,13 +337,26 @@ def main():
     kinds = {k: v for k, v in prof.items()}
     dom = max(kinds, key=lambda k: kinds[k][0])
     dom_ms = kinds[dom][0] / kinds[dom][1]
-    dom_bytes = {"decode_gateup": gu_bytes, "decode_down": dn_bytes}.get(dom, gu_bytes)
-    achieved = dom_bytes / (dom_ms / 1000.0) / 1e9
     total_ms = sum(v[0] for v in kinds.values())
-    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json)",
-                "traffic": kernel_traffic(dom, cfg.name), "algorithmic_bytes_per_launch": dom_bytes,
-                "avg_launch_us": dom_ms * 1000.0}
+    if dom.startswith("prefill_") and dom != "prefill_gather":
+        # tensor-core bound: algorithmic FLOPs of the routed rows (2 per multiply-add)
+        flops = 2.0 * R * cfg.H * 2 * cfg.I if dom == "prefill_gateup" else 2.0 * R * cfg.I * cfg.H
+        achieved = flops / (dom_ms / 1000.0) / 1e12
+        pb = {"prefill_gateup": avg_touched * 2 * proj_bytes(cfg.I, cfg.H) + R * cfg.H * 2 + R * cfg.I * 2,
+              "prefill_down": avg_touched * proj_bytes(cfg.H, cfg.I) + R * cfg.I * 2 + R * cfg.H * 4}[dom]
+        roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s",
+                    "frac": achieved / tf_burst, "frac_of_sustained": achieved / tf_sus,
+                    "peak_source": f"{peak_kind} dense BF16 cuBLAS burst (MEASURED_PEAKS.json); the kernel "
+                                   "computes in F16, whose nominal tensor rate equals BF16's (ratio 1)",
+                    "traffic": kernel_traffic(dom, cfg.name), "algorithmic_flops_per_launch": flops,
+                    "algorithmic_bytes_per_launch": pb, "avg_launch_us": dom_ms * 1000.0}
+    else:
+        dom_bytes = {"decode_gateup": gu_bytes, "decode_down": dn_bytes}.get(dom, gu_bytes)
+        achieved = dom_bytes / (dom_ms / 1000.0) / 1e9
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                    "frac": achieved / hbm, "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json)",
+                    "traffic": kernel_traffic(dom, cfg.name), "algorithmic_bytes_per_launch": dom_bytes,
+                    "avg_launch_us": dom_ms * 1000.0}
     expert_bytes = avg_touched * (2 * proj_bytes(cfg.I, cfg.H) + proj_bytes(cfg.H, cfg.I)) * per_step_layers
     line = {
         "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": ws, "steps": steps_eff, "warmup": warm,
@@ -360,6 +373,8 @@ def main():
         "gpu_launches": launches_per_step * steps_eff,
         "e2e": e2e,
     }
+    if cfg.T * cfg.k > 8 * cfg.E:
+        line["layer_tflops"] = 2.0 * R * 3 * cfg.H * cfg.I * per_step_layers / (ms_step / 1000.0) / 1e12
     if ck is not None:
         line["clocks"] = ck
     if ws == 1:

@@ -100,8 +100,8 @@ int moe_nvfp4_forward(const void* x_dev, const float* logits_dev, int64_t T,
  *                 stacked layers; the sum of the two BF16 values rounded once);
  *  workspace_dev  caller scratch of workspace_bytes >= moe_nvfp4_workspace_bytes(...), 256-byte
  *                 aligned; if NULL the internal workspace is used;
- *  path           MOE_NVFP4_PATH_*; AUTO picks the prefill path when T*k > 8*E and H is a
- *                 multiple of 256 (I of 128), else the decode path.
+ *  path           MOE_NVFP4_PATH_*; AUTO picks the prefill path when T*k > 8*E and H and I
+ *                 are multiples of 256, else the decode path.
  * With a caller workspace nothing is allocated, so the call can be captured in a CUDA graph.
  */
 int moe_nvfp4_forward_ex(const void* x_dev, const float* logits_dev, int64_t T,

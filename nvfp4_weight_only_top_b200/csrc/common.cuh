@@ -158,6 +158,10 @@ __device__ __forceinline__ void mma_16816(float c[4], const uint32_t a[4], uint3
 // SwiGLU of one pair: silu(g) * u = g / (1 + e^-g) * u, in f32.
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
+// SwiGLU with the hardware exponential and fast division (a few ulp; used where the result is
+// rounded to f16 right after).
+__device__ __forceinline__ float silu_mul_fast(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+
 // Multiplier of a projection's stored global: mode 0 the value itself, mode 1 f32(g / 2688).
 __device__ __forceinline__ float global_mult(float g, int mode) {
   return mode == 1 ? __fdiv_rn(g, 2688.0f) : g;
@@ -224,6 +228,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int x, i
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
           "r"(smem_addr(dst)),
       "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// 3-D tiled TMA load of box (x, y, z) of `map` into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_addr(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
       : "memory");
 }
 

@@ -262,7 +262,7 @@ int check_k_T(int64_t T, int E, int k) {
 }
 
 // AUTO takes the tensor-core path once experts average more than 8 routed rows and the
-// shapes allow it (H a multiple of 256, I of 128).
+// shapes allow it (H and I multiples of 256).
 int resolve_path(int path, int64_t T, int k, int E, int H, int I) {
   if (path != MOE_NVFP4_PATH_AUTO) return path;
   return (T * k > (int64_t)8 * E && moe::prefill_supported(H, I)) ? MOE_NVFP4_PATH_PREFILL
@@ -340,7 +340,7 @@ int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
   const int use = resolve_path(path, T, k, E, H, I);
   if (use == MOE_NVFP4_PATH_PREFILL) {
     if (!moe::prefill_supported(H, I))
-      return fail(MOE_NVFP4_ERR_UNSUPPORTED, "prefill path needs H %% 256 == 0 and I %% 128 == 0 (H=%d, I=%d)", H,
+      return fail(MOE_NVFP4_ERR_UNSUPPORTED, "prefill path needs H %% 256 == 0 and I %% 256 == 0 (H=%d, I=%d)", H,
                   I);
     return prefill_impl(x, logits, T, bank, k, out, x_next, workspace, workspace_bytes, stream, dev, info);
   }

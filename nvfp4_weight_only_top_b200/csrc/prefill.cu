@@ -5,15 +5,19 @@
 // in the epilogue), for down 256 consecutive rows of Wd.  The two M-tiles share every tile of
 // activations, halving activation traffic per FLOP.
 //
-// Per CTA (one per SM, persistent over tiles): warps 0-3 dequantize -- each thread owns one
-// weight row of each M-tile, streams its codes and scales from HBM with 128-bit loads two
-// stages ahead, converts E2M1 with cvt and multiplies by the E4M3 block scale in f16 (exact),
-// and stores the f16 row chunk into a 128-byte-swizzled K-major shared-memory stage; warp 4
-// loads the group's activation rows (f16, expert-permuted) with 2-D TMA into swizzled stages;
-// warp 5 issues tcgen05.mma kind::f16 (M = 128, N = rows of the group rounded up to 16,
-// K = 16) into two f32 accumulators in tensor memory and releases each stage with
-// tcgen05.commit.  After a tile's last K stage, warps 0-3 read the accumulators back with
-// tcgen05.ld and apply the global scale (and SwiGLU for gate/up).
+// Per CTA (one per SM, persistent over tiles), warp-specialised, all hand-offs on mbarriers:
+//   warp 6 (one thread): 3-D TMA of the raw NVFP4 tiles -- codes 128 rows x 32 B per M-tile and
+//       stage, E4M3 scales 128 rows x 16 B per M-tile every 4 stages -- straight out of the
+//       bank (dims: bytes of a row, rows, expert), so weight bytes cross the L1 once, in bulk;
+//   warps 0-3 (one thread per weight row of each M-tile): read their row's codes and scales
+//       from shared memory, convert E2M1 with cvt, multiply by the block scale in f16 (exact)
+//       and store the f16 row chunk into a 128-byte-swizzled K-major operand stage;
+//   warp 4 (one thread): 2-D TMA of the group's activation rows (f16, expert order) into
+//       swizzled stages;
+//   warp 5 (one thread): tcgen05.mma kind::f16 (M = 128, N = rows of the group rounded up to
+//       16, K = 16) into two f32 accumulators in tensor memory; tcgen05.commit frees a stage.
+// After a tile's last K stage warps 0-3 read the accumulators back with tcgen05.ld and apply
+// the global scale (and SwiGLU for gate/up).
 //
 // Weight layout: page "Beam 1.0 501B-A23B, streaming pack, NVFP4 experts / MLX 8-bit
 // residents", section "What this pack holds"; SwiGLU in FP32: page "Beam-1.0-501B-A23B VQ
@@ -32,42 +36,56 @@ namespace {
 
 constexpr int kBM = 128;                       // rows per MMA M-tile
 constexpr int kKC = 64;                        // K per stage: one 128-byte swizzle row of f16
-constexpr int kStages = 3;
+constexpr int kStages = 3;                     // operand stages (A f16 + B f16)
+constexpr int kWStages = 3;                    // raw code stages
+constexpr int kSStages = 2;                    // raw scale stages (4 operand stages each)
 constexpr int kMaxN = 256;
 constexpr int kBoxRows = 64;                   // activation rows per TMA box
-constexpr int kThreads = 32 * 6;               // 4 dequant/epilogue warps, TMA warp, MMA warp
+constexpr int kThreads = 32 * 7;
 constexpr int kABytes = kBM * kKC * 2;         // 16 KB: one M-tile of one stage
 constexpr int kBBytes = kMaxN * kKC * 2;       // 32 KB: activations of one stage
+constexpr int kWBytes = kBM * kKC / 2;         // 4 KB: codes of one M-tile of one stage
+constexpr int kSBytes = kBM * 16;              // 2 KB: scales of one M-tile, 4 stages
 constexpr int kTmemCols = 512;                 // two 256-column f32 accumulators
-constexpr int kSmemBytes = kStages * (2 * kABytes + kBBytes) + 1024 /*barriers*/ + 1024 /*align*/;
+constexpr int kOffB = kStages * 2 * kABytes;
+constexpr int kOffW = kOffB + kStages * kBBytes;
+constexpr int kOffS = kOffW + kWStages * 2 * kWBytes;
+constexpr int kOffBar = kOffS + kSStages * 2 * kSBytes;
+constexpr int kSmemBytes = kOffBar + 256 /*barriers*/ + 1024 /*alignment*/;
+static_assert(kSmemBytes <= 232448, "shared memory per block");
 
 struct PrefillParams {
   const uint8_t* bank;
   uint64_t stride;
-  uint64_t codes_off[2], scales_off[2], global_off[2];  // matrix of M-tile 0 / M-tile 1
+  uint64_t global_off[2];  // global scale of the matrix of M-tile 0 / M-tile 1
   int global_mode;
-  int K;                 // inputs per weight row
-  int tiles_per_group;   // output-row tiles per group
-  int gateup;            // 1: M-tile 0 = gate rows, M-tile 1 = same up rows; 0: 256 consecutive rows
-  const int4* groups;    // (expert, first permuted row, rows <= 256, 0)
+  int K;                   // inputs per weight row
+  int tiles_per_group;     // output-row tiles per group
+  int gateup;              // 1: M-tile 0 = gate rows, M-tile 1 = same up rows; 0: 256 consecutive rows
+  const int4* groups;      // (expert, first permuted row, rows <= 256, 0)
   const int32_t* ngroups;
-  void* out;             // gate/up: h f16 [R, out_stride]; down: y f32 [R, out_stride]
+  void* out;               // gate/up: h f16 [R, out_stride]; down: y f32 [R, out_stride]
   int out_stride;
 };
 
-__device__ __forceinline__ uint4 ld_v4_nc(const uint8_t* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
-}
-__device__ __forceinline__ uint32_t ld_u32_nc(const uint8_t* p) {
-  uint32_t v;
-  asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
-}
+struct Maps {
+  CUtensorMap x;           // activations [R, K] f16
+  CUtensorMap codes[2];    // codes of the M-tile 0 / 1 matrix: [E][rows][K/2] bytes
+  CUtensorMap scales[2];   // scales: [E][rows][K/16] bytes
+};
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
 }
 
 // One thread's share of one stage: 64 codes and 4 scale bytes of each of its two rows.
@@ -76,29 +94,59 @@ struct StageFrag {
   uint32_t s[2];
 };
 
+// Maps a CTA-local tile number to (group, output-row tile).
+struct TileCursor {
+  int tiles_per_group;
+  __device__ __forceinline__ void at(int tt, int& g, int& m) const {
+    g = tt / tiles_per_group;
+    m = tt - g * tiles_per_group;
+  }
+};
+
+__device__ __forceinline__ int row0_of(const PrefillParams& p, int m, int mt) {
+  return p.gateup ? m * kBM : m * 2 * kBM + mt * kBM;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap xmap, const PrefillParams p) {
+    prefill_kernel(const __grid_constant__ Maps maps, const PrefillParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint8_t* sA = smem;                                   // [stage][m-tile] 16 KB each
-  uint8_t* sB = smem + kStages * 2 * kABytes;           // [stage] 32 KB each
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * kBBytes);
-  uint64_t* a_full = bars;
-  uint64_t* b_full = bars + kStages;
-  uint64_t* empty = bars + 2 * kStages;
-  uint64_t* d_full = bars + 3 * kStages;
-  uint64_t* d_empty = d_full + 1;
+  uint8_t* sA = smem;                                   // [stage][m-tile] 16 KB, 128B-swizzled
+  uint8_t* sB = smem + kOffB;                           // [stage] 32 KB, 128B-swizzled
+  uint8_t* sW = smem + kOffW;                           // [stage][m-tile] 128 rows x 32 B
+  uint8_t* sS = smem + kOffS;                           // [stage][m-tile] 128 rows x 16 B
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* a_full = bars;                              // [kStages] producers -> MMA
+  uint64_t* b_full = a_full + kStages;                  // [kStages] TMA -> MMA
+  uint64_t* empty = b_full + kStages;                   // [kStages] MMA commit -> producers, TMA
+  uint64_t* w_full = empty + kStages;                   // [kWStages] TMA -> producers
+  uint64_t* w_empty = w_full + kWStages;                // [kWStages] producers -> TMA
+  uint64_t* s_full = w_empty + kWStages;                // [kSStages]
+  uint64_t* s_empty = s_full + kSStages;                // [kSStages]
+  uint64_t* d_full = s_empty + kSStages;                // MMA commit -> epilogue
+  uint64_t* d_empty = d_full + 1;                       // epilogue -> MMA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_empty + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = *p.ngroups * p.tiles_per_group;
-  const int nst = p.K / kKC;
+  const int nst = p.K / kKC;                            // stages per tile (a multiple of 4)
+  const int total = (ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;  // tiles of this CTA
+  const int nq = total * nst;
+  const TileCursor cur{p.tiles_per_group};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&a_full[s], 4 * 32);
       mbar_init(&b_full[s], 1);
       mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < kWStages; ++s) {
+      mbar_init(&w_full[s], 1);
+      mbar_init(&w_empty[s], 4 * 32);
+    }
+    for (int s = 0; s < kSStages; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], 4 * 32);
     }
     mbar_init(d_full, 1);
     mbar_init(d_empty, 4 * 32);
@@ -115,28 +163,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     // ------------------------------------------------------------ dequant + epilogue
     const int t = threadIdx.x;                      // weight row within each M-tile
-    const uint32_t rowb = p.K / 2, scb = p.K / 16;
-    const int total = ((ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x);  // tiles of this CTA
-    // Load cursor (two stages ahead of the stage being stored).
-    int ltile = 0, lc = 0;
-    auto tile_of = [&](int i) { return (int)blockIdx.x + i * (int)gridDim.x; };
-    auto load = [&](int i, int c, StageFrag& f) {
-      if (i >= total) return;
-      const int tt = tile_of(i), g = tt / p.tiles_per_group, m = tt - g * p.tiles_per_group;
-      const uint8_t* rec = p.bank + (uint64_t)__ldg(&p.groups[g].x) * p.stride;
+    const uint32_t w_base = smem_addr(sW), s_base = smem_addr(sS);
+    // The two 16-byte halves of a 32-byte code row are read in an order that alternates every
+    // four rows, so a warp's 128-bit shared loads cover all 32 banks without conflicts.
+    const uint32_t h0 = ((t >> 2) & 1) * 16, h1 = h0 ^ 16;
+    auto fetch = [&](int q, StageFrag& f) {        // raw stage q: shared -> registers
+      const int c = q % nst;
+      const int ws = q % kWStages, ss = (q >> 2) % kSStages;
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
-        const uint64_t row = p.gateup ? (uint64_t)m * kBM + t : (uint64_t)m * 2 * kBM + mt * kBM + t;
-        const uint8_t* cp = rec + p.codes_off[mt] + row * rowb + c * (kKC / 2);
-        f.c[mt][0] = ld_v4_nc(cp);
-        f.c[mt][1] = ld_v4_nc(cp + 16);
-        f.s[mt] = ld_u32_nc(rec + p.scales_off[mt] + row * scb + c * (kKC / 16));
-      }
-    };
-    auto advance = [&](int& i, int& c) {
-      if (++c == nst) {
-        c = 0;
-        ++i;
+        const uint32_t row = w_base + (ws * 2 + mt) * kWBytes + t * 32;
+        const uint4 u = ld_shared_v4(row + h0), v = ld_shared_v4(row + h1);
+        f.c[mt][0] = h0 ? v : u;
+        f.c[mt][1] = h0 ? u : v;
+        f.s[mt] = ld_shared_u32(s_base + (ss * 2 + mt) * kSBytes + t * 16 + (c & 3) * 4);
       }
     };
     auto store = [&](int s, const StageFrag& f) {
@@ -160,7 +200,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     auto epilogue = [&](int i) {
-      const int tt = tile_of(i), g = tt / p.tiles_per_group, m = tt - g * p.tiles_per_group;
+      int g, m;
+      cur.at((int)blockIdx.x + i * (int)gridDim.x, g, m);
       const int4 grp = __ldg(&p.groups[g]);
       const uint8_t* rec = p.bank + (uint64_t)grp.x * p.stride;
       const float gm0 = global_mult(__ldg(reinterpret_cast<const float*>(rec + p.global_off[0])), p.global_mode);
@@ -180,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 32; ++j)
             if (j < nn)
               o[(size_t)j * p.out_stride] =
-                __float2half_rn(silu_mul(__uint_as_float(d0[j]) * gm0, __uint_as_float(d1[j]) * gm1));
+                  __float2half_rn(silu_mul_fast(__uint_as_float(d0[j]) * gm0, __uint_as_float(d1[j]) * gm1));
         } else {
           float* o = static_cast<float*>(p.out) + (size_t)(grp.y + n0) * p.out_stride + m * 2 * kBM + t;
 #pragma unroll
@@ -196,31 +237,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(d_empty);
     };
 
-    StageFrag fa, fb;                                // stages q and q + 1, loaded ahead
-    load(ltile, lc, fa);
-    advance(ltile, lc);
-    load(ltile, lc, fb);
-    advance(ltile, lc);
-    int q = 0;
     bool ok = true;
     const int first = nst < kStages ? nst : kStages;   // stages of a tile stored before the previous epilogue
-    for (int i = 0; i < total && ok; ++i) {
-      for (int c = 0; c < nst; ++c, ++q) {
-        const int s = q % kStages;
-        if (!mbar_wait(&empty[s], ((q / kStages) & 1) ^ 1)) {
-          ok = false;
-          break;
-        }
-        StageFrag nxt;
-        load(ltile, lc, nxt);                          // stage q + 2
-        advance(ltile, lc);
-        store(s, fa);
-        fa = fb;
-        fb = nxt;
-        fence_proxy_async_smem();
-        mbar_arrive(&a_full[s]);
-        if (i > 0 && c == first - 1) epilogue(i - 1);
+    for (int q = 0; q < nq && ok; ++q) {
+      const int c = q % nst;
+      const int ws = q % kWStages, ss = (q >> 2) % kSStages;
+      if (!mbar_wait(&w_full[ws], (q / kWStages) & 1) ||
+          ((c & 3) == 0 && !mbar_wait(&s_full[ss], ((q >> 2) / kSStages) & 1))) {
+        ok = false;
+        break;
       }
+      StageFrag f;
+      fetch(q, f);
+      const int s = q % kStages;
+      if (!mbar_wait(&empty[s], ((q / kStages) & 1) ^ 1)) {
+        ok = false;
+        break;
+      }
+      store(s, f);
+      fence_proxy_async_smem();
+      mbar_arrive(&a_full[s]);
+      // The raw slots go back to the TMA only after the proxy fence above: a TMA write (async
+      // proxy) into a slot that this thread read with generic loads must be ordered after
+      // those reads, or it can overtake them.
+      mbar_arrive(&w_empty[ws]);
+      if ((c & 3) == 3) mbar_arrive(&s_empty[ss]);
+      const int i = q / nst;
+      if (i > 0 && c == first - 1) epilogue(i - 1);
     }
     if (ok && total > 0) epilogue(total - 1);
   } else if (warp == 4) {
@@ -239,10 +282,50 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(&b_full[s], nbox * kBoxRows * kKC * 2);
           for (int b = 0; b < nbox; ++b)
-            tma_load_2d(sB + s * kBBytes + b * kBoxRows * kKC * 2, &xmap, c * kKC, grp.y + b * kBoxRows, &b_full[s]);
+            tma_load_2d(sB + s * kBBytes + b * kBoxRows * kKC * 2, &maps.x, c * kKC, grp.y + b * kBoxRows,
+                        &b_full[s]);
         }
       }
       for (int j = max(0, q - kStages); j < q; ++j) mbar_wait(&b_full[j % kStages], (j / kStages) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ weight TMA
+    if (lane == 0) {
+      bool ok = true;
+      int q = 0, qs = 0;
+      for (; q < nq && ok; ++q) {
+        const int i = q / nst, c = q - i * nst;
+        int g, m;
+        cur.at((int)blockIdx.x + i * (int)gridDim.x, g, m);
+        const int e = __ldg(&p.groups[g].x);
+        if ((c & 3) == 0) {                       // scales of stages c .. c+3
+          const int ss = qs % kSStages;
+          if (!mbar_wait(&s_empty[ss], ((qs / kSStages) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&s_full[ss], 2 * kSBytes);
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt)
+            tma_load_3d(sS + (ss * 2 + mt) * kSBytes, &maps.scales[mt], (c >> 2) * 16, row0_of(p, m, mt), e,
+                        &s_full[ss]);
+          ++qs;
+        }
+        const int ws = q % kWStages;
+        if (!mbar_wait(&w_empty[ws], ((q / kWStages) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&w_full[ws], 2 * kWBytes);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+          tma_load_3d(sW + (ws * 2 + mt) * kWBytes, &maps.codes[mt], c * (kKC / 2), row0_of(p, m, mt), e,
+                      &w_full[ws]);
+      }
+      // Leave no copy in flight (only an error path gets here with copies outstanding).
+      for (int j = max(0, q - kWStages); j < q; ++j) mbar_wait(&w_full[j % kWStages], (j / kWStages) & 1);
+      for (int j = max(0, qs - kSStages); j < qs; ++j) mbar_wait(&s_full[j % kSStages], (j / kSStages) & 1);
     }
     __syncwarp();
   } else {
@@ -337,17 +420,44 @@ int make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int cols) {
   return r == CUDA_SUCCESS ? 0 : -(int)cudaErrorInvalidValue;
 }
 
-int launch_prefill(const PrefillParams& p, const CUtensorMap& map, int num_sms, cudaStream_t s) {
+// Tensor map over one byte matrix of every record: [E][rows][row_bytes] with the record stride
+// between experts; boxes of box_bytes x 128 rows x 1 expert, no swizzle.
+int make_bank_map(CUtensorMap* map, const BankView& bank, uint64_t off, int rows, int row_bytes, int box_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return -(int)cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {(cuuint64_t)row_bytes, (cuuint64_t)rows, (cuuint64_t)bank.E};
+  const cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)bank.stride};
+  const cuuint32_t box[3] = {(cuuint32_t)box_bytes, (cuuint32_t)kBM, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(bank.base + off), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -(int)cudaErrorInvalidValue;
+}
+
+int launch_prefill(const PrefillParams& p, const Maps& maps, int num_sms, cudaStream_t s) {
   cudaError_t err = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (err != cudaSuccess) return -(int)err;
-  prefill_kernel<<<num_sms, kThreads, kSmemBytes, s>>>(map, p);
+  prefill_kernel<<<num_sms, kThreads, kSmemBytes, s>>>(maps, p);
   err = cudaGetLastError();
   return err == cudaSuccess ? 1 : -(int)err;
 }
 
+// Weight maps of the two M-tile matrices (proj0, proj1) whose rows hold K inputs.
+int make_weight_maps(Maps* maps, const BankView& bank, int proj0, int proj1, int rows, int K) {
+  const int projs[2] = {proj0, proj1};
+  for (int mt = 0; mt < 2; ++mt) {
+    int rc = make_bank_map(&maps->codes[mt], bank, bank.codes_off[projs[mt]], rows, K / 2, kKC / 2);
+    if (rc) return rc;
+    rc = make_bank_map(&maps->scales[mt], bank, bank.scales_off[projs[mt]], rows, K / 16, 16);
+    if (rc) return rc;
+  }
+  return 0;
+}
+
 }  // namespace
 
-bool prefill_supported(int H, int I) { return H % 256 == 0 && I % 128 == 0 && H % kKC == 0 && I % kKC == 0; }
+bool prefill_supported(int H, int I) { return H % 256 == 0 && I % 256 == 0; }
 
 int launch_gather(const uint16_t* x, const int32_t* perm, int k, int64_t R, int H, void* xp, cudaStream_t s) {
   const int64_t n = R * (H / 8);
@@ -358,17 +468,15 @@ int launch_gather(const uint16_t* x, const int32_t* perm, int k, int64_t R, int 
 
 int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const RouteBufs& rb, void* h16,
                           int num_sms, cudaStream_t s) {
-  CUtensorMap map;
-  int rc = make_rows_map(&map, xp, R, bank.H);
+  Maps maps;
+  int rc = make_rows_map(&maps.x, xp, R, bank.H);
+  if (!rc) rc = make_weight_maps(&maps, bank, 0, 1, bank.I, bank.H);
   if (rc) return rc;
   PrefillParams p{};
   p.bank = bank.base;
   p.stride = bank.stride;
-  for (int m = 0; m < 2; ++m) {
-    p.codes_off[m] = bank.codes_off[m];
-    p.scales_off[m] = bank.scales_off[m];
-    p.global_off[m] = bank.global_off[m];
-  }
+  p.global_off[0] = bank.global_off[0];
+  p.global_off[1] = bank.global_off[1];
   p.global_mode = bank.global_mode;
   p.K = bank.H;
   p.tiles_per_group = bank.I / kBM;
@@ -377,22 +485,20 @@ int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const
   p.ngroups = rb.ngroups;
   p.out = h16;
   p.out_stride = bank.I;
-  return launch_prefill(p, map, num_sms, s);
+  return launch_prefill(p, maps, num_sms, s);
 }
 
 int launch_prefill_down(const BankView& bank, const void* h16, int64_t R, const RouteBufs& rb, float* y,
                         int num_sms, cudaStream_t s) {
-  CUtensorMap map;
-  int rc = make_rows_map(&map, h16, R, bank.I);
+  Maps maps;
+  int rc = make_rows_map(&maps.x, h16, R, bank.I);
+  if (!rc) rc = make_weight_maps(&maps, bank, 2, 2, bank.H, bank.I);
   if (rc) return rc;
   PrefillParams p{};
   p.bank = bank.base;
   p.stride = bank.stride;
-  for (int m = 0; m < 2; ++m) {
-    p.codes_off[m] = bank.codes_off[2];
-    p.scales_off[m] = bank.scales_off[2];
-    p.global_off[m] = bank.global_off[2];
-  }
+  p.global_off[0] = bank.global_off[2];
+  p.global_off[1] = bank.global_off[2];
   p.global_mode = bank.global_mode;
   p.K = bank.I;
   p.tiles_per_group = bank.H / (2 * kBM);
@@ -401,7 +507,7 @@ int launch_prefill_down(const BankView& bank, const void* h16, int64_t R, const 
   p.ngroups = rb.ngroups;
   p.out = y;
   p.out_stride = bank.H;
-  return launch_prefill(p, map, num_sms, s);
+  return launch_prefill(p, maps, num_sms, s);
 }
 
 }  // namespace moe

@@ -28,6 +28,21 @@ def _run(cfg, bank, xb, lg, path="auto", x_next=False):
     return bits_of(out), (bits_of(xn) if x_next else None)
 
 
+def _prefill_shape_ok(H, I):
+    return H % 256 == 0 and I % 256 == 0
+
+
+def _expect_unsupported(cfg, bank, xb, lg, path):
+    """True (after checking the error) when the path cannot take this shape."""
+    import nvfp4_weight_only_top_b200 as moe
+    if path != "prefill" or _prefill_shape_ok(cfg.H, cfg.I):
+        return False
+    with pytest.raises(moe.MoeError) as ei:
+        _run(cfg, bank, xb, lg, path)
+    assert ei.value.code == -2 and "prefill" in str(ei.value)
+    return True
+
+
 def _oracle(cfg, xb, lg, layer=0, tokens=None, global_mode=0, seed=None):
     src = oracle.GeneratedRecords(cfg.seed if seed is None else seed, layer, cfg.E, cfg.H, cfg.I, global_mode)
     return oracle.layer_forward(xb, lg, cfg.k, src, tokens=tokens, map_fn=pool_map)
@@ -39,6 +54,8 @@ def test_layer_matches_oracle(name, path):
     cfg = moe_inputs.CONFIGS[name]
     buf, bank = device_bank(cfg)
     xb, lg = moe_inputs.make_x(cfg), moe_inputs.make_logits(cfg)
+    if _expect_unsupported(cfg, bank, xb, lg, path):
+        return
     out, _ = _run(cfg, bank, xb, lg, path)
     tokens = moe_inputs.sample_tokens(cfg.T, 512, cfg.seed)
     if name not in _ORACLE_CACHE:
@@ -49,40 +66,35 @@ def test_layer_matches_oracle(name, path):
 @pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("T", [1, 2, 3, 8, 9, 13, 64, 65, 100])
 def test_tiny_ragged_T(T, path):
+    """The tiny layer (I = 256 on the tensor-core path, whose K-stages need I % 256 == 0)."""
     base = moe_inputs.CONFIGS["tiny"]
-    cfg = moe_inputs.LayerConfig("tiny_T", base.E, base.k, base.H, base.I, T, 1, "distinct", seed=T)
+    I = 256 if path == "prefill" else base.I
+    cfg = moe_inputs.LayerConfig("tiny_T", base.E, base.k, base.H, I, T, 1, "distinct", seed=T)
     buf, bank = device_bank(cfg)
     xb, lg = moe_inputs.make_x(cfg), moe_inputs.make_logits(cfg)
     out, _ = _run(cfg, bank, xb, lg, path)
     assert_layer_close(oracle.bf16_bits_to_f64(out), _oracle(cfg, xb, lg)["out"], f"T={T}/{path}")
 
 
-def _prefill_shape_ok(H, I):
-    return H % 256 == 0 and I % 128 == 0
-
-
 @pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("E,k,H,I,T", [(16, 1, 256, 128, 5), (16, 16, 256, 128, 6), (64, 4, 384, 256, 40),
-                                       (8, 2, 128, 128, 3), (32, 8, 1024, 512, 20)])
+                                       (8, 2, 128, 128, 3), (32, 8, 1024, 512, 20), (16, 4, 512, 256, 37),
+                                       (8, 8, 256, 768, 50), (4, 3, 1280, 256, 7)])
 def test_shapes(E, k, H, I, T, path):
-    import nvfp4_weight_only_top_b200 as moe
     cfg = moe_inputs.LayerConfig("shape", E, k, H, I, T, 1, "normal", seed=E + H)
     buf, bank = device_bank(cfg)
     xb, lg = moe_inputs.make_x(cfg), moe_inputs.make_logits(cfg)
-    if path == "prefill" and not _prefill_shape_ok(H, I):
-        with pytest.raises(moe.MoeError) as ei:
-            _run(cfg, bank, xb, lg, path)
-        assert ei.value.code == -2 and "prefill" in str(ei.value)
+    if _expect_unsupported(cfg, bank, xb, lg, path):
         return
     out, _ = _run(cfg, bank, xb, lg, path)
     assert_layer_close(oracle.bf16_bits_to_f64(out), _oracle(cfg, xb, lg)["out"], f"{E},{k},{H},{I},{T}/{path}")
 
 
 @pytest.mark.parametrize("E,k,H,I,T,dist", [
-    (8, 2, 256, 128, 1100, "normal"),      # about 275 rows per expert: groups of 256 plus a ragged group
+    (8, 2, 256, 256, 1100, "normal"),      # about 275 rows per expert: groups of 256 plus a ragged group
     (4, 4, 512, 256, 600, "normal"),       # every expert takes 600 rows: 256 + 256 + 88
-    (16, 2, 768, 384, 300, "zipf"),        # skewed counts, K = 768 / 384: many stages, 3 M-tile pairs
-    (2, 1, 256, 128, 520, "normal")])      # two experts, groups of 1..256 rows
+    (16, 2, 768, 512, 300, "zipf"),        # skewed counts, K = 768 / 512: many stages, 3-4 M-tile pairs
+    (2, 1, 256, 256, 520, "normal")])      # two experts, groups of 1..256 rows
 def test_prefill_groups_beyond_one_tile(E, k, H, I, T, dist):
     cfg = moe_inputs.LayerConfig("prefill_groups", E, k, H, I, T, 1, dist, seed=T + H)
     buf, bank = device_bank(cfg)
@@ -95,7 +107,8 @@ def test_prefill_groups_beyond_one_tile(E, k, H, I, T, dist):
 
 @pytest.mark.parametrize("path", PATHS)
 def test_global_mode_1(path):
-    cfg = moe_inputs.CONFIGS["tiny"]
+    base = moe_inputs.CONFIGS["tiny"]
+    cfg = moe_inputs.LayerConfig("tiny_mode1", base.E, base.k, base.H, 256, base.T, 1, base.logits)
     buf, bank = device_bank(cfg, global_mode=1)
     xb, lg = moe_inputs.make_x(cfg), moe_inputs.make_logits(cfg)
     out, _ = _run(cfg, bank, xb, lg, path)
@@ -182,3 +195,20 @@ def test_verify24_stack_teacher_forced():
     for l in (0, 11, 23):
         ref = _oracle(cfg, xb[l], moe_inputs.make_logits(cfg, layer=l), layer=l)
         assert_layer_close(oracle.bf16_bits_to_f64(ob[l]), ref["out"], f"layer {l}")
+
+
+def test_prefill_bitwise_repeatable():
+    """The tensor-core path has a fixed summation order: repeated calls give identical bits.  A
+    hand-off race between its producer, TMA and MMA roles shows up here as a changed column."""
+    import torch
+    import nvfp4_weight_only_top_b200 as moe
+    cfg = moe_inputs.CONFIGS["prefill_t8192"]
+    buf, bank = device_bank(cfg)
+    x = bf16_tensor(moe_inputs.make_x(cfg))
+    lg = torch.from_numpy(moe_inputs.make_logits(cfg)).cuda()
+    first = moe.moe_nvfp4_forward_ex(x, lg, bank, cfg.k, path=moe.PATH_PREFILL).view(torch.int16).clone()
+    for _ in range(6):
+        again = moe.moe_nvfp4_forward_ex(x, lg, bank, cfg.k, path=moe.PATH_PREFILL).view(torch.int16)
+        torch.cuda.synchronize()
+        assert torch.equal(first, again)
+    assert moe.moe_nvfp4_device_status() == 0
