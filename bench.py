@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--config", default="decode_t1", choices=[c for c in moe_inputs.CONFIGS if c != "tiny"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--ref-budget", type=float, default=20.0,
+                    help="seconds of oracle work for the reference arm / CPU baseline")
     return ap.parse_args()
 
 
@@ -115,19 +117,19 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def dist_init():
+def dist_init(backend: str = "nccl"):
+    """One process per GPU (torchrun env).  backend "gloo" runs the same plumbing on the CPU."""
     import torch
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if backend == "nccl":
+        torch.cuda.set_device(local)
     if ws > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(local)
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300), **kw)
     return ws, rank, local
 
 
@@ -142,12 +144,13 @@ def max_over_ranks(ws, v: float) -> float:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def cpu_oracle_baseline(cfg, budget_s: float = 20.0):
+def cpu_oracle_baseline(cfg, budget_s: float = 20.0, max_tokens: int = 64):
     """Times the FP64 oracle (as it stands) on one host core over a bounded token sample."""
     from threadpoolctl import threadpool_limits
     import oracle
@@ -165,15 +168,18 @@ def cpu_oracle_baseline(cfg, budget_s: float = 20.0):
             oracle.layer_forward(xb, lg, cfg.k, src, tokens=[t])
             tokens_done += 1
             i += 1
-            if time.perf_counter() - t0 > budget_s * 0.5 or i >= 64:
+            if time.perf_counter() - t0 > budget_s * 0.5 or i >= max_tokens:
                 break
     dt = time.perf_counter() - t0
-    return {"value": tokens_done / dt, "unit": "tok/s", "cores": 1, "kind": "oracle",
+    return {"value": tokens_done / dt, "unit": "tok/s", "cores": 1, "kind": "oracle", "tokens": tokens_done,
             "sample": f"{tokens_done} token(s) of {cfg.name}, each through the FP64 oracle "
                       f"(decode of its {cfg.k} expert records + SwiGLU + combine), {dt:.1f} s"}
 
 
 def run_reference(args):
+    """The reference arm: the FP64 oracle on the host cores.  Under torchrun only rank 0 runs;
+    the other ranks exit 0 without work.  A step is one token of the workload through the
+    oracle; the run stops after the requested steps or the time budget, whichever is first."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -181,9 +187,11 @@ def run_reference(args):
     cfg = moe_inputs.CONFIGS[args.config]
     steps = args.steps if args.steps is not None else 2
     warm = args.warmup if args.warmup is not None else 0
-    base = cpu_oracle_baseline(cfg, budget_s=20.0)
-    line = {"metric": METRIC, "value": base["value"], "unit": "tok/s", "n_gpus": args.gpus, "steps": steps,
-            "warmup": warm, "ms_per_step": 1000.0 * cfg.T / base["value"], "higher_is_better": True,
+    if warm > 0:                         # one untimed token (imports, first-touch of the records)
+        cpu_oracle_baseline(cfg, budget_s=0.0, max_tokens=1)
+    base = cpu_oracle_baseline(cfg, budget_s=args.ref_budget, max_tokens=max(1, steps))
+    line = {"metric": METRIC, "value": base["value"], "unit": "tok/s", "n_gpus": args.gpus,
+            "steps": base["tokens"], "warmup": min(warm, 1), "ms_per_step": 1000.0 * cfg.T / base["value"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference", "config": workload_config(cfg),
             "cpu_baseline": base,
@@ -347,11 +355,13 @@ def main():
         roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s",
                     "frac": achieved / tf_burst, "frac_of_sustained": achieved / tf_sus,
                     "peak_source": f"{peak_kind} dense BF16 cuBLAS burst (MEASURED_PEAKS.json); the kernel "
-                                   "computes in F16, whose nominal tensor rate equals BF16's (ratio 1)",
+                                   "computes BF16 x BF16 -> F32 on tcgen05",
                     "traffic": kernel_traffic(dom, cfg.name), "algorithmic_flops_per_launch": flops,
                     "algorithmic_bytes_per_launch": pb, "avg_launch_us": dom_ms * 1000.0}
     else:
-        dom_bytes = {"decode_gateup": gu_bytes, "decode_down": dn_bytes}.get(dom, gu_bytes)
+        fused_bytes = avg_touched * (2 * proj_bytes(cfg.I, cfg.H) + proj_bytes(cfg.H, cfg.I)) + cfg.T * cfg.E * 4 \
+            + 2 * cfg.T * cfg.H * 2
+        dom_bytes = {"decode_gateup": gu_bytes, "decode_down": dn_bytes, "decode_fused": fused_bytes}.get(dom, gu_bytes)
         achieved = dom_bytes / (dom_ms / 1000.0) / 1e9
         roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                     "frac": achieved / hbm, "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json)",
@@ -361,7 +371,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": ws, "steps": steps_eff, "warmup": warm,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f16", "data": "synthetic",
+        "dtype": "bf16" if cfg.T * cfg.k > 8 * cfg.E else "f16", "data": "synthetic",
         "config": dict(workload_config(cfg), l2="inputs larger than L2: each step reads %.0f MB of expert "
                        "records%s" % (expert_bytes / 1e6, " from experts not used in the previous %d steps"
                                       % (L2_WINDOW - 1) if cfg.name == "decode_t1" else " over rotating logit sets"),

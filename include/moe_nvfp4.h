@@ -179,6 +179,7 @@ int moe_nvfp4_last_launch_count(void);
 #define MOE_NVFP4_KERNEL_PREFILL_GATHER 4
 #define MOE_NVFP4_KERNEL_PREFILL_GATEUP 5
 #define MOE_NVFP4_KERNEL_PREFILL_DOWN   6
+#define MOE_NVFP4_KERNEL_DECODE_FUSED   7  /* single-token decode: the whole layer in one kernel */
 #define MOE_NVFP4_KERNEL_KINDS          8
 
 /*

@@ -57,7 +57,7 @@ SIGNATURES = {
 }
 
 KERNEL_KINDS = ["route", "decode_gateup", "decode_down", "combine", "prefill_gather",
-                "prefill_gateup", "prefill_down", "reserved"]
+                "prefill_gateup", "prefill_down", "decode_fused"]
 
 
 def load(path: str = LIB_PATH) -> ctypes.CDLL:

@@ -111,6 +111,40 @@ __device__ __forceinline__ void e2m1x8_to_f16x8(uint32_t w, uint32_t out[4]) {
       : "r"(w));
 }
 
+// Eight E2M1 codes (one u32, code i in bits 4i..4i+3) times an f16x2 block scale (both halves
+// equal) -> four bf16x2; out[j] holds codes 2j (low half) and 2j+1 (high half).  Exact: each
+// product has at most 5 significant bits and lies in [2^-10, 2688], so it is exact in f16, in
+// f32 and in bf16.
+__device__ __forceinline__ void e2m1x8_scaled_to_bf16x8(uint32_t w, uint32_t scale2, uint32_t out[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      ".reg .b32 h0, h1, h2, h3;\n\t"
+      ".reg .b16 l0, u0, l1, u1, l2, u2, l3, u3;\n\t"
+      ".reg .f32 a0, c0, a1, c1, a2, c2, a3, c3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h3, b3;\n\t"
+      "mul.rn.f16x2 h0, h0, %5;\n\t"
+      "mul.rn.f16x2 h1, h1, %5;\n\t"
+      "mul.rn.f16x2 h2, h2, %5;\n\t"
+      "mul.rn.f16x2 h3, h3, %5;\n\t"
+      "mov.b32 {l0, u0}, h0;\n\t"
+      "mov.b32 {l1, u1}, h1;\n\t"
+      "mov.b32 {l2, u2}, h2;\n\t"
+      "mov.b32 {l3, u3}, h3;\n\t"
+      "cvt.f32.f16 a0, l0;\n\t cvt.f32.f16 c0, u0;\n\t"
+      "cvt.f32.f16 a1, l1;\n\t cvt.f32.f16 c1, u1;\n\t"
+      "cvt.f32.f16 a2, l2;\n\t cvt.f32.f16 c2, u2;\n\t"
+      "cvt.f32.f16 a3, l3;\n\t cvt.f32.f16 c3, u3;\n\t"
+      "cvt.rn.bf16x2.f32 %0, c0, a0;\n\t"
+      "cvt.rn.bf16x2.f32 %1, c1, a1;\n\t"
+      "cvt.rn.bf16x2.f32 %2, c2, a2;\n\t"
+      "cvt.rn.bf16x2.f32 %3, c3, a3;\n\t}"
+      : "=r"(out[0]), "=r"(out[1]), "=r"(out[2]), "=r"(out[3])
+      : "r"(w), "r"(scale2));
+}
+
 // Two E4M3 bytes (low byte first) -> f16x2.  Exact (every E4M3 value is an f16 value).
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
   uint32_t r;
@@ -251,6 +285,10 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 // Instruction descriptor, kind::f16: f16 A and B, f32 accumulator, both K-major, M x N.
 __host__ __device__ __forceinline__ uint32_t idesc_f16(int M, int N) {
   return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// The same with bf16 A and B (a_format = b_format = 1).
+__host__ __device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 }  // namespace moe

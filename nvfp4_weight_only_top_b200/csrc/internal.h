@@ -67,16 +67,23 @@ int launch_combine(const float* y, const float* w, const int32_t* inv, int64_t T
 
 size_t decode_smem_bytes(int K, int xrows, bool gateup);
 
+// Decode of a single token: route, gate/up, down and combine in one persistent kernel (plus a
+// memset of the two grid-barrier counters in bar).  h [k, I] and y [k, H] are f32 scratch.
+bool decode1_supported(int H, int I, int k);
+int launch_decode1(const BankView& bank, const float* logits, int k, const uint16_t* x, uint16_t* out,
+                   uint16_t* x_next, float* h, float* y, unsigned* bar, int32_t* ids, float* w, int num_sms,
+                   cudaStream_t s);
+
 // Prefill path: grouped NVFP4 GEMM on tcgen05 tensor cores, groups of up to kPrefillRows rows.
 constexpr int kPrefillRows = 256;
 bool prefill_supported(int H, int I);
-// xp [R, H] f16 = x[perm[r] / k] for every routed row r (expert order).
+// xp [R, H] bf16 = x[perm[r] / k] for every routed row r (expert order).
 int launch_gather(const uint16_t* x, const int32_t* perm, int k, int64_t R, int H, void* xp, cudaStream_t s);
-// h16 [R, I] f16 = silu(xp Wg^T gg) * (xp Wu^T gu).
-int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const RouteBufs& rb, void* h16,
+// hb [R, I] bf16 = silu(xp Wg^T gg) * (xp Wu^T gu).
+int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const RouteBufs& rb, void* hb,
                           int num_sms, cudaStream_t s);
-// y [R, H] f32 = h16 Wd^T gd.
-int launch_prefill_down(const BankView& bank, const void* h16, int64_t R, const RouteBufs& rb, float* y,
+// y [R, H] f32 = hb Wd^T gd.
+int launch_prefill_down(const BankView& bank, const void* hb, int64_t R, const RouteBufs& rb, float* y,
                         int num_sms, cudaStream_t s);
 
 }  // namespace moe

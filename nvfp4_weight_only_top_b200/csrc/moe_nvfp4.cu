@@ -82,7 +82,7 @@ int current_device(int* dev, DeviceInfo* info) {
 
 // Sizes of the workspace sub-buffers, each 256-byte aligned.
 struct WsLayout {
-  size_t ids, w, counts, offsets, perm, inv, groups, ngroups, singles, nsingles, chunk_counts, h, y, total;
+  size_t ids, w, counts, offsets, perm, inv, groups, ngroups, singles, nsingles, chunk_counts, bar, h, y, total;
 };
 
 size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -108,6 +108,7 @@ WsLayout ws_layout(int64_t T, int E, int k, int H, int I, int path) {
   L.singles = take((size_t)E * 16);
   L.nsingles = take(4);
   L.chunk_counts = take(T > moe::kRouteChunk ? (size_t)moe::route_chunks(T) * E * 4 : 0);
+  L.bar = take(8);
   L.h = take(R * (size_t)I * 4);
   L.y = take(R * (size_t)H * 4);
   L.total = o;
@@ -270,7 +271,7 @@ int resolve_path(int path, int64_t T, int k, int E, int H, int I) {
 }
 
 // Prefill path: route (groups of up to 256 rows) -> gather -> tcgen05 gate/up -> tcgen05 down
-// -> combine.  The f16 gathered rows live in the y region and the f16 intermediate in the h
+// -> combine.  The bf16 gathered rows live in the y region and the bf16 intermediate in the h
 // region, so the workspace is the decode path's.
 int prefill_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_bank* bank, int32_t k, void* out,
                  void* x_next, void* workspace, size_t workspace_bytes, void* stream, int dev,
@@ -294,7 +295,7 @@ int prefill_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
   rb.split_singles = 0;
   const moe::BankView bv = view_of(bank);
   const int64_t R = T * k;
-  void* h16 = w8 + L.h;
+  void* hb = w8 + L.h;
   void* xp = w8 + L.y;
   float* y = reinterpret_cast<float*>(w8 + L.y);
   int launches = 0;
@@ -305,11 +306,11 @@ int prefill_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
                          &launches)))
     return rc;
   prof_before(MOE_NVFP4_KERNEL_PREFILL_GATEUP, s);
-  if ((rc = after_launch(moe::launch_prefill_gateup(bv, xp, R, rb, h16, info.sms, s), s, "prefill gate/up",
+  if ((rc = after_launch(moe::launch_prefill_gateup(bv, xp, R, rb, hb, info.sms, s), s, "prefill gate/up",
                          &launches)))
     return rc;
   prof_before(MOE_NVFP4_KERNEL_PREFILL_DOWN, s);
-  if ((rc = after_launch(moe::launch_prefill_down(bv, h16, R, rb, y, info.sms, s), s, "prefill down", &launches)))
+  if ((rc = after_launch(moe::launch_prefill_down(bv, hb, R, rb, y, info.sms, s), s, "prefill down", &launches)))
     return rc;
   prof_before(MOE_NVFP4_KERNEL_COMBINE, s);
   if ((rc = after_launch(moe::launch_combine(y, rb.w, rb.inv, T, k, H, static_cast<const uint16_t*>(x),
@@ -362,16 +363,27 @@ int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
   }
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   moe::RouteBufs rb = route_bufs(w8, L);
+  const moe::BankView bv = view_of(bank);
+  int launches = 0;
+  if (T == 1 && moe::decode1_supported(H, I, k)) {
+    prof_before(MOE_NVFP4_KERNEL_DECODE_FUSED, s);
+    if ((rc = after_launch(moe::launch_decode1(bv, logits, k, static_cast<const uint16_t*>(x),
+                                               static_cast<uint16_t*>(out), static_cast<uint16_t*>(x_next),
+                                               reinterpret_cast<float*>(w8 + L.h), reinterpret_cast<float*>(w8 + L.y),
+                                               reinterpret_cast<unsigned*>(w8 + L.bar), rb.ids, rb.w, info.sms, s),
+                           s, "fused single-token decode", &launches)))
+      return rc;
+    t_last_launches = launches;
+    return MOE_NVFP4_OK;
+  }
   // One-row groups take the CUDA-core row kernels when both widths allow; groups of two or
   // more rows (none when T == 1) take the mma.sync kernels.
   const bool rows = moe::rows_supported(H, true) && moe::rows_supported(I, false);
   const bool multi = !rows || T > 1;
   rb.split_singles = rows ? 1 : 0;
-  const moe::BankView bv = view_of(bank);
   float* h = reinterpret_cast<float*>(w8 + L.h);
   float* y = reinterpret_cast<float*>(w8 + L.y);
   const uint16_t* xb = static_cast<const uint16_t*>(x);
-  int launches = 0;
   prof_before(MOE_NVFP4_KERNEL_ROUTE, s);
   if ((rc = after_launch(moe::launch_route(logits, T, E, k, rb, s), s, "route", &launches))) return rc;
   prof_before(MOE_NVFP4_KERNEL_DECODE_GATEUP, s);

@@ -10,14 +10,15 @@
 //       stage, E4M3 scales 128 rows x 16 B per M-tile every 4 stages -- straight out of the
 //       bank (dims: bytes of a row, rows, expert), so weight bytes cross the L1 once, in bulk;
 //   warps 0-3 (one thread per weight row of each M-tile): read their row's codes and scales
-//       from shared memory, convert E2M1 with cvt, multiply by the block scale in f16 (exact)
-//       and store the f16 row chunk into a 128-byte-swizzled K-major operand stage;
-//   warp 4 (one thread): 2-D TMA of the group's activation rows (f16, expert order) into
+//       from shared memory, convert E2M1 with cvt, multiply by the block scale (exact) and store
+//       the BF16 row chunk into a 128-byte-swizzled K-major operand stage;
+//   warp 4 (one thread): 2-D TMA of the group's BF16 activation rows (expert order) into
 //       swizzled stages;
-//   warp 5 (one thread): tcgen05.mma kind::f16 (M = 128, N = rows of the group rounded up to
-//       16, K = 16) into two f32 accumulators in tensor memory; tcgen05.commit frees a stage.
+//   warp 5 (one thread): tcgen05.mma kind::f16 with BF16 A and B (M = 128, N = rows of the
+//       group rounded up to 16, K = 16) into two f32 accumulators in tensor memory;
+//       tcgen05.commit frees a stage.
 // After a tile's last K stage warps 0-3 read the accumulators back with tcgen05.ld and apply
-// the global scale (and SwiGLU for gate/up).
+// the global scale (and SwiGLU for gate/up, whose result h is stored as BF16).
 //
 // Weight layout: page "Beam 1.0 501B-A23B, streaming pack, NVFP4 experts / MLX 8-bit
 // residents", section "What this pack holds"; SwiGLU in FP32: page "Beam-1.0-501B-A23B VQ
@@ -25,7 +26,6 @@
 // GEMM" on sm_120) dequantize each weight tile once for all of a group's tokens; so does this
 // one, on sm_100a tensor cores.
 #include <cuda.h>
-#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -35,8 +35,8 @@ namespace moe {
 namespace {
 
 constexpr int kBM = 128;                       // rows per MMA M-tile
-constexpr int kKC = 64;                        // K per stage: one 128-byte swizzle row of f16
-constexpr int kStages = 3;                     // operand stages (A f16 + B f16)
+constexpr int kKC = 64;                        // K per stage: one 128-byte swizzle row of bf16
+constexpr int kStages = 3;                     // operand stages (A and B, bf16)
 constexpr int kWStages = 3;                    // raw code stages
 constexpr int kSStages = 2;                    // raw scale stages (4 operand stages each)
 constexpr int kMaxN = 256;
@@ -64,12 +64,12 @@ struct PrefillParams {
   int gateup;              // 1: M-tile 0 = gate rows, M-tile 1 = same up rows; 0: 256 consecutive rows
   const int4* groups;      // (expert, first permuted row, rows <= 256, 0)
   const int32_t* ngroups;
-  void* out;               // gate/up: h f16 [R, out_stride]; down: y f32 [R, out_stride]
+  void* out;               // gate/up: h bf16 [R, out_stride]; down: y f32 [R, out_stride]
   int out_stride;
 };
 
 struct Maps {
-  CUtensorMap x;           // activations [R, K] f16
+  CUtensorMap x;           // activations [R, K] bf16
   CUtensorMap codes[2];    // codes of the M-tile 0 / 1 matrix: [E][rows][K/2] bytes
   CUtensorMap scales[2];   // scales: [E][rows][K/16] bytes
 };
@@ -111,8 +111,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ Maps maps, const PrefillParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint8_t* sA = smem;                                   // [stage][m-tile] 16 KB, 128B-swizzled
-  uint8_t* sB = smem + kOffB;                           // [stage] 32 KB, 128B-swizzled
+  uint8_t* sA = smem;                                   // [stage][m-tile] 16 KB bf16, 128B-swizzled
+  uint8_t* sB = smem + kOffB;                           // [stage] 32 KB bf16, 128B-swizzled
   uint8_t* sW = smem + kOffW;                           // [stage][m-tile] 128 rows x 32 B
   uint8_t* sS = smem + kOffS;                           // [stage][m-tile] 128 rows x 16 B
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -135,21 +135,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const TileCursor cur{p.tiles_per_group};
 
   if (threadIdx.x == 0) {
+    // Producer-side barriers count one arrival per producer warp (lane 0 after __syncwarp):
+    // 128 arrivals on one word would serialise in the shared-memory pipe.
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&a_full[s], 4 * 32);
+      mbar_init(&a_full[s], 4);
       mbar_init(&b_full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int s = 0; s < kWStages; ++s) {
       mbar_init(&w_full[s], 1);
-      mbar_init(&w_empty[s], 4 * 32);
+      mbar_init(&w_empty[s], 4);
     }
     for (int s = 0; s < kSStages; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 4 * 32);
+      mbar_init(&s_empty[s], 4);
     }
     mbar_init(d_full, 1);
-    mbar_init(d_empty, 4 * 32);
+    mbar_init(d_empty, 4);
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -192,10 +194,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {                  // word j = K 8j .. 8j+7 = 16-byte chunk j
           uint32_t e[4];
-          e2m1x8_to_f16x8(w[j], e);
-          const uint32_t s2 = sc[j >> 1];
-          st_shared_v4(base + ((j ^ (t & 7)) << 4), hmul2(e[0], s2), hmul2(e[1], s2), hmul2(e[2], s2),
-                       hmul2(e[3], s2));
+          e2m1x8_scaled_to_bf16x8(w[j], sc[j >> 1], e);
+          st_shared_v4(base + ((j ^ (t & 7)) << 4), e[0], e[1], e[2], e[3]);
         }
       }
     };
@@ -216,12 +216,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         const int nn = min(32, grp.z - n0);
         if (p.gateup) {
-          __half* o = static_cast<__half*>(p.out) + (size_t)(grp.y + n0) * p.out_stride + m * kBM + t;
+          uint16_t* o = static_cast<uint16_t*>(p.out) + (size_t)(grp.y + n0) * p.out_stride + m * kBM + t;
 #pragma unroll
           for (int j = 0; j < 32; ++j)
             if (j < nn)
-              o[(size_t)j * p.out_stride] =
-                  __float2half_rn(silu_mul_fast(__uint_as_float(d0[j]) * gm0, __uint_as_float(d1[j]) * gm1));
+              o[(size_t)j * p.out_stride] = (uint16_t)f32_to_bf16_bits(
+                  silu_mul_fast(__uint_as_float(d0[j]) * gm0, __uint_as_float(d1[j]) * gm1));
         } else {
           float* o = static_cast<float*>(p.out) + (size_t)(grp.y + n0) * p.out_stride + m * 2 * kBM + t;
 #pragma unroll
@@ -234,7 +234,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(d_empty);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(d_empty);
     };
 
     bool ok = true;
@@ -242,26 +243,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int q = 0; q < nq && ok; ++q) {
       const int c = q % nst;
       const int ws = q % kWStages, ss = (q >> 2) % kSStages;
-      if (!mbar_wait(&w_full[ws], (q / kWStages) & 1) ||
-          ((c & 3) == 0 && !mbar_wait(&s_full[ss], ((q >> 2) / kSStages) & 1))) {
+      const bool got = mbar_wait(&w_full[ws], (q / kWStages) & 1) &&
+                       ((c & 3) != 0 || mbar_wait(&s_full[ss], ((q >> 2) / kSStages) & 1));
+      if (!__all_sync(0xffffffffu, got)) {     // warp-uniform: the warp arrives as one below
         ok = false;
         break;
       }
       StageFrag f;
       fetch(q, f);
       const int s = q % kStages;
-      if (!mbar_wait(&empty[s], ((q / kStages) & 1) ^ 1)) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ((q / kStages) & 1) ^ 1))) {
         ok = false;
         break;
       }
       store(s, f);
       fence_proxy_async_smem();
-      mbar_arrive(&a_full[s]);
-      // The raw slots go back to the TMA only after the proxy fence above: a TMA write (async
-      // proxy) into a slot that this thread read with generic loads must be ordered after
-      // those reads, or it can overtake them.
-      mbar_arrive(&w_empty[ws]);
-      if ((c & 3) == 3) mbar_arrive(&s_empty[ss]);
+      __syncwarp();
+      // The raw slots go back to the TMA only after every lane's proxy fence above: a TMA
+      // write (async proxy) into a slot that was read with generic loads must be ordered
+      // after those reads, or it can overtake them.
+      if (lane == 0) {
+        mbar_arrive(&a_full[s]);
+        mbar_arrive(&w_empty[ws]);
+        if ((c & 3) == 3) mbar_arrive(&s_empty[ss]);
+      }
       const int i = q / nst;
       if (i > 0 && c == first - 1) epilogue(i - 1);
     }
@@ -336,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tt = blockIdx.x; tt < ntiles && ok; tt += gridDim.x, ++i) {
         const int4 grp = __ldg(&p.groups[tt / p.tiles_per_group]);
         const int N = (grp.z + 15) & ~15;
-        const uint32_t idesc = idesc_f16(kBM, N);
+        const uint32_t idesc = idesc_bf16(kBM, N);
         if (i > 0 && !mbar_wait(d_empty, (i - 1) & 1)) break;
         tc_fence_after();
         for (int c = 0; c < nst; ++c, ++q) {
@@ -372,22 +377,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Gathers the routed rows of x (bf16 [T, H]) in expert order into f16 [R, H].
+// Gathers the routed rows of x (bf16 [T, H]) in expert order into xp (bf16 [R, H]).
 __global__ void gather_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int k, int64_t R,
-                              int H, __half* __restrict__ xp) {
+                              int H, uint16_t* __restrict__ xp) {
   const int per = H / 8;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= R * per) return;
   const int64_t r = i / per;
   const int c = (int)(i - r * per) * 8;
   const int t = perm[r] / k;
-  const uint4 b = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + c));
-  uint4 o;
-  o.x = pack_f16x2(bf16_bits_to_f32(b.x & 0xFFFF), bf16_bits_to_f32(b.x >> 16));
-  o.y = pack_f16x2(bf16_bits_to_f32(b.y & 0xFFFF), bf16_bits_to_f32(b.y >> 16));
-  o.z = pack_f16x2(bf16_bits_to_f32(b.z & 0xFFFF), bf16_bits_to_f32(b.z >> 16));
-  o.w = pack_f16x2(bf16_bits_to_f32(b.w & 0xFFFF), bf16_bits_to_f32(b.w >> 16));
-  *reinterpret_cast<uint4*>(xp + r * H + c) = o;
+  *reinterpret_cast<uint4*>(xp + r * H + c) = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + c));
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -406,7 +405,7 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Tensor map over a row-major f16 matrix [rows, cols]: boxes of 64 columns x 64 rows, 128B swizzle.
+// Tensor map over a row-major bf16 matrix [rows, cols]: boxes of 64 columns x 64 rows, 128B swizzle.
 int make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int cols) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return -(int)cudaErrorNotSupported;
@@ -414,7 +413,7 @@ int make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int cols) {
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
   const cuuint32_t box[2] = {kKC, kBoxRows};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? 0 : -(int)cudaErrorInvalidValue;
@@ -461,12 +460,12 @@ bool prefill_supported(int H, int I) { return H % 256 == 0 && I % 256 == 0; }
 
 int launch_gather(const uint16_t* x, const int32_t* perm, int k, int64_t R, int H, void* xp, cudaStream_t s) {
   const int64_t n = R * (H / 8);
-  gather_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(x, perm, k, R, H, static_cast<__half*>(xp));
+  gather_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(x, perm, k, R, H, static_cast<uint16_t*>(xp));
   const cudaError_t err = cudaGetLastError();
   return err == cudaSuccess ? 1 : -(int)err;
 }
 
-int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const RouteBufs& rb, void* h16,
+int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const RouteBufs& rb, void* hb,
                           int num_sms, cudaStream_t s) {
   Maps maps;
   int rc = make_rows_map(&maps.x, xp, R, bank.H);
@@ -483,15 +482,15 @@ int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const
   p.gateup = 1;
   p.groups = rb.groups;
   p.ngroups = rb.ngroups;
-  p.out = h16;
+  p.out = hb;
   p.out_stride = bank.I;
   return launch_prefill(p, maps, num_sms, s);
 }
 
-int launch_prefill_down(const BankView& bank, const void* h16, int64_t R, const RouteBufs& rb, float* y,
+int launch_prefill_down(const BankView& bank, const void* hb, int64_t R, const RouteBufs& rb, float* y,
                         int num_sms, cudaStream_t s) {
   Maps maps;
-  int rc = make_rows_map(&maps.x, h16, R, bank.I);
+  int rc = make_rows_map(&maps.x, hb, R, bank.I);
   if (!rc) rc = make_weight_maps(&maps, bank, 2, 2, bank.H, bank.I);
   if (rc) return rc;
   PrefillParams p{};

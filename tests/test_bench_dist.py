@@ -1,0 +1,72 @@
+"""bench.py's multi-process plumbing on the CPU (gloo, world size 2): the max-over-ranks timing,
+the barrier, the whole-job token count, and the reference arm's rank-0-only rule.  The layer is
+data parallel with no collective on its data path ("replicas"); only this plumbing is shared."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, ws, port, q):
+    os.environ.update({"WORLD_SIZE": str(ws), "RANK": str(rank), "LOCAL_RANK": str(rank),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    sys.path.insert(0, ROOT)
+    import bench
+    import torch.distributed as dist
+    w, r, _ = bench.dist_init(backend="gloo")
+    bench.barrier(w)
+    ms = bench.max_over_ranks(w, 10.0 + 5.0 * r)         # each rank's own device time
+    tokens = 3 * 7 * w                                     # T x steps x ranks: the whole job
+    q.put((r, w, ms, tokens / (ms / 1000.0)))
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_whole_job_value_gloo():
+    ws, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main, args=(r, ws, port, q)) for r in range(ws)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=120) for _ in range(ws)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r, w, ms, value in got:
+        assert w == 2 and ms == 15.0                       # the slowest rank sets the time
+        assert value == pytest.approx(42 / 0.015)          # all ranks' tokens over that time
+
+
+def _bench(args, env_extra):
+    env = dict(os.environ, **env_extra)
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], capture_output=True,
+                          text=True, env=env, timeout=300, cwd=ROOT)
+
+
+def test_reference_arm_rank0_prints_one_line_other_ranks_nothing():
+    r0 = _bench(["--impl", "reference", "--config", "decode_t1", "--steps", "1", "--warmup", "0",
+                 "--ref-budget", "0.1"], {"WORLD_SIZE": "2", "RANK": "0"})
+    assert r0.returncode == 0, r0.stderr
+    lines = [l for l in r0.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in d
+    assert d["impl"] == "reference" and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    r1 = _bench(["--impl", "reference", "--config", "decode_t1", "--steps", "1", "--warmup", "0",
+                 "--ref-budget", "0.1"], {"WORLD_SIZE": "2", "RANK": "1"})
+    assert r1.returncode == 0 and r1.stdout.strip() == ""

@@ -212,3 +212,20 @@ def test_prefill_bitwise_repeatable():
         torch.cuda.synchronize()
         assert torch.equal(first, again)
     assert moe.moe_nvfp4_device_status() == 0
+
+
+@pytest.mark.parametrize("E,k,H,I,mode", [(32, 8, 1024, 512, 0), (64, 4, 2048, 1024, 1), (16, 1, 4096, 1536, 0),
+                                          (256, 8, 5120, 2560, 1), (8, 8, 1024, 512, 0)])
+def test_single_token_fused_kernel(E, k, H, I, mode):
+    """T = 1 runs route, gate/up, down and combine in one persistent kernel (one launch); its
+    output matches the oracle and its residual is bit-exact."""
+    import nvfp4_weight_only_top_b200 as moe
+    cfg = moe_inputs.LayerConfig("single", E, k, H, I, 1, 1, "normal", seed=E + k + H)
+    buf, bank = device_bank(cfg, global_mode=mode)
+    xb, lg = moe_inputs.make_x(cfg), moe_inputs.make_logits(cfg)
+    for path in ("auto", "decode"):
+        out, xn = _run(cfg, bank, xb, lg, path, x_next=True)
+        assert moe.moe_nvfp4_last_launch_count() == 1
+        ref = _oracle(cfg, xb, lg, global_mode=mode)
+        assert_layer_close(oracle.bf16_bits_to_f64(out), ref["out"], f"T=1 {E},{k},{H},{I}/{path}")
+        assert np.array_equal(xn, oracle.residual_add(xb, out))
