@@ -1,5 +1,5 @@
 // Decode of a single token (T = 1) as ONE persistent kernel: route -> gate/up + SwiGLU ->
-// down -> combine, with two grid-wide barriers and no other launch.
+// down -> combine, with no grid-wide barrier and no other launch.
 //
 // With one token every routed row is its own expert, the work is 2 FLOP per weight byte, and
 // the layer is a pure stream of k expert records (177 MB at E=256, k=8, H=5120, I=2560) from
@@ -8,13 +8,16 @@
 //     no router kernel, no hand-off;
 //   * one producer warp per CTA streams the CTA's weight rows with large 1-D bulk copies
 //     (TMA) into a 4-stage shared-memory ring -- first its share of the gate/up rows, then,
-//     without waiting for anything, its share of the down rows, so HBM stays busy across the
-//     grid barrier that makes h visible;
+//     without waiting for anything, its share of the down rows;
+//   * the work is cut into contiguous shares so that a CTA's down rows belong to the same one
+//     or two slots (experts) as its gate/up rows: before its down rows a CTA waits only until
+//     the h of those slots is complete (a per-slot counter), not for the whole grid;
 //   * eight consumer warps dot the rows against the activations held in registers (f16, the
 //     lane's own K positions) with packed f16 FMAs per 16-input block, fold each block into
 //     f32 with its E4M3 scale, and reduce across the warp;
-//   * after the last barrier each CTA combines a slice of the output (f32 in slot order, one
-//     BF16 rounding, optional residual), exactly as the combine kernel does.
+//   * the combine of a block of 32 output rows is done by the warp that writes the block's
+//     last y values (a per-block counter), in slot order with f32 accumulation and one BF16
+//     rounding (and the optional residual), exactly as the combine kernel does.
 //
 // Weight layout: page "Beam 1.0 501B-A23B, streaming pack, NVFP4 experts / MLX 8-bit
 // residents", section "What this pack holds"; router logits and SwiGLU in FP32: page
@@ -33,6 +36,8 @@ constexpr int kNW = 8;                       // consumer warps
 constexpr int kThreads1 = 32 * (kNW + 1);    // + one producer warp
 constexpr int kRing = 4;                     // stages in the ring
 constexpr int kMaxK = 32;
+constexpr int kMaxBlocks = 256;              // H / 32 row blocks of the combine
+constexpr int kMaxLast = 64;                 // down stages of one CTA (bound checked on the host)
 
 struct D1Params {
   const uint8_t* bank;
@@ -46,7 +51,7 @@ struct D1Params {
   uint16_t* x_next;      // [H] bf16 or null
   float* h;              // [k, I] f32 scratch
   float* y;              // [k, H] f32 scratch
-  unsigned* bar;         // [2] grid-barrier counters, zero on entry
+  unsigned* bar;         // [kMaxK + H/32] completion counters, zero on entry
   int32_t* ids;          // [k] routing result (for inspection)
   float* w;              // [k]
 };
@@ -104,11 +109,10 @@ __device__ __forceinline__ float unit_dot(const uint4 c, uint32_t sc2, const uin
   return fmaf(sf.x, a.x + a.y, sf.y * (b.x + b.y));
 }
 
-// Grid-wide barrier of the persistent grid (all CTAs resident: cooperative launch).  One
-// thread per CTA; bounded: gives up after kWaitCycles, records a timeout and returns false.
-__device__ bool grid_arrive_wait(unsigned* counter, unsigned target) {
-  __threadfence();
-  atomicAdd(counter, 1u);
+// Waits until *counter reaches target (other CTAs of the persistent grid add to it; all are
+// resident: cooperative launch).  Bounded: gives up after kWaitCycles, records a timeout and
+// returns false.
+__device__ bool wait_count(const unsigned* counter, unsigned target) {
   const long long t0 = clock64();
   while (ld_acquire(counter) < target) {
     if (clock64() - t0 > kWaitCycles) {
@@ -133,18 +137,22 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
   constexpr int H = UG * 1024, I = UD * 512;
   constexpr int kCodes1 = kNW * H / 2, kScales1 = kNW * H / 16;       // per matrix, 8 rows
   constexpr int kStage1 = 2 * (kCodes1 + kScales1);
-  constexpr int kRows2 = 2 * kNW;                                     // down rows per stage
+  constexpr int kRows2 = 4 * kNW;                                     // down rows per stage
   constexpr int kCodes2 = kRows2 * I / 2, kScales2 = kRows2 * I / 16;
   constexpr int kStage2 = kCodes2 + kScales2;
   constexpr int kStage = kStage1 > kStage2 ? kStage1 : kStage2;
   constexpr int kUnits2 = I / 32;                                     // units per down row
 
   extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRing * kStage);
+  // ring | x (bf16 [H]) | h of up to two slots (f32 [2][I]) | barriers, routing
+  uint16_t* sx = reinterpret_cast<uint16_t*>(smem + kRing * kStage);
+  float* sh = reinterpret_cast<float*>(sx + H);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sh + 2 * I);
   uint64_t* empty = full + kRing;
-  int* s_ids = reinterpret_cast<int*>(empty + kRing);
+  uint64_t* gm_full = empty + kRing;                        // the global multipliers are in s_gm
+  int* s_ids = reinterpret_cast<int*>(gm_full + 1);
   float* s_w = reinterpret_cast<float*>(s_ids + kMaxK);
-  float* s_gm = s_w + kMaxK;                                // [3][kMaxK] global multipliers
+  float* s_gm = s_w + kMaxK;                                // [3][kMaxK]
   int* s_ok = reinterpret_cast<int*>(s_gm + 3 * kMaxK);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -154,14 +162,25 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
   share(n1, blockIdx.x, gridDim.x, lo1, hi1);
   share(n2, blockIdx.x, gridDim.x, lo2, hi2);
   const int cnt1 = hi1 - lo1, cnt = cnt1 + (hi2 - lo2);     // this CTA's stages, both phases
+  unsigned* slot_done = p.bar;                              // [k]: gate/up stages completed
+  unsigned* block_done = p.bar + kMaxK;                     // [H/32]: down stages written
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRing; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kNW);
     }
+    mbar_init(gm_full, 1);
     *s_ok = 1;
     fence_barrier_init();
+  }
+  if (warp != 0) {                                          // x into shared memory, once
+    // 16-byte chunk c of 32-input unit u is stored at chunk c ^ ((u >> 1) & 3) of the unit, so
+    // that the lanes of a warp, which read consecutive units, hit different banks.
+    for (int i = (int)threadIdx.x - 32; i < H / 8; i += (int)blockDim.x - 32) {
+      const int u = i >> 2, c = i & 3;
+      reinterpret_cast<uint4*>(sx)[4 * u + (c ^ ((u >> 1) & 3))] = __ldg(reinterpret_cast<const uint4*>(p.x) + i);
+    }
   }
   if (warp == 0) {                                          // every CTA routes the token
     int id;
@@ -170,11 +189,6 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
     if (lane < k) {
       s_ids[lane] = id;
       s_w[lane] = wt;
-      const uint8_t* rec = p.bank + (uint64_t)id * p.stride;
-#pragma unroll
-      for (int m = 0; m < 3; ++m)
-        s_gm[m * kMaxK + lane] =
-            global_mult(__ldg(reinterpret_cast<const float*>(rec + p.global_off[m])), p.global_mode);
       if (blockIdx.x == 0) {
         p.ids[lane] = id;
         p.w[lane] = wt;
@@ -185,29 +199,46 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
 
   if (warp == kNW) {
     // ---------------------------------------------------------------- producer
+    const uint64_t pol = policy_evict_first();
+    auto issue = [&](int q) {                               // stage q into its ring slot
+      const int s = q % kRing;
+      uint8_t* dst = smem + s * kStage;
+      if (q < cnt1) {
+        const int u = lo1 + q, j = u / (I / kNW), r0 = (u - j * (I / kNW)) * kNW;
+        const uint8_t* rec = p.bank + (uint64_t)s_ids[j] * p.stride;
+        mbar_arrive_expect_tx(&full[s], kStage1);
+        bulk_g2s(dst, rec + p.codes_off[0] + (uint64_t)r0 * (H / 2), kCodes1, &full[s], pol);
+        bulk_g2s(dst + kCodes1, rec + p.codes_off[1] + (uint64_t)r0 * (H / 2), kCodes1, &full[s], pol);
+        bulk_g2s(dst + 2 * kCodes1, rec + p.scales_off[0] + (uint64_t)r0 * (H / 16), kScales1, &full[s], pol);
+        bulk_g2s(dst + 2 * kCodes1 + kScales1, rec + p.scales_off[1] + (uint64_t)r0 * (H / 16), kScales1,
+                 &full[s], pol);
+      } else {
+        const int u = lo2 + (q - cnt1), j = u / (H / kRows2), r0 = (u - j * (H / kRows2)) * kRows2;
+        const uint8_t* rec = p.bank + (uint64_t)s_ids[j] * p.stride;
+        mbar_arrive_expect_tx(&full[s], kStage2);
+        bulk_g2s(dst, rec + p.codes_off[2] + (uint64_t)r0 * (I / 2), kCodes2, &full[s], pol);
+        bulk_g2s(dst + kCodes2, rec + p.scales_off[2] + (uint64_t)r0 * (I / 16), kScales2, &full[s], pol);
+      }
+    };
+    const int first = cnt < kRing ? cnt : kRing;            // the ring starts empty
+    if (lane == 0)
+      for (int q = 0; q < first; ++q) issue(q);
+    // With those in flight, the global multipliers of the k slots (one lane per slot).
+    if (lane < k) {
+      const uint8_t* rec = p.bank + (uint64_t)s_ids[lane] * p.stride;
+      float g[3];
+#pragma unroll
+      for (int m = 0; m < 3; ++m) g[m] = __ldg(reinterpret_cast<const float*>(rec + p.global_off[m]));
+#pragma unroll
+      for (int m = 0; m < 3; ++m) s_gm[m * kMaxK + lane] = global_mult(g[m], p.global_mode);
+    }
+    __syncwarp();
     if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      int q = 0;
+      mbar_arrive(gm_full);
+      int q = first;
       for (; q < cnt; ++q) {
-        const int s = q % kRing;
-        if (!mbar_wait(&empty[s], ((q / kRing) & 1) ^ 1)) break;
-        uint8_t* dst = smem + s * kStage;
-        if (q < cnt1) {
-          const int u = lo1 + q, j = u / (I / kNW), r0 = (u - j * (I / kNW)) * kNW;
-          const uint8_t* rec = p.bank + (uint64_t)s_ids[j] * p.stride;
-          mbar_arrive_expect_tx(&full[s], kStage1);
-          bulk_g2s(dst, rec + p.codes_off[0] + (uint64_t)r0 * (H / 2), kCodes1, &full[s], pol);
-          bulk_g2s(dst + kCodes1, rec + p.codes_off[1] + (uint64_t)r0 * (H / 2), kCodes1, &full[s], pol);
-          bulk_g2s(dst + 2 * kCodes1, rec + p.scales_off[0] + (uint64_t)r0 * (H / 16), kScales1, &full[s], pol);
-          bulk_g2s(dst + 2 * kCodes1 + kScales1, rec + p.scales_off[1] + (uint64_t)r0 * (H / 16), kScales1,
-                   &full[s], pol);
-        } else {
-          const int u = lo2 + (q - cnt1), j = u / (H / kRows2), r0 = (u - j * (H / kRows2)) * kRows2;
-          const uint8_t* rec = p.bank + (uint64_t)s_ids[j] * p.stride;
-          mbar_arrive_expect_tx(&full[s], kStage2);
-          bulk_g2s(dst, rec + p.codes_off[2] + (uint64_t)r0 * (I / 2), kCodes2, &full[s], pol);
-          bulk_g2s(dst + kCodes2, rec + p.scales_off[2] + (uint64_t)r0 * (I / 16), kScales2, &full[s], pol);
-        }
+        if (!mbar_wait(&empty[q % kRing], ((q / kRing) & 1) ^ 1)) break;
+        issue(q);
       }
       // Leave no copy in flight (only an error path gets here with copies outstanding).
       for (int i = q - kRing > 0 ? q - kRing : 0; i < q; ++i) mbar_wait(&full[i % kRing], (i / kRing) & 1);
@@ -222,10 +253,11 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
     uint32_t xr[UG][16];
 #pragma unroll
     for (int u = 0; u < UG; ++u) {
-      const uint16_t* xp = p.x + 32 * (lane + 32 * u);
+      const int un = lane + 32 * u;
+      const uint4* xp = reinterpret_cast<const uint4*>(sx) + 4 * un;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const uint4 b = __ldg(reinterpret_cast<const uint4*>(xp + 8 * q));
+        const uint4 b = xp[q ^ ((un >> 1) & 3)];
         xr[u][4 * q + 0] = pack_f16x2(bf16_bits_to_f32(b.x & 0xFFFF), bf16_bits_to_f32(b.x >> 16));
         xr[u][4 * q + 1] = pack_f16x2(bf16_bits_to_f32(b.y & 0xFFFF), bf16_bits_to_f32(b.y >> 16));
         xr[u][4 * q + 2] = pack_f16x2(bf16_bits_to_f32(b.z & 0xFFFF), bf16_bits_to_f32(b.z >> 16));
@@ -233,13 +265,14 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
       }
     }
     int q = 0;
+    bool have_gm = false;
     for (; q < cnt1 && ok; ++q) {
       const int s = q % kRing;
+      const int u0 = lo1 + q, j = u0 / (I / kNW), r = (u0 - j * (I / kNW)) * kNW + warp;
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (q / kRing) & 1))) {
         ok = false;
         break;
       }
-      const int u0 = lo1 + q, j = u0 / (I / kNW), r = (u0 - j * (I / kNW)) * kNW + warp;
       const uint32_t st = sbase + s * kStage;
       const uint32_t cg = st + warp * (H / 2), cu = st + kCodes1 + warp * (H / 2);
       const uint32_t sg = st + 2 * kCodes1 + warp * (H / 16), su = sg + kScales1;
@@ -262,32 +295,86 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
         accG += __shfl_xor_sync(0xFFFFFFFFu, accG, off);
         accU += __shfl_xor_sync(0xFFFFFFFFu, accU, off);
       }
+      if (!have_gm) {
+        have_gm = true;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(gm_full, 0))) {
+          ok = false;
+          break;
+        }
+      }
       if (lane == 0) p.h[(size_t)j * I + r] = silu_mul(accG * s_gm[j], accU * s_gm[kMaxK + j]);
     }
-    // Grid barrier 1: every h row written.
+    // Publish this CTA's gate/up stages per slot, then wait for the slots of its down rows.
     named_bar_sync(1, 32 * kNW);
-    if (threadIdx.x == 0) *s_ok = (ok && grid_arrive_wait(&p.bar[0], gridDim.x)) ? 1 : 0;
+    if (threadIdx.x == 0) {
+      __threadfence();
+      for (int u = lo1; u < hi1;) {
+        const int j = u / (I / kNW), uend = min(hi1, (j + 1) * (I / kNW));
+        atomicAdd(&slot_done[j], (unsigned)(uend - u));
+        u = uend;
+      }
+      bool good = ok;
+      if (hi2 > lo2)
+        for (int j = lo2 / (H / kRows2); good && j <= (hi2 - 1) / (H / kRows2); ++j)
+          good = wait_count(&slot_done[j], I / kNW);
+      *s_ok = good ? 1 : 0;
+    }
     named_bar_sync(1, 32 * kNW);
     ok = ok && *s_ok;
+    // h of the (at most two) slots of this CTA's down rows into shared memory, once per CTA
+    // rather than once per warp: every CTA reads the same few KB, so per-warp loads would
+    // pile onto the same L2 lines.
+    const int jlo = lo2 / (H / kRows2);
+    if (ok && hi2 > lo2) {
+      // All of a thread's loads are issued before any store, so their latencies overlap.
+      constexpr int kPer = (2 * I / 4 + 32 * kNW - 1) / (32 * kNW);
+      const int n4 = ((hi2 - 1) / (H / kRows2) - jlo + 1) * I / 4;
+      const float4* src = reinterpret_cast<const float4*>(p.h + (size_t)jlo * I);
+      float4 v[kPer];
+#pragma unroll
+      for (int t = 0; t < kPer; ++t) {
+        const int i = (int)threadIdx.x + t * 32 * kNW;
+        if (i < n4) v[t] = __ldcg(src + i);
+      }
+      // Chunk c of unit u (32 floats) of a slot is stored at chunk c ^ (u & 7) of the unit
+      // (bank spread for the per-lane reads below).
+#pragma unroll
+      for (int t = 0; t < kPer; ++t) {
+        const int i = (int)threadIdx.x + t * 32 * kNW;
+        if (i < n4) {
+          const int sl = i / (I / 4), w = i - sl * (I / 4), u = w >> 3, c = w & 7;
+          reinterpret_cast<float4*>(sh)[sl * (I / 4) + 8 * u + (c ^ (u & 7))] = v[t];
+        }
+      }
+    }
+    named_bar_sync(1, 32 * kNW);
 
-    // Phase 2: down.  Warp w takes rows r0 + 2w, r0 + 2w + 1 of the stage; lane l its units
-    // cu = l + 32 u (u < UD) of the two rows laid end to end: row cu / kUnits2, K unit
-    // cu % kUnits2, with h at those K positions in registers (reloaded when the slot changes).
+    // Phase 2: down.  Warp w takes rows 4w .. 4w+3 of the stage as two pairs; in a pair, lane l
+    // takes units cu = l + 32 u (u < UD) of the two rows laid end to end: row cu / kUnits2, K
+    // unit cu % kUnits2, with h at those K positions in registers (reloaded when the slot
+    // changes).
     uint32_t hr[UD][16];
     int hj = -1;
     for (; q < cnt && ok; ++q) {
       const int s = q % kRing;
-      const int u0 = lo2 + (q - cnt1), j = u0 / (H / kRows2), r0 = (u0 - j * (H / kRows2)) * kRows2 + 2 * warp;
+      const int u0 = lo2 + (q - cnt1), j = u0 / (H / kRows2), r0 = (u0 - j * (H / kRows2)) * kRows2 + 4 * warp;
+      if (!have_gm) {
+        have_gm = true;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(gm_full, 0))) {
+          ok = false;
+          break;
+        }
+      }
       if (j != hj) {
         hj = j;
-        const float* hp = p.h + (size_t)j * I;
+        const float* hp = sh + (size_t)(j - jlo) * I;
 #pragma unroll
         for (int u = 0; u < UD; ++u) {
           const int ku = (lane + 32 * u) % kUnits2;
           const float4* src = reinterpret_cast<const float4*>(hp + 32 * ku);
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
-            const float4 a = __ldcg(src + q4);
+            const float4 a = src[q4 ^ (ku & 7)];
             hr[u][2 * q4] = pack_f16x2(a.x, a.y);
             hr[u][2 * q4 + 1] = pack_f16x2(a.z, a.w);
           }
@@ -298,67 +385,57 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
         break;
       }
       const uint32_t st = sbase + s * kStage;
-      const uint32_t cd = st + 2 * warp * (I / 2), sd = st + kCodes2 + 2 * warp * (I / 16);
-      float acc0 = 0.0f, acc1 = 0.0f;
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-      for (int u = 0; u < UD; ++u) {
-        const int cu = lane + 32 * u;                       // unit within the pair of rows
-        const float part = unit_dot(lds128(cd + cu * 16), lds16(sd + cu * 2), hr[u]);
-        if (cu < kUnits2)
-          acc0 += part;
-        else
-          acc1 += part;
+      for (int pr = 0; pr < 2; ++pr) {
+        const uint32_t cd = st + (4 * warp + 2 * pr) * (I / 2), sd = st + kCodes2 + (4 * warp + 2 * pr) * (I / 16);
+#pragma unroll
+        for (int u = 0; u < UD; ++u) {
+          const int cu = lane + 32 * u;                     // unit within the pair of rows
+          const float part = unit_dot(lds128(cd + cu * 16), lds16(sd + cu * 2), hr[u]);
+          if (cu < kUnits2)
+            acc[2 * pr] += part;
+          else
+            acc[2 * pr + 1] += part;
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        acc0 += __shfl_xor_sync(0xFFFFFFFFu, acc0, off);
-        acc1 += __shfl_xor_sync(0xFFFFFFFFu, acc1, off);
+      for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] += __shfl_xor_sync(0xFFFFFFFFu, acc[i], off);
+      if (lane < 4) {
+        const float v = lane == 0 ? acc[0] : lane == 1 ? acc[1] : lane == 2 ? acc[2] : acc[3];
+        p.y[(size_t)j * H + r0 + lane] = v * s_gm[2 * kMaxK + j];
       }
-      if (lane < 2) p.y[(size_t)j * H + r0 + lane] = (lane == 0 ? acc0 : acc1) * s_gm[2 * kMaxK + j];
     }
-    // Grid barrier 2: every y row written.
+    // Combine.  Block b = rows 32b .. 32b+31: one down stage per slot, so k contributions.
+    // Each CTA publishes its stages (one fence, one atomic per stage) and combines the blocks
+    // for which it added the last contribution.
     named_bar_sync(1, 32 * kNW);
-    if (threadIdx.x == 0) *s_ok = (ok && grid_arrive_wait(&p.bar[1], gridDim.x)) ? 1 : 0;
-    named_bar_sync(1, 32 * kNW);
-    if (*s_ok) {
-      // Combine: out[c] = bf16(sum_j w_j y[j][c]) in slot order; x_next = bf16(x + out).
-      int c0, c1;
-      share(H / 8, blockIdx.x, gridDim.x, c0, c1);
-      for (int cc = c0 + (int)threadIdx.x; cc < c1; cc += 32 * kNW) {
-        const int c = 8 * cc;
-        float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        for (int j = 0; j < k; ++j) {
-          const float wj = s_w[j];
-          const float4* src = reinterpret_cast<const float4*>(p.y + (size_t)j * H + c);
-          const float4 a = __ldcg(src), b = __ldcg(src + 1);
-          acc[0] = fmaf(wj, a.x, acc[0]);
-          acc[1] = fmaf(wj, a.y, acc[1]);
-          acc[2] = fmaf(wj, a.z, acc[2]);
-          acc[3] = fmaf(wj, a.w, acc[3]);
-          acc[4] = fmaf(wj, b.x, acc[4]);
-          acc[5] = fmaf(wj, b.y, acc[5]);
-          acc[6] = fmaf(wj, b.z, acc[6]);
-          acc[7] = fmaf(wj, b.w, acc[7]);
+    int* s_last = s_ok + 1;                                 // blocks this CTA combines
+    if (threadIdx.x == 0) {
+      int n = 0;
+      if (ok) {
+        __threadfence();
+        for (int u = lo2; u < hi2; ++u) {
+          const int b = u % (H / kRows2);
+          if (atomicAdd(&block_done[b], 1u) == (unsigned)k - 1u) s_last[n++] = b;
         }
-        uint32_t o[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = f32_to_bf16_bits(acc[i]);
-        *reinterpret_cast<uint4*>(p.out + c) =
-            make_uint4(o[0] | (o[1] << 16), o[2] | (o[3] << 16), o[4] | (o[5] << 16), o[6] | (o[7] << 16));
-        if (p.x_next != nullptr) {
-          const uint4 xv = __ldg(reinterpret_cast<const uint4*>(p.x + c));
-          const uint32_t xs[8] = {xv.x & 0xFFFF, xv.x >> 16, xv.y & 0xFFFF, xv.y >> 16,
-                                  xv.z & 0xFFFF, xv.z >> 16, xv.w & 0xFFFF, xv.w >> 16};
-          uint32_t rr[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) rr[i] = f32_to_bf16_bits(bf16_bits_to_f32(xs[i]) + bf16_bits_to_f32(o[i]));
-          *reinterpret_cast<uint4*>(p.x_next + c) =
-              make_uint4(rr[0] | (rr[1] << 16), rr[2] | (rr[3] << 16), rr[4] | (rr[5] << 16), rr[6] | (rr[7] << 16));
-        }
+        if (n) __threadfence();
       }
+      *s_ok = n;
+    }
+    named_bar_sync(1, 32 * kNW);
+    for (int i = warp; i < *s_ok; i += kNW) {
+      const int c = 32 * s_last[i] + lane;
+      float a = 0.0f;
+      for (int jj = 0; jj < k; ++jj) a = fmaf(s_w[jj], __ldcg(p.y + (size_t)jj * H + c), a);
+      const uint32_t o = f32_to_bf16_bits(a);
+      p.out[c] = (uint16_t)o;
+      if (p.x_next != nullptr) p.x_next[c] = (uint16_t)f32_to_bf16_bits(bf16_bits_to_f32(__ldg(p.x + c)) + bf16_bits_to_f32(o));
     }
   }
 }
@@ -367,9 +444,9 @@ template <int UG, int UD>
 int launch_d1(const D1Params& p, int num_sms, cudaStream_t s) {
   constexpr int H = UG * 1024, I = UD * 512;
   constexpr int kStage1 = 2 * (kNW * H / 2 + kNW * H / 16);
-  constexpr int kStage2 = 2 * kNW * I / 2 + 2 * kNW * I / 16;
+  constexpr int kStage2 = 4 * kNW * I / 2 + 4 * kNW * I / 16;
   constexpr int kStage = kStage1 > kStage2 ? kStage1 : kStage2;
-  const int smem = kRing * kStage + 2 * kRing * 8 + 5 * kMaxK * 4 + 16;
+  const int smem = kRing * kStage + H * 2 + 2 * I * 4 + (2 * kRing + 1) * 8 + 5 * kMaxK * 4 + 4 + 4 * kMaxLast;
   auto kern = decode1_kernel<UG, UD>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return -(int)err;
@@ -390,8 +467,8 @@ int launch_d1(const D1Params& p, int num_sms, cudaStream_t s) {
 
 }  // namespace
 
-bool decode1_supported(int H, int I, int k) {
-  if (k > kMaxK) return false;
+bool decode1_supported(int H, int I, int k, int num_sms) {
+  if (k > kMaxK || H / 32 > kMaxBlocks || num_sms < 1 || (k * (H / 32) + num_sms - 1) / num_sms > kMaxLast) return false;
   return (H == 5120 && I == 2560) || (H == 1024 && I == 512) || (H == 2048 && I == 1024) ||
          (H == 4096 && I == 1536);
 }
@@ -419,7 +496,7 @@ int launch_decode1(const BankView& bank, const float* logits, int k, const uint1
   p.bar = bar;
   p.ids = ids;
   p.w = w;
-  cudaError_t err = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned), s);
+  cudaError_t err = cudaMemsetAsync(bar, 0, (kMaxK + bank.H / 32) * sizeof(unsigned), s);
   if (err != cudaSuccess) return -(int)err;
   if (bank.H == 5120 && bank.I == 2560) return launch_d1<5, 5>(p, num_sms, s);
   if (bank.H == 1024 && bank.I == 512) return launch_d1<1, 1>(p, num_sms, s);

@@ -108,7 +108,7 @@ WsLayout ws_layout(int64_t T, int E, int k, int H, int I, int path) {
   L.singles = take((size_t)E * 16);
   L.nsingles = take(4);
   L.chunk_counts = take(T > moe::kRouteChunk ? (size_t)moe::route_chunks(T) * E * 4 : 0);
-  L.bar = take(8);
+  L.bar = take(moe::kDecode1BarBytes);
   L.h = take(R * (size_t)I * 4);
   L.y = take(R * (size_t)H * 4);
   L.total = o;
@@ -365,7 +365,7 @@ int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
   moe::RouteBufs rb = route_bufs(w8, L);
   const moe::BankView bv = view_of(bank);
   int launches = 0;
-  if (T == 1 && moe::decode1_supported(H, I, k)) {
+  if (T == 1 && moe::decode1_supported(H, I, k, info.sms)) {
     prof_before(MOE_NVFP4_KERNEL_DECODE_FUSED, s);
     if ((rc = after_launch(moe::launch_decode1(bv, logits, k, static_cast<const uint16_t*>(x),
                                                static_cast<uint16_t*>(out), static_cast<uint16_t*>(x_next),
