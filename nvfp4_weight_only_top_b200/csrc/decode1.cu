@@ -4,8 +4,8 @@
 // With one token every routed row is its own expert, the work is 2 FLOP per weight byte, and
 // the layer is a pure stream of k expert records (177 MB at E=256, k=8, H=5120, I=2560) from
 // HBM.  What costs time besides the bytes is the number of dependent steps, so:
-//   * every CTA routes the token itself (top-k of E logits, the router of route_warp.cuh):
-//     no router kernel, no hand-off;
+//   * every CTA routes the token itself (top-k of E logits in the router's order: logit
+//     descending, lower index first; softmax over the k in f32): no router kernel, no hand-off;
 //   * one producer warp per CTA streams the CTA's weight rows with large 1-D bulk copies
 //     (TMA) into a 4-stage shared-memory ring -- first its share of the gate/up rows, then,
 //     without waiting for anything, its share of the down rows;
@@ -38,6 +38,7 @@ constexpr int kRing = 4;                     // stages in the ring
 constexpr int kMaxK = 32;
 constexpr int kMaxBlocks = 256;              // H / 32 row blocks of the combine
 constexpr int kMaxLast = 64;                 // down stages of one CTA (bound checked on the host)
+constexpr int kMaxRankE = 256;               // experts routed by the in-kernel rank count
 
 struct D1Params {
   const uint8_t* bank;
@@ -142,12 +143,16 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
   constexpr int kStage2 = kCodes2 + kScales2;
   constexpr int kStage = kStage1 > kStage2 ? kStage1 : kStage2;
   constexpr int kUnits2 = I / 32;                                     // units per down row
+  static_assert((kRing * kStage + H * 2 + 2 * I * 4) % 16 == 0, "16-byte alignment of the routing keys");
 
   extern __shared__ __align__(128) uint8_t smem[];
   // ring | x (bf16 [H]) | h of up to two slots (f32 [2][I]) | barriers, routing
   uint16_t* sx = reinterpret_cast<uint16_t*>(smem + kRing * kStage);
   float* sh = reinterpret_cast<float*>(sx + H);
-  uint64_t* full = reinterpret_cast<uint64_t*>(sh + 2 * I);
+  // Routing keys first: they are read as 16-byte pairs and need 16-byte alignment (the
+  // offset here is a multiple of 16: ring stages, x and h all are).
+  uint64_t* s_key = reinterpret_cast<uint64_t*>(sh + 2 * I);  // [kMaxRankE] routing keys
+  uint64_t* full = s_key + kMaxRankE;
   uint64_t* empty = full + kRing;
   uint64_t* gm_full = empty + kRing;                        // the global multipliers are in s_gm
   int* s_ids = reinterpret_cast<int*>(gm_full + 1);
@@ -174,20 +179,55 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
     *s_ok = 1;
     fence_barrier_init();
   }
-  if (warp != 0) {                                          // x into shared memory, once
-    // 16-byte chunk c of 32-input unit u is stored at chunk c ^ ((u >> 1) & 3) of the unit, so
+  // Every CTA routes the token itself.  Expert e's rank is the number of experts ahead of it
+  // in the order (logit desc, index asc) -- the order of the warp router -- counted by one
+  // thread per expert against all E keys; the experts of rank < k fill slots 0 .. k-1.
+  {
+    // The logit and this thread's share of x are loaded together; x goes to shared memory once
+    // per CTA, 16-byte chunk c of 32-input unit u at chunk c ^ ((u >> 1) & 3) of the unit, so
     // that the lanes of a warp, which read consecutive units, hit different banks.
-    for (int i = (int)threadIdx.x - 32; i < H / 8; i += (int)blockDim.x - 32) {
-      const int u = i >> 2, c = i & 3;
-      reinterpret_cast<uint4*>(sx)[4 * u + (c ^ ((u >> 1) & 3))] = __ldg(reinterpret_cast<const uint4*>(p.x) + i);
+    const int e = threadIdx.x;
+    const float lg = (e < kMaxRankE && e < p.E) ? __ldg(p.logits + e) : 0.0f;
+    constexpr int kXPer = (H / 8 + kThreads1 - 1) / kThreads1;
+    uint4 xv[kXPer];
+#pragma unroll
+    for (int t = 0; t < kXPer; ++t) {
+      const int i = (int)threadIdx.x + t * kThreads1;
+      if (i < H / 8) xv[t] = __ldg(reinterpret_cast<const uint4*>(p.x) + i);
+    }
+    if (e < kMaxRankE) s_key[e] = e < p.E ? ((uint64_t)rank_key(lg) << 32) | (uint32_t)(0xFFFFFFFFu - e) : 0ull;
+#pragma unroll
+    for (int t = 0; t < kXPer; ++t) {
+      const int i = (int)threadIdx.x + t * kThreads1;
+      if (i < H / 8) {
+        const int u = i >> 2, c = i & 3;
+        reinterpret_cast<uint4*>(sx)[4 * u + (c ^ ((u >> 1) & 3))] = xv[t];
+      }
     }
   }
-  if (warp == 0) {                                          // every CTA routes the token
-    int id;
-    float wt;
-    route_row(p.logits, p.E, k, lane, id, wt);
+  __syncthreads();
+  if (threadIdx.x < p.E) {
+    const uint64_t me = s_key[threadIdx.x];
+    int ahead = 0;
+    const ulonglong2* kk = reinterpret_cast<const ulonglong2*>(s_key);
+#pragma unroll 8
+    for (int i = 0; i < kMaxRankE / 2; ++i) {              // keys beyond E are 0: never ahead
+      const ulonglong2 v = kk[i];
+      ahead += (v.x > me) + (v.y > me);
+    }
+    if (ahead < k) s_ids[ahead] = threadIdx.x;
+  }
+  __syncthreads();
+  if (warp == 0) {                                          // softmax over the k selected
+    const int id = lane < k ? s_ids[lane] : 0;
+    const float l = lane < k ? __ldg(p.logits + id) : 0.0f;
+    const float lmax = __shfl_sync(0xFFFFFFFFu, l, 0);
+    const float ex = lane < k ? expf(l - lmax) : 0.0f;
+    float sum = ex;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
+    const float wt = ex / sum;
     if (lane < k) {
-      s_ids[lane] = id;
       s_w[lane] = wt;
       if (blockIdx.x == 0) {
         p.ids[lane] = id;
@@ -446,7 +486,8 @@ int launch_d1(const D1Params& p, int num_sms, cudaStream_t s) {
   constexpr int kStage1 = 2 * (kNW * H / 2 + kNW * H / 16);
   constexpr int kStage2 = 4 * kNW * I / 2 + 4 * kNW * I / 16;
   constexpr int kStage = kStage1 > kStage2 ? kStage1 : kStage2;
-  const int smem = kRing * kStage + H * 2 + 2 * I * 4 + (2 * kRing + 1) * 8 + 5 * kMaxK * 4 + 4 + 4 * kMaxLast;
+  const int smem =
+      kRing * kStage + H * 2 + 2 * I * 4 + (2 * kRing + 1) * 8 + kMaxRankE * 8 + 5 * kMaxK * 4 + 4 + 4 * kMaxLast;
   auto kern = decode1_kernel<UG, UD>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return -(int)err;
@@ -467,8 +508,8 @@ int launch_d1(const D1Params& p, int num_sms, cudaStream_t s) {
 
 }  // namespace
 
-bool decode1_supported(int H, int I, int k, int num_sms) {
-  if (k > kMaxK || H / 32 > kMaxBlocks || num_sms < 1 || (k * (H / 32) + num_sms - 1) / num_sms > kMaxLast) return false;
+bool decode1_supported(int H, int I, int k, int E, int num_sms) {
+  if (E > kMaxRankE || k > kMaxK || H / 32 > kMaxBlocks || num_sms < 1 || (k * (H / 32) + num_sms - 1) / num_sms > kMaxLast) return false;
   return (H == 5120 && I == 2560) || (H == 1024 && I == 512) || (H == 2048 && I == 1024) ||
          (H == 4096 && I == 1536);
 }

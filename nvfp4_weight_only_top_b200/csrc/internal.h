@@ -71,7 +71,7 @@ size_t decode_smem_bytes(int K, int xrows, bool gateup);
 // memset of its completion counters in bar, kDecode1BarBytes).  h [k, I] and y [k, H] are f32
 // scratch.
 constexpr size_t kDecode1BarBytes = (32 + 256) * 4;
-bool decode1_supported(int H, int I, int k, int num_sms);
+bool decode1_supported(int H, int I, int k, int E, int num_sms);
 int launch_decode1(const BankView& bank, const float* logits, int k, const uint16_t* x, uint16_t* out,
                    uint16_t* x_next, float* h, float* y, unsigned* bar, int32_t* ids, float* w, int num_sms,
                    cudaStream_t s);

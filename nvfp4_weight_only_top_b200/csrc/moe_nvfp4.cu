@@ -365,7 +365,7 @@ int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
   moe::RouteBufs rb = route_bufs(w8, L);
   const moe::BankView bv = view_of(bank);
   int launches = 0;
-  if (T == 1 && moe::decode1_supported(H, I, k, info.sms)) {
+  if (T == 1 && moe::decode1_supported(H, I, k, E, info.sms)) {
     prof_before(MOE_NVFP4_KERNEL_DECODE_FUSED, s);
     if ((rc = after_launch(moe::launch_decode1(bv, logits, k, static_cast<const uint16_t*>(x),
                                                static_cast<uint16_t*>(out), static_cast<uint16_t*>(x_next),
