@@ -15,15 +15,21 @@
 //   * eight consumer warps dot the rows against the activations held in registers (f16, the
 //     lane's own K positions) with packed f16 FMAs per 16-input block, fold each block into
 //     f32 with its E4M3 scale, and reduce across the warp;
-//   * the combine of a block of 32 output rows is done by the warp that writes the block's
-//     last y values (a per-block counter), in slot order with f32 accumulation and one BF16
-//     rounding (and the optional residual), exactly as the combine kernel does.
+//   * the combine of a block of 32 output rows is done by the CTA that writes the block's last
+//     y values (a per-block counter), in slot order with f32 accumulation and one BF16
+//     rounding (and the optional residual), exactly as the combine kernel does;
+//   * the completion counters come from a library-owned pool of counter sets that every call
+//     leaves at zero (the last CTA clears its set), so a call is this one launch, nothing else.
 //
 // Weight layout: page "Beam 1.0 501B-A23B, streaming pack, NVFP4 experts / MLX 8-bit
 // residents", section "What this pack holds"; router logits and SwiGLU in FP32: page
 // "Beam-1.0-501B-A23B VQ GGUF", section "What stays native".  The pages' "flat decode MoE
 // scheduler" (page "Beam-1.0-501B-A23B, EXL3 3-bit, for 2x RTX PRO 6000 Blackwell", section
 // "How it fits") likewise runs decode over one flat work list across experts.
+#include <atomic>
+#include <mutex>
+#include <vector>
+
 #include "common.cuh"
 #include "internal.h"
 #include "route_warp.cuh"
@@ -39,6 +45,14 @@ constexpr int kMaxK = 32;
 constexpr int kMaxBlocks = 256;              // H / 32 row blocks of the combine
 constexpr int kMaxLast = 64;                 // down stages of one CTA (bound checked on the host)
 constexpr int kMaxRankE = 256;               // experts routed by the in-kernel rank count
+// Completion counters: kMaxK per-slot counts, kMaxBlocks per-block counts, one exit count.
+constexpr int kCounterWords = kMaxK + kMaxBlocks + 1;
+constexpr int kCounterSets = 64;             // calls that may be in flight at once per device
+
+// Counter sets owned by the library, one used per call in turn.  They start at zero (module
+// load) and each call leaves its set at zero again (the last CTA to finish clears it), so no
+// call needs a memset.
+__device__ unsigned g_d1_counters[kCounterSets][kCounterWords];
 
 struct D1Params {
   const uint8_t* bank;
@@ -52,7 +66,7 @@ struct D1Params {
   uint16_t* x_next;      // [H] bf16 or null
   float* h;              // [k, I] f32 scratch
   float* y;              // [k, H] f32 scratch
-  unsigned* bar;         // [kMaxK + H/32] completion counters, zero on entry
+  unsigned* bar;         // [kCounterWords] completion counters: zero on entry, zero again on exit
   int32_t* ids;          // [k] routing result (for inspection)
   float* w;              // [k]
 };
@@ -469,6 +483,18 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
       *s_ok = n;
     }
     named_bar_sync(1, 32 * kNW);
+    // The last CTA through here clears the counter set for the call that uses it next.
+    if (threadIdx.x == 0) {
+      unsigned* exit_count = p.bar + kMaxK + kMaxBlocks;
+      __threadfence();
+      if (atomicAdd(exit_count, 1u) == gridDim.x - 1) {
+        __threadfence();                    // every other CTA's counter updates come before
+        for (int i = 0; i < kMaxK; ++i) slot_done[i] = 0;
+        for (int i = 0; i < H / 32; ++i) block_done[i] = 0;
+        *exit_count = 0;
+        __threadfence();
+      }
+    }
     for (int i = warp; i < *s_ok; i += kNW) {
       const int c = 32 * s_last[i] + lane;
       float a = 0.0f;
@@ -514,9 +540,35 @@ bool decode1_supported(int H, int I, int k, int E, int num_sms) {
          (H == 4096 && I == 1536);
 }
 
+// Device address of this device's counter sets (the current device), resolved once.
+static unsigned* d1_counter_base(int dev) {
+  static std::mutex mu;
+  static std::vector<unsigned*> base;
+  std::lock_guard<std::mutex> lk(mu);
+  if ((int)base.size() <= dev) base.resize(dev + 1, nullptr);
+  if (!base[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_d1_counters) != cudaSuccess) return nullptr;
+    base[dev] = static_cast<unsigned*>(ptr);
+  }
+  return base[dev];
+}
+
+static std::atomic<unsigned> g_d1_next_set{0};
+
+int decode1_reset_counters() {
+  void* ptr = nullptr;
+  cudaError_t err = cudaGetSymbolAddress(&ptr, g_d1_counters);
+  if (err == cudaSuccess) err = cudaMemset(ptr, 0, sizeof(g_d1_counters));
+  return err == cudaSuccess ? 0 : -(int)err;
+}
+
 int launch_decode1(const BankView& bank, const float* logits, int k, const uint16_t* x, uint16_t* out,
-                   uint16_t* x_next, float* h, float* y, unsigned* bar, int32_t* ids, float* w, int num_sms,
+                   uint16_t* x_next, float* h, float* y, int32_t* ids, float* w, int dev, int num_sms,
                    cudaStream_t s) {
+  unsigned* sets = d1_counter_base(dev);
+  if (!sets) return -(int)cudaErrorInvalidSymbol;
+  unsigned* bar = sets + (size_t)(g_d1_next_set.fetch_add(1u) % kCounterSets) * kCounterWords;
   D1Params p{};
   p.bank = bank.base;
   p.stride = bank.stride;
@@ -537,8 +589,6 @@ int launch_decode1(const BankView& bank, const float* logits, int k, const uint1
   p.bar = bar;
   p.ids = ids;
   p.w = w;
-  cudaError_t err = cudaMemsetAsync(bar, 0, (kMaxK + bank.H / 32) * sizeof(unsigned), s);
-  if (err != cudaSuccess) return -(int)err;
   if (bank.H == 5120 && bank.I == 2560) return launch_d1<5, 5>(p, num_sms, s);
   if (bank.H == 1024 && bank.I == 512) return launch_d1<1, 1>(p, num_sms, s);
   if (bank.H == 2048 && bank.I == 1024) return launch_d1<2, 2>(p, num_sms, s);

@@ -67,14 +67,16 @@ int launch_combine(const float* y, const float* w, const int32_t* inv, int64_t T
 
 size_t decode_smem_bytes(int K, int xrows, bool gateup);
 
-// Decode of a single token: route, gate/up, down and combine in one persistent kernel (plus a
-// memset of its completion counters in bar, kDecode1BarBytes).  h [k, I] and y [k, H] are f32
-// scratch.
-constexpr size_t kDecode1BarBytes = (32 + 256) * 4;
+// Decode of a single token: route, gate/up, down and combine in one persistent kernel.  h [k, I]
+// and y [k, H] are f32 scratch; its completion counters come from a library-owned pool of
+// self-clearing counter sets on device dev (the current device).
 bool decode1_supported(int H, int I, int k, int E, int num_sms);
 int launch_decode1(const BankView& bank, const float* logits, int k, const uint16_t* x, uint16_t* out,
-                   uint16_t* x_next, float* h, float* y, unsigned* bar, int32_t* ids, float* w, int num_sms,
+                   uint16_t* x_next, float* h, float* y, int32_t* ids, float* w, int dev, int num_sms,
                    cudaStream_t s);
+// Clears every counter set of the current device (after a kernel gave up on a bounded wait, a
+// set may be left non-zero).  Synchronous.
+int decode1_reset_counters();
 
 // Prefill path: grouped NVFP4 GEMM on tcgen05 tensor cores, groups of up to kPrefillRows rows.
 constexpr int kPrefillRows = 256;
@@ -82,10 +84,11 @@ bool prefill_supported(int H, int I);
 // xp [R, H] bf16 = x[perm[r] / k] for every routed row r (expert order).
 int launch_gather(const uint16_t* x, const int32_t* perm, int k, int64_t R, int H, void* xp, cudaStream_t s);
 // hb [R, I] bf16 = silu(xp Wg^T gg) * (xp Wu^T gu).
+// tile_ctr: a counter zeroed before the launch (tiles are handed out dynamically).
 int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const RouteBufs& rb, void* hb,
-                          int num_sms, cudaStream_t s);
+                          unsigned* tile_ctr, int num_sms, cudaStream_t s);
 // y [R, H] f32 = hb Wd^T gd.
 int launch_prefill_down(const BankView& bank, const void* hb, int64_t R, const RouteBufs& rb, float* y,
-                        int num_sms, cudaStream_t s);
+                        unsigned* tile_ctr, int num_sms, cudaStream_t s);
 
 }  // namespace moe

@@ -108,7 +108,7 @@ WsLayout ws_layout(int64_t T, int E, int k, int H, int I, int path) {
   L.singles = take((size_t)E * 16);
   L.nsingles = take(4);
   L.chunk_counts = take(T > moe::kRouteChunk ? (size_t)moe::route_chunks(T) * E * 4 : 0);
-  L.bar = take(moe::kDecode1BarBytes);
+  L.bar = take(2 * sizeof(unsigned));        // tile counters of the tensor-core path
   L.h = take(R * (size_t)I * 4);
   L.y = take(R * (size_t)H * 4);
   L.total = o;
@@ -296,6 +296,11 @@ int prefill_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
   const moe::BankView bv = view_of(bank);
   const int64_t R = T * k;
   void* hb = w8 + L.h;
+  unsigned* tile_ctr = reinterpret_cast<unsigned*>(w8 + L.bar);   // two tile counters, zeroed here
+  {
+    const cudaError_t e = cudaMemsetAsync(tile_ctr, 0, 2 * sizeof(unsigned), s);
+    if (e != cudaSuccess) return cuda_fail(e, "clear tile counters");
+  }
   void* xp = w8 + L.y;
   float* y = reinterpret_cast<float*>(w8 + L.y);
   int launches = 0;
@@ -306,11 +311,11 @@ int prefill_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
                          &launches)))
     return rc;
   prof_before(MOE_NVFP4_KERNEL_PREFILL_GATEUP, s);
-  if ((rc = after_launch(moe::launch_prefill_gateup(bv, xp, R, rb, hb, info.sms, s), s, "prefill gate/up",
+  if ((rc = after_launch(moe::launch_prefill_gateup(bv, xp, R, rb, hb, tile_ctr, info.sms, s), s, "prefill gate/up",
                          &launches)))
     return rc;
   prof_before(MOE_NVFP4_KERNEL_PREFILL_DOWN, s);
-  if ((rc = after_launch(moe::launch_prefill_down(bv, hb, R, rb, y, info.sms, s), s, "prefill down", &launches)))
+  if ((rc = after_launch(moe::launch_prefill_down(bv, hb, R, rb, y, tile_ctr + 1, info.sms, s), s, "prefill down", &launches)))
     return rc;
   prof_before(MOE_NVFP4_KERNEL_COMBINE, s);
   if ((rc = after_launch(moe::launch_combine(y, rb.w, rb.inv, T, k, H, static_cast<const uint16_t*>(x),
@@ -370,7 +375,7 @@ int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
     if ((rc = after_launch(moe::launch_decode1(bv, logits, k, static_cast<const uint16_t*>(x),
                                                static_cast<uint16_t*>(out), static_cast<uint16_t*>(x_next),
                                                reinterpret_cast<float*>(w8 + L.h), reinterpret_cast<float*>(w8 + L.y),
-                                               reinterpret_cast<unsigned*>(w8 + L.bar), rb.ids, rb.w, info.sms, s),
+                                               rb.ids, rb.w, dev, info.sms, s),
                            s, "fused single-token decode", &launches)))
       return rc;
     t_last_launches = launches;
@@ -544,7 +549,12 @@ int moe_nvfp4_device_status(void) {
   const int zero = 0;
   e = cudaMemcpyToSymbol(moe::g_status, &zero, sizeof(int));
   if (e != cudaSuccess) return cuda_fail(e, "clear device status");
-  if (v != 0) return fail(MOE_NVFP4_ERR_TIMEOUT, "a bounded device wait gave up (status %d)", v);
+  if (v != 0) {
+    // A kernel that gave up may have left its completion counters set: clear them all.
+    const int rc = moe::decode1_reset_counters();
+    if (rc < 0) return cuda_fail((cudaError_t)(-rc), "clear decode counters");
+    return fail(MOE_NVFP4_ERR_TIMEOUT, "a bounded device wait gave up (status %d)", v);
+  }
   return MOE_NVFP4_OK;
 }
 

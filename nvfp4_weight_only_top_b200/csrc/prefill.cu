@@ -20,6 +20,11 @@
 // After a tile's last K stage warps 0-3 read the accumulators back with tcgen05.ld and apply
 // the global scale (and SwiGLU for gate/up, whose result h is stored as BF16).
 //
+// Tiles are handed out dynamically: the weight-TMA thread takes the next tile index from a
+// global counter and passes it to the other roles through a small queue in shared memory.
+// The router lists the groups with a full 256 rows first, so the large tiles go out first and
+// the small remainder tiles fill in at the end.
+//
 // Weight layout: page "Beam 1.0 501B-A23B, streaming pack, NVFP4 experts / MLX 8-bit
 // residents", section "What this pack holds"; SwiGLU in FP32: page "Beam-1.0-501B-A23B VQ
 // GGUF", section "What stays native".  The pages' prefill kernels ("decode-once prefill MoE
@@ -47,11 +52,13 @@ constexpr int kBBytes = kMaxN * kKC * 2;       // 32 KB: activations of one stag
 constexpr int kWBytes = kBM * kKC / 2;         // 4 KB: codes of one M-tile of one stage
 constexpr int kSBytes = kBM * 16;              // 2 KB: scales of one M-tile, 4 stages
 constexpr int kTmemCols = 512;                 // two 256-column f32 accumulators
+constexpr int kTQ = 4;                         // tile queue entries
+constexpr int kTQConsumers = 4 + 1 + 1;        // producer warps, activation TMA, MMA
 constexpr int kOffB = kStages * 2 * kABytes;
 constexpr int kOffW = kOffB + kStages * kBBytes;
 constexpr int kOffS = kOffW + kWStages * 2 * kWBytes;
 constexpr int kOffBar = kOffS + kSStages * 2 * kSBytes;
-constexpr int kSmemBytes = kOffBar + 256 /*barriers*/ + 1024 /*alignment*/;
+constexpr int kSmemBytes = kOffBar + 512 /*barriers, tile queue*/ + 1024 /*alignment*/;
 static_assert(kSmemBytes <= 232448, "shared memory per block");
 
 struct PrefillParams {
@@ -64,6 +71,7 @@ struct PrefillParams {
   int gateup;              // 1: M-tile 0 = gate rows, M-tile 1 = same up rows; 0: 256 consecutive rows
   const int4* groups;      // (expert, first permuted row, rows <= 256, 0)
   const int32_t* ngroups;
+  unsigned* tile_ctr;      // tiles handed out so far (zero at launch)
   void* out;               // gate/up: h bf16 [R, out_stride]; down: y f32 [R, out_stride]
   int out_stride;
 };
@@ -125,14 +133,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_empty = s_full + kSStages;                // [kSStages]
   uint64_t* d_full = s_empty + kSStages;                // MMA commit -> epilogue
   uint64_t* d_empty = d_full + 1;                       // epilogue -> MMA
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_empty + 1);
+  uint64_t* tq_full = d_empty + 1;                      // [kTQ] scheduler -> roles
+  uint64_t* tq_empty = tq_full + kTQ;                   // [kTQ] roles -> scheduler
+  int* s_tq = reinterpret_cast<int*>(tq_empty + kTQ);   // [kTQ] tile index, -1 = no more
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_tq + kTQ);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = *p.ngroups * p.tiles_per_group;
   const int nst = p.K / kKC;                            // stages per tile (a multiple of 4)
-  const int total = (ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;  // tiles of this CTA
-  const int nq = total * nst;
   const TileCursor cur{p.tiles_per_group};
+  // Takes tile number i of this CTA from the queue (every role sees the same sequence).
+  auto pop_tile = [&](int i, int& tt) -> bool {
+    const int slot = i % kTQ;
+    if (!mbar_wait(&tq_full[slot], (i / kTQ) & 1)) return false;
+    tt = ((volatile int*)s_tq)[slot];
+    return true;
+  };
 
   if (threadIdx.x == 0) {
     // Producer-side barriers count one arrival per producer warp (lane 0 after __syncwarp):
@@ -152,6 +168,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(d_full, 1);
     mbar_init(d_empty, 4);
+    for (int s = 0; s < kTQ; ++s) {
+      mbar_init(&tq_full[s], 1);
+      mbar_init(&tq_empty[s], kTQConsumers);
+    }
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -199,9 +219,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     };
-    auto epilogue = [&](int i) {
+    auto epilogue = [&](int tt, int i) {
       int g, m;
-      cur.at((int)blockIdx.x + i * (int)gridDim.x, g, m);
+      cur.at(tt, g, m);
       const int4 grp = __ldg(&p.groups[g]);
       const uint8_t* rec = p.bank + (uint64_t)grp.x * p.stride;
       const float gm0 = global_mult(__ldg(reinterpret_cast<const float*>(rec + p.global_off[0])), p.global_mode);
@@ -240,43 +260,57 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     bool ok = true;
     const int first = nst < kStages ? nst : kStages;   // stages of a tile stored before the previous epilogue
-    for (int q = 0; q < nq && ok; ++q) {
-      const int c = q % nst;
-      const int ws = q % kWStages, ss = (q >> 2) % kSStages;
-      const bool got = mbar_wait(&w_full[ws], (q / kWStages) & 1) &&
-                       ((c & 3) != 0 || mbar_wait(&s_full[ss], ((q >> 2) / kSStages) & 1));
-      if (!__all_sync(0xffffffffu, got)) {     // warp-uniform: the warp arrives as one below
+    int q = 0, i = 0, prev = -1;
+    for (; ok; ++i) {
+      int tt = -1;
+      if (!__all_sync(0xffffffffu, pop_tile(i, tt))) {
         ok = false;
         break;
       }
-      StageFrag f;
-      fetch(q, f);
-      const int s = q % kStages;
-      if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ((q / kStages) & 1) ^ 1))) {
-        ok = false;
-        break;
-      }
-      store(s, f);
-      fence_proxy_async_smem();
       __syncwarp();
-      // The raw slots go back to the TMA only after every lane's proxy fence above: a TMA
-      // write (async proxy) into a slot that was read with generic loads must be ordered
-      // after those reads, or it can overtake them.
-      if (lane == 0) {
-        mbar_arrive(&a_full[s]);
-        mbar_arrive(&w_empty[ws]);
-        if ((c & 3) == 3) mbar_arrive(&s_empty[ss]);
+      if (lane == 0) mbar_arrive(&tq_empty[i % kTQ]);
+      if (tt < 0) break;
+      for (int c = 0; c < nst; ++c, ++q) {
+        const int ws = q % kWStages, ss = (q >> 2) % kSStages;
+        const bool got = mbar_wait(&w_full[ws], (q / kWStages) & 1) &&
+                         ((c & 3) != 0 || mbar_wait(&s_full[ss], ((q >> 2) / kSStages) & 1));
+        if (!__all_sync(0xffffffffu, got)) {     // warp-uniform: the warp arrives as one below
+          ok = false;
+          break;
+        }
+        StageFrag f;
+        fetch(q, f);
+        const int s = q % kStages;
+        if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ((q / kStages) & 1) ^ 1))) {
+          ok = false;
+          break;
+        }
+        store(s, f);
+        fence_proxy_async_smem();
+        __syncwarp();
+        // The raw slots go back to the TMA only after every lane's proxy fence above: a TMA
+        // write (async proxy) into a slot that was read with generic loads must be ordered
+        // after those reads, or it can overtake them.
+        if (lane == 0) {
+          mbar_arrive(&a_full[s]);
+          mbar_arrive(&w_empty[ws]);
+          if ((c & 3) == 3) mbar_arrive(&s_empty[ss]);
+        }
+        if (i > 0 && c == first - 1) epilogue(prev, i - 1);
       }
-      const int i = q / nst;
-      if (i > 0 && c == first - 1) epilogue(i - 1);
+      prev = tt;
     }
-    if (ok && total > 0) epilogue(total - 1);
+    if (ok && i > 0) epilogue(prev, i - 1);
   } else if (warp == 4) {
     // ------------------------------------------------------------ activation TMA
     if (lane == 0) {
       int q = 0;
       bool ok = true;
-      for (int tt = blockIdx.x; tt < ntiles && ok; tt += gridDim.x) {
+      for (int i = 0; ok; ++i) {
+        int tt = -1;
+        if (!pop_tile(i, tt)) break;
+        mbar_arrive(&tq_empty[i % kTQ]);
+        if (tt < 0) break;
         const int4 grp = __ldg(&p.groups[tt / p.tiles_per_group]);
         const int nbox = (grp.z + kBoxRows - 1) / kBoxRows;
         for (int c = 0; c < nst; ++c, ++q) {
@@ -299,34 +333,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       bool ok = true;
       int q = 0, qs = 0;
-      for (; q < nq && ok; ++q) {
-        const int i = q / nst, c = q - i * nst;
+      for (int i = 0; ok; ++i) {
+        // Next tile for every role of this CTA.
+        const int slot = i % kTQ;
+        if (!mbar_wait(&tq_empty[slot], ((i / kTQ) & 1) ^ 1)) break;
+        int tt = (int)atomicAdd(p.tile_ctr, 1u);
+        if (tt >= ntiles) tt = -1;
+        ((volatile int*)s_tq)[slot] = tt;
+        mbar_arrive(&tq_full[slot]);
+        if (tt < 0) break;
         int g, m;
-        cur.at((int)blockIdx.x + i * (int)gridDim.x, g, m);
+        cur.at(tt, g, m);
         const int e = __ldg(&p.groups[g].x);
-        if ((c & 3) == 0) {                       // scales of stages c .. c+3
-          const int ss = qs % kSStages;
-          if (!mbar_wait(&s_empty[ss], ((qs / kSStages) & 1) ^ 1)) {
+        for (int c = 0; c < nst && ok; ++c, ++q) {
+          if ((c & 3) == 0) {                       // scales of stages c .. c+3
+            const int ss = qs % kSStages;
+            if (!mbar_wait(&s_empty[ss], ((qs / kSStages) & 1) ^ 1)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&s_full[ss], 2 * kSBytes);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+              tma_load_3d(sS + (ss * 2 + mt) * kSBytes, &maps.scales[mt], (c >> 2) * 16, row0_of(p, m, mt), e,
+                          &s_full[ss]);
+            ++qs;
+          }
+          const int ws = q % kWStages;
+          if (!mbar_wait(&w_empty[ws], ((q / kWStages) & 1) ^ 1)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&s_full[ss], 2 * kSBytes);
+          mbar_arrive_expect_tx(&w_full[ws], 2 * kWBytes);
 #pragma unroll
           for (int mt = 0; mt < 2; ++mt)
-            tma_load_3d(sS + (ss * 2 + mt) * kSBytes, &maps.scales[mt], (c >> 2) * 16, row0_of(p, m, mt), e,
-                        &s_full[ss]);
-          ++qs;
+            tma_load_3d(sW + (ws * 2 + mt) * kWBytes, &maps.codes[mt], c * (kKC / 2), row0_of(p, m, mt), e,
+                        &w_full[ws]);
         }
-        const int ws = q % kWStages;
-        if (!mbar_wait(&w_empty[ws], ((q / kWStages) & 1) ^ 1)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&w_full[ws], 2 * kWBytes);
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-          tma_load_3d(sW + (ws * 2 + mt) * kWBytes, &maps.codes[mt], c * (kKC / 2), row0_of(p, m, mt), e,
-                      &w_full[ws]);
       }
       // Leave no copy in flight (only an error path gets here with copies outstanding).
       for (int j = max(0, q - kWStages); j < q; ++j) mbar_wait(&w_full[j % kWStages], (j / kWStages) & 1);
@@ -336,9 +379,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      int q = 0, i = 0;
+      int q = 0;
       bool ok = true;
-      for (int tt = blockIdx.x; tt < ntiles && ok; tt += gridDim.x, ++i) {
+      for (int i = 0; ok; ++i) {
+        int tt = -1;
+        if (!pop_tile(i, tt)) break;
+        mbar_arrive(&tq_empty[i % kTQ]);
+        if (tt < 0) break;
         const int4 grp = __ldg(&p.groups[tt / p.tiles_per_group]);
         const int N = (grp.z + 15) & ~15;
         const uint32_t idesc = idesc_bf16(kBM, N);
@@ -466,7 +513,7 @@ int launch_gather(const uint16_t* x, const int32_t* perm, int k, int64_t R, int 
 }
 
 int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const RouteBufs& rb, void* hb,
-                          int num_sms, cudaStream_t s) {
+                          unsigned* tile_ctr, int num_sms, cudaStream_t s) {
   Maps maps;
   int rc = make_rows_map(&maps.x, xp, R, bank.H);
   if (!rc) rc = make_weight_maps(&maps, bank, 0, 1, bank.I, bank.H);
@@ -482,13 +529,14 @@ int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const
   p.gateup = 1;
   p.groups = rb.groups;
   p.ngroups = rb.ngroups;
+  p.tile_ctr = tile_ctr;
   p.out = hb;
   p.out_stride = bank.I;
   return launch_prefill(p, maps, num_sms, s);
 }
 
 int launch_prefill_down(const BankView& bank, const void* hb, int64_t R, const RouteBufs& rb, float* y,
-                        int num_sms, cudaStream_t s) {
+                        unsigned* tile_ctr, int num_sms, cudaStream_t s) {
   Maps maps;
   int rc = make_rows_map(&maps.x, hb, R, bank.I);
   if (!rc) rc = make_weight_maps(&maps, bank, 2, 2, bank.H, bank.I);
@@ -504,6 +552,7 @@ int launch_prefill_down(const BankView& bank, const void* hb, int64_t R, const R
   p.gateup = 0;
   p.groups = rb.groups;
   p.ngroups = rb.ngroups;
+  p.tile_ctr = tile_ctr;
   p.out = y;
   p.out_stride = bank.H;
   return launch_prefill(p, maps, num_sms, s);

@@ -56,33 +56,38 @@ __device__ int block_scan_excl(int* a, int n, int* warp_tmp) {
 
 // From per-expert counts in shared memory: offsets and the two group lists.  An expert's rows
 // are cut into groups of group_rows; when split_singles is set, a last group of a single row
-// goes to the one-row list instead.
-__device__ void finish_counts(int* cnt, int* tmp, int* tmp1, int* warp_tmp, int E, int group_rows,
+// goes to the one-row list instead.  All full groups (exactly group_rows rows) come first, in
+// expert order, then the partial ones: a kernel that hands out groups in list order starts
+// with the large work items and fills in with the small ones.
+__device__ void finish_counts(int* cnt, int* tmp, int* tmp1, int* tmp2, int* warp_tmp, int E, int group_rows,
                               const RouteBufs& b) {
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const int c = cnt[e], full = c / group_rows, r = c - full * group_rows;
     const int single = (b.split_singles && r == 1) ? 1 : 0;
     b.counts[e] = c;
-    tmp[e] = full + ((r > 0 && !single) ? 1 : 0);
+    tmp[e] = full;
+    tmp2[e] = (r > 0 && !single) ? 1 : 0;
     tmp1[e] = single;
   }
   __syncthreads();
-  const int ng = block_scan_excl(tmp, E, warp_tmp);         // tmp: first multi-row group of e
+  const int nf = block_scan_excl(tmp, E, warp_tmp);         // tmp: first full group of e
+  const int np = block_scan_excl(tmp2, E, warp_tmp);        // tmp2: its partial group, after the full ones
   const int ns = block_scan_excl(tmp1, E, warp_tmp);        // tmp1: its one-row group slot
   const int R = block_scan_excl(cnt, E, warp_tmp);          // cnt -> offsets (in place)
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     b.offsets[e] = cnt[e];
     const int c = b.counts[e];
+    const int full = c / group_rows;
     const int single = (b.split_singles && c % group_rows == 1) ? 1 : 0;
-    const int last = c - single;                 // rows that go to multi-row groups
-    int g = tmp[e];
-    for (int q = 0; q * group_rows < last; ++q, ++g)
-      b.groups[g] = make_int4(e, cnt[e] + q * group_rows, min(group_rows, last - q * group_rows), 0);
-    if (single) b.singles[tmp1[e]] = make_int4(e, cnt[e] + last, 1, 0);
+    const int rest = c - full * group_rows - single;        // rows of the partial group
+    for (int q = 0; q < full; ++q)
+      b.groups[tmp[e] + q] = make_int4(e, cnt[e] + q * group_rows, group_rows, 0);
+    if (rest > 0) b.groups[nf + tmp2[e]] = make_int4(e, cnt[e] + full * group_rows, rest, 0);
+    if (single) b.singles[tmp1[e]] = make_int4(e, cnt[e] + c - 1, 1, 0);
   }
   if (threadIdx.x == 0) {
     b.offsets[E] = R;
-    *b.ngroups = ng;
+    *b.ngroups = nf + np;
     *b.nsingles = ns;
   }
 }
@@ -90,7 +95,7 @@ __device__ void finish_counts(int* cnt, int* tmp, int* tmp1, int* warp_tmp, int 
 // Single-CTA routing for T <= kRouteChunk: router, histogram, scan, groups, stable scatter.
 __global__ void __launch_bounds__(512) route_small_kernel(const float* __restrict__ logits,
                                                           int T, int E, int k, RouteBufs b) {
-  __shared__ int cnt[kMaxE], tmp[kMaxE], tmp1[kMaxE], run[kMaxE], warp_tmp[32];
+  __shared__ int cnt[kMaxE], tmp[kMaxE], tmp1[kMaxE], tmp2[kMaxE], run[kMaxE], warp_tmp[32];
   __shared__ int sids[kRouteChunk * 32];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
@@ -107,7 +112,7 @@ __global__ void __launch_bounds__(512) route_small_kernel(const float* __restric
     }
   }
   __syncthreads();
-  finish_counts(cnt, tmp, tmp1, warp_tmp, E, b.group_rows, b);
+  finish_counts(cnt, tmp, tmp1, tmp2, warp_tmp, E, b.group_rows, b);
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) run[e] = cnt[e];   // cnt now = offsets
   __syncthreads();
@@ -152,7 +157,7 @@ __global__ void __launch_bounds__(256) route_chunk_kernel(const float* __restric
 
 // Multi-CTA routing, step 2 (one CTA): per-expert prefix over chunks, counts, offsets, groups.
 __global__ void __launch_bounds__(1024) route_scan_kernel(int nchunks, int E, RouteBufs b) {
-  __shared__ int cnt[kMaxE], tmp[kMaxE], tmp1[kMaxE], warp_tmp[32];
+  __shared__ int cnt[kMaxE], tmp[kMaxE], tmp1[kMaxE], tmp2[kMaxE], warp_tmp[32];
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int run = 0;
     for (int c = 0; c < nchunks; ++c) {
@@ -164,7 +169,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int nchunks, int E, Ro
     cnt[e] = run;
   }
   __syncthreads();
-  finish_counts(cnt, tmp, tmp1, warp_tmp, E, b.group_rows, b);
+  finish_counts(cnt, tmp, tmp1, tmp2, warp_tmp, E, b.group_rows, b);
 }
 
 // Multi-CTA routing, step 3: stable placement of the chunk's rows.
