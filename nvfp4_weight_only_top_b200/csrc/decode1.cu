@@ -32,11 +32,14 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "decode_fused.cuh"
 #include "route_warp.cuh"
 
 namespace moe {
 
 namespace {
+
+using namespace fused;
 
 constexpr int kNW = 8;                       // consumer warps
 constexpr int kThreads1 = 32 * (kNW + 1);    // + one producer warp
@@ -70,80 +73,6 @@ struct D1Params {
   int32_t* ids;          // [k] routing result (for inspection)
   float* w;              // [k]
 };
-
-__device__ __forceinline__ uint32_t hfma2_(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t r;
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
-  return r;
-}
-__device__ __forceinline__ uint32_t hadd2_(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-__device__ __forceinline__ float2 f16x2_to_f2(uint32_t v) {
-  float a, b;
-  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
-      : "=f"(a), "=f"(b)
-      : "r"(v));
-  return make_float2(a, b);
-}
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ uint32_t lds16(uint32_t addr) {
-  uint16_t v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// One 32-input unit: codes (4 words) and its two E4M3 block scales against 16 f16x2 of x.
-__device__ __forceinline__ float unit_dot(const uint4 c, uint32_t sc2, const uint32_t (&x)[16]) {
-  const float2 sf = f16x2_to_f2(e4m3x2_to_f16x2((uint16_t)sc2));
-  uint32_t e0[4], e1[4], e2[4], e3[4];
-  e2m1x8_to_f16x8(c.x, e0);
-  e2m1x8_to_f16x8(c.y, e1);
-  e2m1x8_to_f16x8(c.z, e2);
-  e2m1x8_to_f16x8(c.w, e3);
-  uint32_t p0 = hfma2_(e0[0], x[0], 0u), p0b = hfma2_(e0[1], x[1], 0u);
-  uint32_t p1 = hfma2_(e2[0], x[8], 0u), p1b = hfma2_(e2[1], x[9], 0u);
-  p0 = hfma2_(e0[2], x[2], p0), p0b = hfma2_(e0[3], x[3], p0b);
-  p1 = hfma2_(e2[2], x[10], p1), p1b = hfma2_(e2[3], x[11], p1b);
-  p0 = hfma2_(e1[0], x[4], p0), p0b = hfma2_(e1[1], x[5], p0b);
-  p1 = hfma2_(e3[0], x[12], p1), p1b = hfma2_(e3[1], x[13], p1b);
-  p0 = hfma2_(e1[2], x[6], p0), p0b = hfma2_(e1[3], x[7], p0b);
-  p1 = hfma2_(e3[2], x[14], p1), p1b = hfma2_(e3[3], x[15], p1b);
-  const float2 a = f16x2_to_f2(hadd2_(p0, p0b)), b = f16x2_to_f2(hadd2_(p1, p1b));
-  return fmaf(sf.x, a.x + a.y, sf.y * (b.x + b.y));
-}
-
-// Waits until *counter reaches target (other CTAs of the persistent grid add to it; all are
-// resident: cooperative launch).  Bounded: gives up after kWaitCycles, records a timeout and
-// returns false.
-__device__ bool wait_count(const unsigned* counter, unsigned target) {
-  const long long t0 = clock64();
-  while (ld_acquire(counter) < target) {
-    if (clock64() - t0 > kWaitCycles) {
-      atomicExch(&g_status, kStatusTimeout);
-      return false;
-    }
-    __nanosleep(64);
-  }
-  return true;
-}
-
-// Contiguous share [lo, hi) of n work units for CTA c of G.
-__device__ __forceinline__ void share(int n, int c, int G, int& lo, int& hi) {
-  lo = (int)(((long long)n * c) / G);
-  hi = (int)(((long long)n * (c + 1)) / G);
-}
 
 // UG = H / 1024 units per lane per row (gate/up: 32 lanes x UG units x 32 inputs = H);
 // UD = I / 512 units per lane over a pair of down rows.
@@ -556,7 +485,7 @@ static unsigned* d1_counter_base(int dev) {
 
 static std::atomic<unsigned> g_d1_next_set{0};
 
-int decode1_reset_counters() {
+int decode1_reset_pool() {
   void* ptr = nullptr;
   cudaError_t err = cudaGetSymbolAddress(&ptr, g_d1_counters);
   if (err == cudaSuccess) err = cudaMemset(ptr, 0, sizeof(g_d1_counters));

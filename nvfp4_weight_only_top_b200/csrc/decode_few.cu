@@ -1,0 +1,498 @@
+// Decode of a few tokens (2 <= T <= 16, T k routed rows <= the SM count) as one persistent
+// kernel after the router: gate/up + SwiGLU -> down -> combine over one slot per routed row.
+//
+// The structure is the single-token kernel's (decode1.cu): a producer warp streams row blocks of
+// each slot's expert with 1-D bulk copies into a 4-stage ring; eight consumer warps dot them
+// against x (or h) held in registers; work is cut into contiguous shares so that a CTA's rows
+// belong to at most two slots, and a CTA waits only for the h of its own down slots.  Here the
+// slots are the routed rows in the router's permutation order (expert order: the slots of one
+// expert are neighbours, so its weight rows are read by neighbouring CTAs at about the same time
+// and the repeats come from L2), x is that of each slot's token, and the combine block of 32
+// outputs is per token.  Weight layout: page "Beam 1.0 501B-A23B, streaming pack, NVFP4 experts /
+// MLX 8-bit residents", section "What this pack holds"; SwiGLU in FP32: page
+// "Beam-1.0-501B-A23B VQ GGUF", section "What stays native".
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+#include "decode_fused.cuh"
+
+namespace moe {
+
+namespace {
+
+using namespace fused;
+
+constexpr int kNW = 8;                       // consumer warps
+constexpr int kThreads1 = 32 * (kNW + 1);    // + one producer warp
+constexpr int kRing = 4;                     // stages in the ring
+constexpr int kMaxK = 32;
+constexpr int kMaxT = 16;                    // tokens of one call
+constexpr int kMaxSlots = 160;               // routed rows (T k) of one call
+constexpr int kMaxBlocks = 256;              // H / 32 row blocks of the combine
+constexpr int kMaxLast = 264;                // down stages of one CTA (bound checked on the host)
+// Completion counters: per-slot counts, per (token, block) counts, one exit count.
+constexpr int kCounterWords = kMaxSlots + kMaxT * kMaxBlocks + 1;
+constexpr int kCounterSets = 64;             // calls that may be in flight at once per device
+
+// Counter sets owned by the library, one used per call in turn.  They start at zero (module
+// load) and each call leaves its set at zero again (the last CTA to finish clears it), so no
+// call needs a memset.
+__device__ unsigned g_dn_counters[kCounterSets][kCounterWords];
+
+struct DNParams {
+  const uint8_t* bank;
+  uint64_t stride;
+  uint64_t codes_off[3], scales_off[3], global_off[3];
+  int global_mode;
+  int E, k, T;
+
+  const uint16_t* x;     // [T, H] bf16
+  uint16_t* out;         // [T, H] bf16
+  uint16_t* x_next;      // [T, H] bf16 or null
+  float* h;              // [T k, I] f32 scratch, one row per slot
+  float* y;              // [T k, H] f32 scratch
+  unsigned* bar;         // [kCounterWords] completion counters: zero on entry, zero again on exit
+  const int32_t* ids;    // [T, k] the router's experts
+  const float* w;        // [T, k] the router's weights
+  const int32_t* perm;   // [T k] slot r is routed row perm[r] = t k + j (expert order)
+  const int32_t* inv;    // [T k] the slot of routed row t k + j
+};
+
+// UG = H / 1024 units per lane per row (gate/up: 32 lanes x UG units x 32 inputs = H);
+// UD = I / 512 units per lane over a pair of down rows.
+template <int UG, int UD>
+__global__ void __launch_bounds__(kThreads1, 1) decode_few_kernel(const DNParams p) {
+  constexpr int H = UG * 1024, I = UD * 512;
+  constexpr int kCodes1 = kNW * H / 2, kScales1 = kNW * H / 16;       // per matrix, 8 rows
+  constexpr int kStage1 = 2 * (kCodes1 + kScales1);
+  constexpr int kRows2 = 4 * kNW;                                     // down rows per stage
+  constexpr int kCodes2 = kRows2 * I / 2, kScales2 = kRows2 * I / 16;
+  constexpr int kStage2 = kCodes2 + kScales2;
+  constexpr int kStage = kStage1 > kStage2 ? kStage1 : kStage2;
+  constexpr int kUnits2 = I / 32;                                     // units per down row
+  static_assert((kRing * kStage + 2 * H * 2 + 2 * I * 4) % 16 == 0, "16-byte alignment of the tables");
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  // ring | x of up to two tokens (bf16 [2][H]) | h of up to two slots (f32 [2][I]) | barriers,
+  // slot tables
+  uint16_t* sx = reinterpret_cast<uint16_t*>(smem + kRing * kStage);
+  float* sh = reinterpret_cast<float*>(sx + 2 * H);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sh + 2 * I);
+  uint64_t* empty = full + kRing;
+  uint64_t* gm_full = empty + kRing;                        // the global multipliers are in s_gm
+  int* s_se = reinterpret_cast<int*>(gm_full + 1);          // [kMaxSlots] expert of slot r
+  int* s_st = s_se + kMaxSlots;                             // [kMaxSlots] token of slot r
+  float* s_gm = reinterpret_cast<float*>(s_st + kMaxSlots); // [3][kMaxSlots] global multipliers
+  int* s_ok = reinterpret_cast<int*>(s_gm + 3 * kMaxSlots);
+  int* s_last = s_ok + 1;                                   // [kMaxLast] (token, block)s to combine
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k = p.k, T = p.T, R = T * k;
+  const int n1 = R * (I / kNW), n2 = R * (H / kRows2);      // stages of each phase, whole grid
+  int lo1, hi1, lo2, hi2;
+  share(n1, blockIdx.x, gridDim.x, lo1, hi1);
+  share(n2, blockIdx.x, gridDim.x, lo2, hi2);
+  const int cnt1 = hi1 - lo1, cnt = cnt1 + (hi2 - lo2);     // this CTA's stages, both phases
+  unsigned* slot_done = p.bar;                              // [R]: gate/up stages completed
+  unsigned* block_done = p.bar + kMaxSlots;                 // [T][H/32]: down stages written
+  // Slots of this CTA's gate/up rows: ra .. rb (at most two: R <= number of CTAs).
+  const int ra = lo1 / (I / kNW), rb = hi1 > lo1 ? (hi1 - 1) / (I / kNW) : ra;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kNW);
+    }
+    mbar_init(gm_full, 1);
+    *s_ok = 1;
+    fence_barrier_init();
+  }
+  {
+    // Several tokens: the router kernel's output.  Slot r is routed row perm[r] (expert order,
+    // so the slots of one expert are neighbours and their weight rows are read close in time).
+    for (int r = threadIdx.x; r < R; r += blockDim.x) {
+      const int pr = __ldg(p.perm + r);
+      s_se[r] = __ldg(p.ids + pr);
+      s_st[r] = pr / k;
+    }
+    __syncthreads();
+    // x of the tokens of slots ra and rb, bank-spread as in the single-token case.
+    for (int i = threadIdx.x; i < 2 * (H / 8); i += blockDim.x) {
+      const int b = i / (H / 8), ii = i - b * (H / 8);
+      if (b == 1 && rb == ra) break;
+      const int u = ii >> 2, c = ii & 3;
+      reinterpret_cast<uint4*>(sx + b * H)[4 * u + (c ^ ((u >> 1) & 3))] =
+          __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)s_st[b ? rb : ra] * H) + ii);
+    }
+    __syncthreads();
+  }
+
+  if (warp == kNW) {
+    // ---------------------------------------------------------------- producer
+    const uint64_t pol = policy_evict_first();
+    auto issue = [&](int q) {                               // stage q into its ring slot
+      const int s = q % kRing;
+      uint8_t* dst = smem + s * kStage;
+      if (q < cnt1) {
+        const int u = lo1 + q, j = u / (I / kNW), r0 = (u - j * (I / kNW)) * kNW;
+        const uint8_t* rec = p.bank + (uint64_t)s_se[j] * p.stride;
+        mbar_arrive_expect_tx(&full[s], kStage1);
+        bulk_g2s(dst, rec + p.codes_off[0] + (uint64_t)r0 * (H / 2), kCodes1, &full[s], pol);
+        bulk_g2s(dst + kCodes1, rec + p.codes_off[1] + (uint64_t)r0 * (H / 2), kCodes1, &full[s], pol);
+        bulk_g2s(dst + 2 * kCodes1, rec + p.scales_off[0] + (uint64_t)r0 * (H / 16), kScales1, &full[s], pol);
+        bulk_g2s(dst + 2 * kCodes1 + kScales1, rec + p.scales_off[1] + (uint64_t)r0 * (H / 16), kScales1,
+                 &full[s], pol);
+      } else {
+        const int u = lo2 + (q - cnt1), j = u / (H / kRows2), r0 = (u - j * (H / kRows2)) * kRows2;
+        const uint8_t* rec = p.bank + (uint64_t)s_se[j] * p.stride;
+        mbar_arrive_expect_tx(&full[s], kStage2);
+        bulk_g2s(dst, rec + p.codes_off[2] + (uint64_t)r0 * (I / 2), kCodes2, &full[s], pol);
+        bulk_g2s(dst + kCodes2, rec + p.scales_off[2] + (uint64_t)r0 * (I / 16), kScales2, &full[s], pol);
+      }
+    };
+    const int first = cnt < kRing ? cnt : kRing;            // the ring starts empty
+    if (lane == 0)
+      for (int q = 0; q < first; ++q) issue(q);
+    // With those in flight, the global multipliers of the slots.
+    for (int r = lane; r < R; r += 32) {
+      const uint8_t* rec = p.bank + (uint64_t)s_se[r] * p.stride;
+      float g[3];
+#pragma unroll
+      for (int m = 0; m < 3; ++m) g[m] = __ldg(reinterpret_cast<const float*>(rec + p.global_off[m]));
+#pragma unroll
+      for (int m = 0; m < 3; ++m) s_gm[m * kMaxSlots + r] = global_mult(g[m], p.global_mode);
+    }
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(gm_full);
+      int q = first;
+      for (; q < cnt; ++q) {
+        if (!mbar_wait(&empty[q % kRing], ((q / kRing) & 1) ^ 1)) break;
+        issue(q);
+      }
+      // Leave no copy in flight (only an error path gets here with copies outstanding).
+      for (int i = q - kRing > 0 ? q - kRing : 0; i < q; ++i) mbar_wait(&full[i % kRing], (i / kRing) & 1);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- consumers
+    const uint32_t sbase = smem_addr(smem);
+    bool ok = true;
+    // Phase 1: gate/up.  Warp w takes row r0 + w of both matrices; lane l its units
+    // l + 32 u (u < UG) of the row, with x at those K positions held in registers.
+    uint32_t xr[UG][16];
+    int q = 0;
+    bool have_gm = false;
+    // The gate/up rows of this CTA lie in slot ra, then (from stage q_split on) in slot rb; x of
+    // each slot's token is loaded into registers once, outside the stage loop.
+    const int q_split = rb == ra ? cnt1 : (ra + 1) * (I / kNW) - lo1;
+    for (int seg = 0; seg < 2 && ok; ++seg) {
+      if (seg == 1 && rb == ra && q > 0) {
+        // same token: xr stays
+      } else {
+        const uint16_t* xs = sx + (seg == 1 ? H : 0);
+#pragma unroll
+        for (int u = 0; u < UG; ++u) {
+          const int un = lane + 32 * u;
+          const uint4* xp = reinterpret_cast<const uint4*>(xs) + 4 * un;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 b = xp[c ^ ((un >> 1) & 3)];
+            xr[u][4 * c + 0] = pack_f16x2(bf16_bits_to_f32(b.x & 0xFFFF), bf16_bits_to_f32(b.x >> 16));
+            xr[u][4 * c + 1] = pack_f16x2(bf16_bits_to_f32(b.y & 0xFFFF), bf16_bits_to_f32(b.y >> 16));
+            xr[u][4 * c + 2] = pack_f16x2(bf16_bits_to_f32(b.z & 0xFFFF), bf16_bits_to_f32(b.z >> 16));
+            xr[u][4 * c + 3] = pack_f16x2(bf16_bits_to_f32(b.w & 0xFFFF), bf16_bits_to_f32(b.w >> 16));
+          }
+        }
+      }
+    const int q_end = seg == 0 ? q_split : cnt1;
+    for (; q < q_end && ok; ++q) {
+      const int s = q % kRing;
+      const int u0 = lo1 + q, j = u0 / (I / kNW), r = (u0 - j * (I / kNW)) * kNW + warp;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (q / kRing) & 1))) {
+        ok = false;
+        break;
+      }
+      const uint32_t st = sbase + s * kStage;
+      const uint32_t cg = st + warp * (H / 2), cu = st + kCodes1 + warp * (H / 2);
+      const uint32_t sg = st + 2 * kCodes1 + warp * (H / 16), su = sg + kScales1;
+      float accG = 0.0f, accU = 0.0f;
+#pragma unroll
+      for (int u = 0; u < UG; ++u) {
+        const int un = lane + 32 * u;
+        accG += unit_dot(lds128(cg + un * 16), lds16(sg + un * 2), xr[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < UG; ++u) {
+        const int un = lane + 32 * u;
+        accU += unit_dot(lds128(cu + un * 16), lds16(su + un * 2), xr[u]);
+      }
+      fence_proxy_async_smem();            // the reads above come before the slot's next TMA
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        accG += __shfl_xor_sync(0xFFFFFFFFu, accG, off);
+        accU += __shfl_xor_sync(0xFFFFFFFFu, accU, off);
+      }
+      if (!have_gm) {
+        have_gm = true;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(gm_full, 0))) {
+          ok = false;
+          break;
+        }
+      }
+      if (lane == 0) p.h[(size_t)j * I + r] = silu_mul(accG * s_gm[j], accU * s_gm[kMaxSlots + j]);
+    }
+    }
+    // Publish this CTA's gate/up stages per slot, then wait for the slots of its down rows.
+    named_bar_sync(1, 32 * kNW);
+    if (threadIdx.x == 0) {
+      __threadfence();
+      for (int u = lo1; u < hi1;) {
+        const int j = u / (I / kNW), uend = min(hi1, (j + 1) * (I / kNW));
+        atomicAdd(&slot_done[j], (unsigned)(uend - u));
+        u = uend;
+      }
+      bool good = ok;
+      if (hi2 > lo2)
+        for (int j = lo2 / (H / kRows2); good && j <= (hi2 - 1) / (H / kRows2); ++j)
+          good = wait_count(&slot_done[j], I / kNW);
+      *s_ok = good ? 1 : 0;
+    }
+    named_bar_sync(1, 32 * kNW);
+    ok = ok && *s_ok;
+    // h of the (at most two) slots of this CTA's down rows into shared memory, once per CTA
+    // rather than once per warp: every CTA reads the same few KB, so per-warp loads would
+    // pile onto the same L2 lines.
+    const int jlo = lo2 / (H / kRows2);
+    if (ok && hi2 > lo2) {
+      // All of a thread's loads are issued before any store, so their latencies overlap.
+      constexpr int kPer = (2 * I / 4 + 32 * kNW - 1) / (32 * kNW);
+      const int n4 = ((hi2 - 1) / (H / kRows2) - jlo + 1) * I / 4;
+      const float4* src = reinterpret_cast<const float4*>(p.h + (size_t)jlo * I);
+      float4 v[kPer];
+#pragma unroll
+      for (int t = 0; t < kPer; ++t) {
+        const int i = (int)threadIdx.x + t * 32 * kNW;
+        if (i < n4) v[t] = __ldcg(src + i);
+      }
+      // Chunk c of unit u (32 floats) of a slot is stored at chunk c ^ (u & 7) of the unit
+      // (bank spread for the per-lane reads below).
+#pragma unroll
+      for (int t = 0; t < kPer; ++t) {
+        const int i = (int)threadIdx.x + t * 32 * kNW;
+        if (i < n4) {
+          const int sl = i / (I / 4), w = i - sl * (I / 4), u = w >> 3, c = w & 7;
+          reinterpret_cast<float4*>(sh)[sl * (I / 4) + 8 * u + (c ^ (u & 7))] = v[t];
+        }
+      }
+    }
+    named_bar_sync(1, 32 * kNW);
+
+    // Phase 2: down.  Warp w takes rows 4w .. 4w+3 of the stage as two pairs; in a pair, lane l
+    // takes units cu = l + 32 u (u < UD) of the two rows laid end to end: row cu / kUnits2, K
+    // unit cu % kUnits2, with h at those K positions in registers (reloaded when the slot
+    // changes).
+    uint32_t hr[UD][16];
+    int hj = -1;
+    for (; q < cnt && ok; ++q) {
+      const int s = q % kRing;
+      const int u0 = lo2 + (q - cnt1), j = u0 / (H / kRows2), r0 = (u0 - j * (H / kRows2)) * kRows2 + 4 * warp;
+      if (!have_gm) {
+        have_gm = true;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(gm_full, 0))) {
+          ok = false;
+          break;
+        }
+      }
+      if (j != hj) {
+        hj = j;
+        const float* hp = sh + (size_t)(j - jlo) * I;
+#pragma unroll
+        for (int u = 0; u < UD; ++u) {
+          const int ku = (lane + 32 * u) % kUnits2;
+          const float4* src = reinterpret_cast<const float4*>(hp + 32 * ku);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 a = src[q4 ^ (ku & 7)];
+            hr[u][2 * q4] = pack_f16x2(a.x, a.y);
+            hr[u][2 * q4 + 1] = pack_f16x2(a.z, a.w);
+          }
+        }
+      }
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (q / kRing) & 1))) {
+        ok = false;
+        break;
+      }
+      const uint32_t st = sbase + s * kStage;
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) {
+        const uint32_t cd = st + (4 * warp + 2 * pr) * (I / 2), sd = st + kCodes2 + (4 * warp + 2 * pr) * (I / 16);
+#pragma unroll
+        for (int u = 0; u < UD; ++u) {
+          const int cu = lane + 32 * u;                     // unit within the pair of rows
+          const float part = unit_dot(lds128(cd + cu * 16), lds16(sd + cu * 2), hr[u]);
+          if (cu < kUnits2)
+            acc[2 * pr] += part;
+          else
+            acc[2 * pr + 1] += part;
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] += __shfl_xor_sync(0xFFFFFFFFu, acc[i], off);
+      if (lane < 4) {
+        const float v = lane == 0 ? acc[0] : lane == 1 ? acc[1] : lane == 2 ? acc[2] : acc[3];
+        p.y[(size_t)j * H + r0 + lane] = v * s_gm[2 * kMaxSlots + j];
+      }
+    }
+    // Combine.  Block (t, b) = rows 32b .. 32b+31 of token t: one down stage for each of the
+    // token's k slots, so k contributions.  Each CTA publishes its stages (one fence, one
+    // atomic per stage) and combines the blocks for which it added the last contribution.
+    named_bar_sync(1, 32 * kNW);
+    if (threadIdx.x == 0) {
+      int n = 0;
+      if (ok) {
+        __threadfence();
+        for (int u = lo2; u < hi2; ++u) {
+          const int r = u / (H / kRows2), b = u - r * (H / kRows2);
+          const int tb = s_st[r] * (H / 32) + b;
+          if (atomicAdd(&block_done[tb], 1u) == (unsigned)k - 1u) s_last[n++] = tb;
+        }
+        if (n) __threadfence();
+      }
+      *s_ok = n;
+    }
+    named_bar_sync(1, 32 * kNW);
+    // The last CTA through here clears the counter set for the call that uses it next.
+    if (threadIdx.x == 0) {
+      unsigned* exit_count = p.bar + kMaxSlots + kMaxT * kMaxBlocks;
+      __threadfence();
+      if (atomicAdd(exit_count, 1u) == gridDim.x - 1) {
+        __threadfence();                    // every other CTA's counter updates come before
+        for (int i = 0; i < R; ++i) slot_done[i] = 0;
+        for (int i = 0; i < T * (H / 32); ++i) block_done[i] = 0;
+        *exit_count = 0;
+        __threadfence();
+      }
+    }
+    for (int i = warp; i < *s_ok; i += kNW) {
+      const int t = s_last[i] / (H / 32), c = 32 * (s_last[i] - t * (H / 32)) + lane;
+      float a = 0.0f;
+      for (int jj = 0; jj < k; ++jj)
+        a = fmaf(__ldg(p.w + t * k + jj), __ldcg(p.y + (size_t)__ldg(p.inv + t * k + jj) * H + c), a);
+      const uint32_t o = f32_to_bf16_bits(a);
+      p.out[(size_t)t * H + c] = (uint16_t)o;
+      if (p.x_next != nullptr)
+        p.x_next[(size_t)t * H + c] =
+            (uint16_t)f32_to_bf16_bits(bf16_bits_to_f32(__ldg(p.x + (size_t)t * H + c)) + bf16_bits_to_f32(o));
+    }
+  }
+}
+
+template <int UG, int UD>
+int launch_dn(const DNParams& p, int num_sms, cudaStream_t s) {
+  constexpr int H = UG * 1024, I = UD * 512;
+  constexpr int kStage1 = 2 * (kNW * H / 2 + kNW * H / 16);
+  constexpr int kStage2 = 4 * kNW * I / 2 + 4 * kNW * I / 16;
+  constexpr int kStage = kStage1 > kStage2 ? kStage1 : kStage2;
+  const int smem = kRing * kStage + 2 * H * 2 + 2 * I * 4 + (2 * kRing + 1) * 8 + 5 * kMaxSlots * 4 + 4 + 4 * kMaxLast;
+  auto kern = decode_few_kernel<UG, UD>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return -(int)err;
+  // Cooperative launch: all CTAs are resident at once, which the grid barriers need.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms);
+  cfg.blockDim = dim3(kThreads1);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, kern, p);
+  return err == cudaSuccess ? 1 : -(int)err;
+}
+
+}  // namespace
+
+bool decode_few_supported(int H, int I, int k, int T, int num_sms) {
+  const int R = T * k;
+  // A CTA's rows must span at most two slots (R <= number of CTAs); the counter sets bound T,
+  // R and H / 32.
+  if (T < 2 || T > kMaxT || k > kMaxK || R > kMaxSlots || R > num_sms || H / 32 > kMaxBlocks ||
+      (R * (H / 32) + num_sms - 1) / num_sms > kMaxLast)
+    return false;
+  return (H == 5120 && I == 2560) || (H == 1024 && I == 512) || (H == 2048 && I == 1024) ||
+         (H == 4096 && I == 1536);
+}
+
+// Device address of this device's counter sets (the current device), resolved once.
+static unsigned* dn_counter_base(int dev) {
+  static std::mutex mu;
+  static std::vector<unsigned*> base;
+  std::lock_guard<std::mutex> lk(mu);
+  if ((int)base.size() <= dev) base.resize(dev + 1, nullptr);
+  if (!base[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_dn_counters) != cudaSuccess) return nullptr;
+    base[dev] = static_cast<unsigned*>(ptr);
+  }
+  return base[dev];
+}
+
+static std::atomic<unsigned> g_dn_next_set{0};
+
+int decode_few_reset_pool() {
+  void* ptr = nullptr;
+  cudaError_t err = cudaGetSymbolAddress(&ptr, g_dn_counters);
+  if (err == cudaSuccess) err = cudaMemset(ptr, 0, sizeof(g_dn_counters));
+  return err == cudaSuccess ? 0 : -(int)err;
+}
+
+int launch_decode_few(const BankView& bank, int T, int k, const uint16_t* x, uint16_t* out, uint16_t* x_next,
+                      float* h, float* y, const int32_t* ids, const float* w, const int32_t* perm,
+                      const int32_t* inv, int dev, int num_sms, cudaStream_t s) {
+  unsigned* sets = dn_counter_base(dev);
+  if (!sets) return -(int)cudaErrorInvalidSymbol;
+  unsigned* bar = sets + (size_t)(g_dn_next_set.fetch_add(1u) % kCounterSets) * kCounterWords;
+  DNParams p{};
+  p.bank = bank.base;
+  p.stride = bank.stride;
+  for (int m = 0; m < 3; ++m) {
+    p.codes_off[m] = bank.codes_off[m];
+    p.scales_off[m] = bank.scales_off[m];
+    p.global_off[m] = bank.global_off[m];
+  }
+  p.global_mode = bank.global_mode;
+  p.E = bank.E;
+  p.k = k;
+  p.T = T;
+  p.x = x;
+  p.out = out;
+  p.x_next = x_next;
+  p.h = h;
+  p.y = y;
+  p.bar = bar;
+  p.ids = ids;
+  p.w = w;
+  p.perm = perm;
+  p.inv = inv;
+  if (bank.H == 5120 && bank.I == 2560) return launch_dn<5, 5>(p, num_sms, s);
+  if (bank.H == 1024 && bank.I == 512) return launch_dn<1, 1>(p, num_sms, s);
+  if (bank.H == 2048 && bank.I == 1024) return launch_dn<2, 2>(p, num_sms, s);
+  if (bank.H == 4096 && bank.I == 1536) return launch_dn<4, 3>(p, num_sms, s);
+  return -(int)cudaErrorInvalidValue;
+}
+
+}  // namespace moe

@@ -74,9 +74,16 @@ bool decode1_supported(int H, int I, int k, int E, int num_sms);
 int launch_decode1(const BankView& bank, const float* logits, int k, const uint16_t* x, uint16_t* out,
                    uint16_t* x_next, float* h, float* y, int32_t* ids, float* w, int dev, int num_sms,
                    cudaStream_t s);
-// Clears every counter set of the current device (after a kernel gave up on a bounded wait, a
-// set may be left non-zero).  Synchronous.
-int decode1_reset_counters();
+int decode1_reset_pool();
+
+// Decode of 2 .. 16 tokens (T k <= number of SMs) in one persistent kernel after the router:
+// gate/up, down and combine over one slot per routed row, in the router's permutation order.
+// h [T k, I] and y [T k, H] are f32 scratch; counters as for the single-token kernel.
+bool decode_few_supported(int H, int I, int k, int T, int num_sms);
+int launch_decode_few(const BankView& bank, int T, int k, const uint16_t* x, uint16_t* out, uint16_t* x_next,
+                      float* h, float* y, const int32_t* ids, const float* w, const int32_t* perm,
+                      const int32_t* inv, int dev, int num_sms, cudaStream_t s);
+int decode_few_reset_pool();
 
 // Prefill path: grouped NVFP4 GEMM on tcgen05 tensor cores, groups of up to kPrefillRows rows.
 constexpr int kPrefillRows = 256;

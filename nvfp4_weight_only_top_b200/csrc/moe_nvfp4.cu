@@ -381,6 +381,22 @@ int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
     t_last_launches = launches;
     return MOE_NVFP4_OK;
   }
+  if (moe::decode_few_supported(H, I, k, (int)T, info.sms)) {
+    // A few tokens: the router, then one persistent kernel over one slot per routed row in the
+    // router's permutation order (expert order).
+    prof_before(MOE_NVFP4_KERNEL_ROUTE, s);
+    if ((rc = after_launch(moe::launch_route(logits, T, E, k, rb, s), s, "route", &launches))) return rc;
+    prof_before(MOE_NVFP4_KERNEL_DECODE_FUSED, s);
+    if ((rc = after_launch(moe::launch_decode_few(bv, (int)T, k, static_cast<const uint16_t*>(x),
+                                                  static_cast<uint16_t*>(out), static_cast<uint16_t*>(x_next),
+                                                  reinterpret_cast<float*>(w8 + L.h),
+                                                  reinterpret_cast<float*>(w8 + L.y), rb.ids, rb.w, rb.perm, rb.inv,
+                                                  dev, info.sms, s),
+                           s, "fused few-token decode", &launches)))
+      return rc;
+    t_last_launches = launches;
+    return MOE_NVFP4_OK;
+  }
   // One-row groups take the CUDA-core row kernels when both widths allow; groups of two or
   // more rows (none when T == 1) take the mma.sync kernels.
   const bool rows = moe::rows_supported(H, true) && moe::rows_supported(I, false);
@@ -551,7 +567,8 @@ int moe_nvfp4_device_status(void) {
   if (e != cudaSuccess) return cuda_fail(e, "clear device status");
   if (v != 0) {
     // A kernel that gave up may have left its completion counters set: clear them all.
-    const int rc = moe::decode1_reset_counters();
+    int rc = moe::decode1_reset_pool();
+    if (rc == 0) rc = moe::decode_few_reset_pool();
     if (rc < 0) return cuda_fail((cudaError_t)(-rc), "clear decode counters");
     return fail(MOE_NVFP4_ERR_TIMEOUT, "a bounded device wait gave up (status %d)", v);
   }
