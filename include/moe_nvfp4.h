@@ -51,10 +51,22 @@ extern "C" {
                                            during stream capture                             */
 #define MOE_NVFP4_ERR_TIMEOUT     (-5)  /* a bounded device-side wait gave up (device status) */
 
-/* Expert-GEMM path selection for moe_nvfp4_forward_ex. */
+/*
+ * Expert-GEMM path selection for moe_nvfp4_forward_ex.
+ * DECODE (memory-bound, CUDA cores):
+ *   T = 1, H x I in {5120x2560, 4096x1536, 2048x1024, 1024x512}, E <= 256: the whole layer in
+ *     one persistent kernel (routing, gate/up, down and combine; one launch);
+ *   2 <= T <= 16 with T k <= the SM count, same shapes: the router kernel, then one persistent
+ *     kernel over the routed rows (two launches);
+ *   otherwise: router kernel(s), grouped GEMV/GEMM kernels, combine.
+ *   The persistent kernels take completion counters from 64 library-owned counter sets per
+ *   device and kernel, one per call in turn: at most 64 such calls may be in flight at once on
+ *   one device.
+ * PREFILL (tcgen05 tensor cores, BF16 x BF16 -> F32): H and I multiples of 256.
+ */
 #define MOE_NVFP4_PATH_AUTO    0
-#define MOE_NVFP4_PATH_DECODE  1   /* memory-bound grouped GEMV/GEMM, any number of tokens */
-#define MOE_NVFP4_PATH_PREFILL 2   /* tensor-core (tcgen05) grouped GEMM                     */
+#define MOE_NVFP4_PATH_DECODE  1   /* memory-bound kernels, any number of tokens */
+#define MOE_NVFP4_PATH_PREFILL 2   /* tensor-core (tcgen05) grouped GEMM          */
 
 /*
  * Expert bank: E records in device memory, record e at base + e * record_stride.
@@ -164,7 +176,8 @@ const char* moe_nvfp4_last_error(void);
 /*
  * Reads and clears the current device's sticky kernel status (synchronises the device):
  * MOE_NVFP4_OK, or MOE_NVFP4_ERR_TIMEOUT if a bounded wait inside a kernel gave up since the
- * last call.  A timeout means the kernel returned early and its outputs are invalid.
+ * last call.  A timeout means the kernel returned early and its outputs are invalid; the
+ * persistent decode kernels' counter sets are then cleared so that later calls start clean.
  */
 int moe_nvfp4_device_status(void);
 
