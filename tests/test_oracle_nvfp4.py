@@ -4,7 +4,6 @@ The decoders are checked against library decodings (ml_dtypes, torch), the recor
 against the numbers the streaming-pack page prints, and the index conventions against a
 test-side encoder that writes known matrices in the stated layout.
 """
-import math
 
 import ml_dtypes
 import numpy as np
@@ -103,12 +102,18 @@ def test_single_nibble_lands_in_its_column():
 
 
 def test_global_mode_1_is_f32_division():
-    for g in [np.float32(2688.0), np.float32(1.0), np.float32(0.0023292375 * 2688)]:
+    from fractions import Fraction
+    for g in [np.float32(2688.0), np.float32(1.0), np.float32(0.0023292375 * 2688), np.float32(7.0),
+              np.float32(1e-3), np.float32(3.0e4)]:
         m = oracle.global_multiplier(g, 1)
-        exact = float(g) / 2688.0
-        # correctly rounded f32 of the quotient
-        assert m == float(np.float32(exact)) or abs(m - exact) <= 0.5 * math.ulp(np.float32(exact))
+        exact = Fraction(float(g)) / 2688
+        # an f32 value, and the correctly rounded one: no other f32 lies closer to g / 2688
+        assert float(np.float32(m)) == m
+        lo, hi = np.nextafter(np.float32(m), np.float32(-np.inf)), np.nextafter(np.float32(m), np.float32(np.inf))
+        d = abs(Fraction(m) - exact)
+        assert d <= abs(Fraction(float(lo)) - exact) and d <= abs(Fraction(float(hi)) - exact)
     assert oracle.global_multiplier(np.float32(2688.0), 1) == 1.0
+    assert oracle.global_multiplier(np.float32(0.75), 0) == 0.75
 
 
 def test_read_record_uses_descriptor_offsets():
@@ -159,3 +164,41 @@ def test_read_record_part_roles():
     assert Wg.shape == (I, H) and np.all(Wg == 1.0 * 1.0 * 0.5)
     assert Wu.shape == (I, H) and np.all(Wu == 2.0 * 2.0 * 1.0)
     assert Wd.shape == (H, I) and np.all(Wd == 4.0 * 4.0 * 1.5)
+
+
+def test_decode_codes_inverts_the_writer():
+    rng = np.random.default_rng(17)
+    codes = rng.integers(0, 16, (5, 48))
+    words, _ = _encode(codes, np.zeros((5, 3)))
+    assert np.array_equal(oracle.decode_codes(words, 48), codes)
+
+
+@pytest.mark.parametrize("part", [0, 1, 2])
+def test_read_record_index_layout_of_each_part(part):
+    """Per projection of a hand-built record: one nonzero code lands at its (out, in) position,
+    and one distinct block scale covers exactly its 16 inputs of its row (gate and up are
+    [I, H], down is [H, I])."""
+    H, I = 64, 32
+    lay = moe_inputs.record_layout(1, H, I)
+    O, K = [(I, H), (I, H), (H, I)][part]
+    rng = np.random.default_rng(23 + part)
+    for o, i in [(0, 0), (O - 1, K - 1), (1, K - 9), (O - 2, 17)] + [tuple(v) for v in rng.integers(0, [O, K], (4, 2))]:
+        rec = np.zeros(lay.record_bytes, dtype=np.uint8)
+        for p in range(3):
+            rec[lay.scales_off[p]:lay.scales_off[p] + O * K // 16] = 0x38          # 1.0
+            rec[lay.global_off[p]:lay.global_off[p] + 4] = np.array([1.0], '<f4').view(np.uint8)
+        byte = lay.codes_off[part] + (o * K + i) // 2
+        rec[byte] = 0x2 << (4 * (i % 2))                                          # code 2 = 1.0
+        W = oracle.read_record(rec, H, I, lay.codes_off, lay.scales_off, lay.global_off)
+        assert np.argwhere(W[part] != 0).tolist() == [[o, i]] and W[part][o, i] == 1.0
+        assert all(not np.any(W[q]) for q in range(3) if q != part)
+    for o, b in [(0, 0), (O - 1, K // 16 - 1), (O // 2, 1)]:
+        rec = np.zeros(lay.record_bytes, dtype=np.uint8)
+        rec[lay.codes_off[part]:lay.codes_off[part] + O * K // 2] = 0x22              # all 1.0
+        rec[lay.scales_off[part]:lay.scales_off[part] + O * K // 16] = 0x38
+        rec[lay.scales_off[part] + o * (K // 16) + b] = 0x40                         # 2.0
+        rec[lay.global_off[part]:lay.global_off[part] + 4] = np.array([1.0], '<f4').view(np.uint8)
+        W = oracle.read_record(rec, H, I, lay.codes_off, lay.scales_off, lay.global_off)[part]
+        want = np.ones((O, K))
+        want[o, 16 * b:16 * b + 16] = 2.0
+        assert np.array_equal(W, want)
