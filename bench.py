@@ -70,9 +70,10 @@ def kernel_traffic(kind: str, workload: str):
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    src = os.path.join(ROOT, "nvfp4_weight_only_top_b200", "csrc", d["source"])
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    return d["dram_bytes_per_launch"] if h == d["source_sha256"] else None
+    h = hashlib.sha256()
+    for name in d.get("sources", [d.get("source")]):     # every file the kernel is built from
+        h.update(open(os.path.join(ROOT, "nvfp4_weight_only_top_b200", "csrc", name), "rb").read())
+    return d["dram_bytes_per_launch"] if h.hexdigest() == d["source_sha256"] else None
 
 
 class ClockSampler:

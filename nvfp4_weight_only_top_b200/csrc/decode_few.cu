@@ -223,12 +223,12 @@ __global__ void __launch_bounds__(kThreads1, 1) decode_few_kernel(const DNParams
 #pragma unroll
       for (int u = 0; u < UG; ++u) {
         const int un = lane + 32 * u;
-        accG += unit_dot(lds128(cg + un * 16), lds16(sg + un * 2), xr[u]);
+        unit_dot_acc(lds128(cg + un * 16), lds16(sg + un * 2), xr[u], accG);
       }
 #pragma unroll
       for (int u = 0; u < UG; ++u) {
         const int un = lane + 32 * u;
-        accU += unit_dot(lds128(cu + un * 16), lds16(su + un * 2), xr[u]);
+        unit_dot_acc(lds128(cu + un * 16), lds16(su + un * 2), xr[u], accU);
       }
       fence_proxy_async_smem();            // the reads above come before the slot's next TMA
       __syncwarp();
@@ -336,11 +336,19 @@ __global__ void __launch_bounds__(kThreads1, 1) decode_few_kernel(const DNParams
 #pragma unroll
         for (int u = 0; u < UD; ++u) {
           const int cu = lane + 32 * u;                     // unit within the pair of rows
-          const float part = unit_dot(lds128(cd + cu * 16), lds16(sd + cu * 2), hr[u]);
-          if (cu < kUnits2)
-            acc[2 * pr] += part;
-          else
-            acc[2 * pr + 1] += part;
+          const uint4 cw = lds128(cd + cu * 16);
+          const uint32_t sw = lds16(sd + cu * 2);
+          if (32 * u + 31 < kUnits2) {                      // every lane in the first row
+            unit_dot_acc(cw, sw, hr[u], acc[2 * pr]);
+          } else if (32 * u >= kUnits2) {                   // every lane in the second row
+            unit_dot_acc(cw, sw, hr[u], acc[2 * pr + 1]);
+          } else {
+            const float part = unit_dot(cw, sw, hr[u]);
+            if (cu < kUnits2)
+              acc[2 * pr] += part;
+            else
+              acc[2 * pr + 1] += part;
+          }
         }
       }
       fence_proxy_async_smem();
