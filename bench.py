@@ -151,6 +151,14 @@ def max_over_ranks(ws, v: float) -> float:
     return float(t.item())
 
 
+def replay_stats(replay_ms: list, steps_per_replay: int) -> dict:
+    """Median, best and worst time per step (ms) over the timed graph replays."""
+    per = sorted(t / steps_per_replay for t in replay_ms)
+    n = len(per)
+    med = per[n // 2] if n % 2 else 0.5 * (per[n // 2 - 1] + per[n // 2])
+    return {"median": med, "best": per[0], "worst": per[-1]}
+
+
 def cpu_oracle_baseline(cfg, budget_s: float = 20.0, max_tokens: int = 64):
     """Times the FP64 oracle (as it stands) on one host core over a bounded token sample."""
     from threadpoolctl import threadpool_limits
@@ -280,15 +288,17 @@ def main():
     clocks = ClockSampler(local, enabled=(rank == 0 and not args.no_clocks))
     barrier(ws)
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s)
-    for _ in range(reps):
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]   # one between replays
+    evs[0].record(s)
+    for r in range(reps):
         graph.replay()
-    e1.record(s)
+        evs[r + 1].record(s)
     torch.cuda.synchronize()
     barrier(ws)
     ck = clocks.stop()
-    ms = max_over_ranks(ws, e0.elapsed_time(e1))
+    ms = max_over_ranks(ws, evs[0].elapsed_time(evs[-1]))
+    spread = replay_stats([evs[r].elapsed_time(evs[r + 1]) for r in range(reps)], gsteps)
+    spread = {key: max_over_ranks(ws, v) for key, v in spread.items()}
     ms_step = ms / steps_eff
     tokens = cfg.T * steps_eff * ws
     value = tokens / (ms / 1000.0)
@@ -378,7 +388,9 @@ def main():
     expert_bytes = avg_touched * (2 * proj_bytes(cfg.I, cfg.H) + proj_bytes(cfg.H, cfg.I)) * per_step_layers
     line = {
         "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": ws, "steps": steps_eff, "warmup": warm,
-        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "ms_per_step": ms_step,
+        "ms_per_step_spread": dict(spread, replays=reps, steps_per_replay=gsteps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if cfg.T * cfg.k > 8 * cfg.E else "f16", "data": "synthetic",
         "config": dict(workload_config(cfg), l2="inputs larger than L2: each step reads %.0f MB of expert "
                        "records%s" % (expert_bytes / 1e6, " from experts not used in the previous %d steps"

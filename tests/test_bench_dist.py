@@ -29,7 +29,9 @@ def _rank_main(rank, ws, port, q):
     bench.barrier(w)
     ms = bench.max_over_ranks(w, 10.0 + 5.0 * r)         # each rank's own device time
     tokens = 3 * 7 * w                                     # T x steps x ranks: the whole job
-    q.put((r, w, ms, tokens / (ms / 1000.0)))
+    spread = bench.replay_stats([8.0 + 4.0 * r, 4.0, 6.0], 2)   # per-replay times of this rank
+    spread = {key: bench.max_over_ranks(w, v) for key, v in spread.items()}
+    q.put((r, w, ms, tokens / (ms / 1000.0), spread))
     dist.destroy_process_group()
 
 
@@ -44,9 +46,16 @@ def test_max_over_ranks_and_whole_job_value_gloo():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for r, w, ms, value in got:
+    for r, w, ms, value, spread in got:
         assert w == 2 and ms == 15.0                       # the slowest rank sets the time
         assert value == pytest.approx(42 / 0.015)          # all ranks' tokens over that time
+        assert spread == {"median": 3.0, "best": 2.0, "worst": 6.0}   # per step, max over ranks
+
+
+def test_replay_stats_per_step():
+    import bench
+    assert bench.replay_stats([6.4], 64) == {"median": 0.1, "best": 0.1, "worst": 0.1}
+    assert bench.replay_stats([3.0, 1.0, 2.0, 4.0], 1) == {"median": 2.5, "best": 1.0, "worst": 4.0}
 
 
 def _bench(args, env_extra):
