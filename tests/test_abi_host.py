@@ -93,3 +93,35 @@ def test_workspace_bytes_is_host_only():
 def test_input_generator_key_matches_native():
     for args in [(0, 0, 0, 0), (7, 3, 255, 1), (123456789, 23, 17, 0)]:
         assert mdev.stream_key_native(*args) == moe_inputs.gen.stream_key(*args)
+
+
+def _fwd_ex(bank, T=4, k=2, path=_abi.PATH_AUTO):
+    lib = moe.lib()
+    return lib.moe_nvfp4_forward_ex(ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000), T, ctypes.byref(bank), k,
+                                    ctypes.c_void_p(0x40000), None, None, 0, path, None)
+
+
+def test_unknown_path_and_oversized_T_are_rejected_on_the_host():
+    assert _fwd_ex(_bank(), path=3) == _abi.ERR_INVALID_ARG
+    assert _fwd_ex(_bank(), path=-1) == _abi.ERR_INVALID_ARG
+    assert "path" in moe.moe_nvfp4_last_error()
+    assert _fwd_ex(_bank(), T=1 << 40) == _abi.ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("part", [0, 1, 2])
+def test_projection_offsets_are_validated(part):
+    lay = moe_inputs.record_layout(16, 256, 128)
+    for field, bad in (("codes_off", 8), ("scales_off", 4), ("global_off", 2)):
+        offs = list(getattr(lay, field))
+        offs[part] += bad
+        assert _fwd(_bank(**{field: offs})) == _abi.ERR_INVALID_ARG, (field, part)
+    offs = list(lay.codes_off)
+    offs[part] = lay.record_stride                    # starts past the end of the record
+    assert _fwd(_bank(codes_off=offs)) == _abi.ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the behaviour without a CUDA device")
+def test_valid_call_without_a_device_fails_loudly():
+    """No CPU fallback: with every argument valid and no CUDA device, the call returns an error."""
+    assert _fwd(_bank()) == _abi.ERR_UNSUPPORTED
+    assert "no CUDA device" in moe.moe_nvfp4_last_error()
