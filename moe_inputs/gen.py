@@ -226,7 +226,8 @@ def sample_tokens(T: int, n: int = 512, seed: int = 0) -> np.ndarray:
 
 def disjoint_routing_logits(E: int, k: int, sets: int, window: int, seed: int = 0) -> np.ndarray:
     """[sets, 1, E] f32 logits for one token each, such that the k largest logits of set s
-    name k experts that none of the previous window-1 sets names.
+    name k experts that none of the previous window-1 sets names, counting cyclically (the
+    sets are used in a loop, so the last sets also avoid the experts of the first ones).
 
     Each row holds the same multiset as an N(0,1) draw of E values: the k largest values of
     the draw are given to k experts chosen uniformly among those not used in the window,
@@ -239,6 +240,8 @@ def disjoint_routing_logits(E: int, k: int, sets: int, window: int, seed: int = 
     for s in range(sets):
         banned = set()
         for r in recent[-(window - 1):] if window > 1 else []:
+            banned |= r
+        for r in recent[:max(0, s + window - sets)]:      # sets 0 .. s+window-1-sets follow s cyclically
             banned |= r
         free = np.array([e for e in range(E) if e not in banned])
         chosen = rng.choice(free, k, replace=False)
