@@ -241,8 +241,11 @@ def disjoint_routing_logits(E: int, k: int, sets: int, window: int, seed: int = 
         banned = set()
         for r in recent[-(window - 1):] if window > 1 else []:
             banned |= r
+        wrap = set()
         for r in recent[:max(0, s + window - sets)]:      # sets 0 .. s+window-1-sets follow s cyclically
-            banned |= r
+            wrap |= r
+        if E - len(banned | wrap) >= k:                   # (too few experts left: window only)
+            banned |= wrap
         free = np.array([e for e in range(E) if e not in banned])
         chosen = rng.choice(free, k, replace=False)
         vals = np.sort(rng.standard_normal(E).astype(np.float32))[::-1]
