@@ -322,16 +322,18 @@ def main():
         lgh = [torch.from_numpy(lg_np[i]).pin_memory() for i in range(nsets)]
         oh = torch.empty_like(xh).pin_memory()
         n_e2e = min(steps_eff, 2000 if cfg.T <= 64 else 20)
+        # The caller's host arrays (numpy views of the pinned buffers), made once, as a caller
+        # holding its activations in host memory would.
+        xa, oa = xh.numpy().view(np.uint16), oh.numpy().view(np.uint16)
+        la = [t.numpy() for t in lgh]
         for i in range(min(warm, 20)):
-            moe.moe_nvfp4_forward_host(xh.numpy().view(np.uint16), lgh[i % nsets].numpy(), banks[0], cfg.k,
-                                       out_host=oh.numpy().view(np.uint16))
+            moe.moe_nvfp4_forward_host(xa, la[i % nsets], banks[0], cfg.k, out_host=oa)
         barrier(ws)
         torch.cuda.synchronize()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(s)
         for i in range(n_e2e):
-            moe.moe_nvfp4_forward_host(xh.numpy().view(np.uint16), lgh[i % nsets].numpy(), banks[0], cfg.k,
-                                       out_host=oh.numpy().view(np.uint16))
+            moe.moe_nvfp4_forward_host(xa, la[i % nsets], banks[0], cfg.k, out_host=oa)
         f1.record(s)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(ws, f0.elapsed_time(f1))

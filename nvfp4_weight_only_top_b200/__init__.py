@@ -101,10 +101,12 @@ def moe_nvfp4_forward_host(x_host: np.ndarray, logits_host: np.ndarray, bank: Ba
     logits_host = np.ascontiguousarray(logits_host, dtype=np.float32)
     if out_host is None:
         out_host = np.empty_like(x_host)
-    _check(lib().moe_nvfp4_forward_host(x_host.ctypes.data_as(ctypes.c_void_p),
-                                        logits_host.ctypes.data_as(ctypes.c_void_p), x_host.shape[0],
-                                        ctypes.byref(bank), k, out_host.ctypes.data_as(ctypes.c_void_p),
-                                        _stream(stream)))
+    elif out_host.dtype != np.uint16 or not out_host.flags.c_contiguous or out_host.shape != x_host.shape:
+        raise ValueError("out_host must be a C-contiguous uint16 array shaped like x_host")
+    # (ctypes.c_void_p of the integer address: a third of the cost of ndarray.ctypes.data_as)
+    _check(lib().moe_nvfp4_forward_host(ctypes.c_void_p(x_host.ctypes.data), ctypes.c_void_p(logits_host.ctypes.data),
+                                        x_host.shape[0], ctypes.byref(bank), k,
+                                        ctypes.c_void_p(out_host.ctypes.data), _stream(stream)))
     return out_host
 
 

@@ -125,3 +125,28 @@ def test_valid_call_without_a_device_fails_loudly():
     """No CPU fallback: with every argument valid and no CUDA device, the call returns an error."""
     assert _fwd(_bank()) == _abi.ERR_UNSUPPORTED
     assert "no CUDA device" in moe.moe_nvfp4_last_error()
+
+
+def test_forward_host_passes_the_callers_buffers(monkeypatch):
+    """The binding hands the C entry point the caller's own host arrays (no copies when they
+    are already contiguous and of the right type) and rejects an output it cannot fill."""
+    calls = []
+
+    class FakeLib:
+        def moe_nvfp4_forward_host(self, x, lg, T, bank, k, out, stream):
+            calls.append((x.value, lg.value, T, k, out.value, stream.value))
+            return 0
+
+    class Stream:
+        cuda_stream = 1234
+
+    monkeypatch.setattr(moe, "_LIB", FakeLib())
+    x = np.zeros((3, 256), np.uint16)
+    lg = np.zeros((3, 16), np.float32)
+    out = np.empty_like(x)
+    assert moe.moe_nvfp4_forward_host(x, lg, _bank(), 2, out_host=out, stream=Stream()) is out
+    assert calls == [(x.ctypes.data, lg.ctypes.data, 3, 2, out.ctypes.data, 1234)]
+    got = moe.moe_nvfp4_forward_host(x, lg.astype(np.float64), _bank(), 2, stream=Stream())
+    assert got.shape == x.shape and got.dtype == np.uint16 and calls[-1][1] != lg.ctypes.data
+    with pytest.raises(ValueError):
+        moe.moe_nvfp4_forward_host(x, lg, _bank(), 2, out_host=np.empty((2, 256), np.uint16), stream=Stream())
