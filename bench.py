@@ -69,11 +69,14 @@ def kernel_traffic(kind: str, workload: str):
     p = os.path.join(ROOT, "profiles", f"{kind}_{workload}.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    h = hashlib.sha256()
-    for name in d.get("sources", [d.get("source")]):     # every file the kernel is built from
-        h.update(open(os.path.join(ROOT, "nvfp4_weight_only_top_b200", "csrc", name), "rb").read())
-    return d["dram_bytes_per_launch"] if h.hexdigest() == d["source_sha256"] else None
+    try:
+        d = json.load(open(p))
+        h = hashlib.sha256()
+        for name in d.get("sources", [d.get("source")]):     # every file the kernel is built from
+            h.update(open(os.path.join(ROOT, "nvfp4_weight_only_top_b200", "csrc", name), "rb").read())
+        return d["dram_bytes_per_launch"] if h.hexdigest() == d["source_sha256"] else None
+    except (OSError, KeyError, TypeError, ValueError):    # an unreadable summary counts as none
+        return None
 
 
 class ClockSampler:

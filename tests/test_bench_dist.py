@@ -79,3 +79,19 @@ def test_reference_arm_rank0_prints_one_line_other_ranks_nothing():
     r1 = _bench(["--impl", "reference", "--config", "decode_t1", "--steps", "1", "--warmup", "0",
                  "--ref-budget", "0.1"], {"WORLD_SIZE": "2", "RANK": "1"})
     assert r1.returncode == 0 and r1.stdout.strip() == ""
+
+
+def test_committed_traffic_summaries_resolve():
+    """Every per-launch DRAM summary under profiles/ names existing kernel sources; the lookup
+    returns its figure while the sources are unchanged and never raises."""
+    import glob
+    import bench
+    files = glob.glob(os.path.join(ROOT, "profiles", "*.json"))
+    assert files
+    for f in files:
+        d = json.load(open(f))
+        for name in d.get("sources", [d.get("source")]):
+            assert os.path.exists(os.path.join(ROOT, "nvfp4_weight_only_top_b200", "csrc", name)), (f, name)
+        v = bench.kernel_traffic(d["kind"], d["workload"])
+        assert v is None or v == d["dram_bytes_per_launch"]
+    assert bench.kernel_traffic("no_such_kernel", "decode_t1") is None
