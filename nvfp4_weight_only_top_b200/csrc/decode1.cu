@@ -403,33 +403,44 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
       }
     }
     // Combine.  Block b = rows 32b .. 32b+31: one down stage per slot, so k contributions.
-    // Each CTA publishes its stages (one fence, one atomic per stage) and combines the blocks
-    // for which it added the last contribution.
-    named_bar_sync(1, 32 * kNW);
+    // One consumer thread per down stage publishes it (fence, then the block's counter), so the
+    // counter round trips overlap instead of queueing behind one thread; a thread that adds a
+    // block's last contribution records the block (s_ok counts them), and the CTA combines the
+    // blocks it recorded.
     int* s_last = s_ok + 1;                                 // blocks this CTA combines
-    if (threadIdx.x == 0) {
-      int n = 0;
-      if (ok) {
+    if (threadIdx.x == 0) *s_ok = 0;                        // every thread read it long ago
+    named_bar_sync(1, 32 * kNW);
+    if (ok)
+      for (int u = lo2 + (int)threadIdx.x; u < hi2; u += 32 * kNW) {
+        const int b = u % (H / kRows2);
         __threadfence();
-        for (int u = lo2; u < hi2; ++u) {
-          const int b = u % (H / kRows2);
-          if (atomicAdd(&block_done[b], 1u) == (unsigned)k - 1u) s_last[n++] = b;
+        if (atomicAdd(&block_done[b], 1u) == (unsigned)k - 1u) {
+          __threadfence();
+          s_last[atomicAdd(s_ok, 1)] = b;
         }
-        if (n) __threadfence();
       }
-      *s_ok = n;
-    }
     named_bar_sync(1, 32 * kNW);
     // The last CTA through here clears the counter set for the call that uses it next.
-    if (threadIdx.x == 0) {
+    // (warp 0: one lane takes the exit count, the whole warp clears the set).
+    if (warp == 0) {
       unsigned* exit_count = p.bar + kMaxK + kMaxBlocks;
-      __threadfence();
-      if (atomicAdd(exit_count, 1u) == gridDim.x - 1) {
-        __threadfence();                    // every other CTA's counter updates come before
-        for (int i = 0; i < kMaxK; ++i) slot_done[i] = 0;
-        for (int i = 0; i < H / 32; ++i) block_done[i] = 0;
-        *exit_count = 0;
+      unsigned last = 0;
+      if (lane == 0) {
         __threadfence();
+        last = atomicAdd(exit_count, 1u) == gridDim.x - 1 ? 1u : 0u;
+        __threadfence();                    // every other CTA's counter updates come before
+      }
+      __syncwarp();
+      if (__shfl_sync(0xFFFFFFFFu, last, 0)) {
+        __threadfence();
+        for (int i = lane; i < kMaxK; i += 32) slot_done[i] = 0;
+        for (int i = lane; i < H / 32; i += 32) block_done[i] = 0;
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();
+          *exit_count = 0;
+          __threadfence();
+        }
       }
     }
     for (int i = warp; i < *s_ok; i += kNW) {
