@@ -44,3 +44,10 @@ from .moe import (  # noqa: F401
     residual_add,
 )
 from .sources import GeneratedRecords  # noqa: F401
+from .encode import (  # noqa: F401
+    e2m1_round,
+    e4m3_round,
+    tensor_global,
+    encode_projection,
+    pack_codes,
+)

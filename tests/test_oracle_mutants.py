@@ -16,11 +16,12 @@ import numpy as np
 import pytest
 
 import oracle
+import oracle.encode
 import oracle.moe
 import oracle.nvfp4
 import oracle.sources
 
-PIN_MODULES = ("test_oracle_nvfp4", "test_oracle_layer")
+PIN_MODULES = ("test_oracle_nvfp4", "test_oracle_layer", "test_oracle_encode")
 
 # (label, oracle module, exact source text, replacement)
 MUTANTS = [
@@ -90,6 +91,21 @@ MUTANTS = [
     ("bf16 rounding keeps 7 bits", "moe", "e.astype(np.int64) - 8", "e.astype(np.int64) - 7"),
     ("residual drops the layer output", "moe", "round_to_bf16_bits(bf16_bits_to_f64(x_bits) + bf16_bits_to_f64(out_bits))",
      "round_to_bf16_bits(bf16_bits_to_f64(x_bits))"),
+    # --- encoder
+    ("rounding ties go up", "encode", "pick_hi = (dhi < dlo) | ((dhi == dlo) & (hi % 2 == 0))", "pick_hi = dhi <= dlo"),
+    ("rounding ties go to odd", "encode", "(hi % 2 == 0)", "(hi % 2 == 1)"),
+    ("global over 448", "encode", "amax / _F32(2688.0)", "amax / _F32(448.0)"),
+    ("global from the first element", "encode", "_F32(np.max(np.abs(w)))", "_F32(np.abs(w).reshape(-1)[0])"),
+    ("block scale not divided by 6", "encode", "denom = _F32(_F32(6.0) * s2)", "denom = s2"),
+    ("block amax signed", "encode", "np.max(np.abs(blocks), axis=2)", "np.max(blocks, axis=2)"),
+    ("block amax along rows", "encode", "amax_b = np.max(np.abs(blocks), axis=2)",
+     "amax_b = np.repeat(np.max(np.abs(blocks), axis=(0, 2))[None, :], blocks.shape[0], axis=0)"),
+    ("codes ignore the block scale", "encode", "r = (blocks / eff[:, :, None])", "r = (blocks / s2)"),
+    ("code sign bit dropped", "encode", "(np.signbit(r).astype(np.int64) << 3)", "(0 * np.signbit(r).astype(np.int64))"),
+    ("mode 1 stores the multiplier", "encode", "stored = s2 if global_mode == 0 else amax", "stored = s2"),
+    ("packed high nibble first", "encode", "(pairs[:, :, 0] | (pairs[:, :, 1] << 4))", "(pairs[:, :, 1] | (pairs[:, :, 0] << 4))"),
+    ("effective scale without the global", "encode", "eff = (E4M3_VALUES[scales].astype(np.float32) * s2)",
+     "eff = (E4M3_VALUES[scales].astype(np.float32) * 1.0)"),
 ]
 
 
