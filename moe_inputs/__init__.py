@@ -13,6 +13,7 @@ from .gen import (  # noqa: F401
     record_bytes,
     bank_host,
     make_x,
+    make_x_wide,
     make_logits,
     sample_tokens,
     disjoint_routing_logits,

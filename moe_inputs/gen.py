@@ -27,9 +27,12 @@ GOLDEN = 0x9E3779B97F4A7C15
 _M1 = 0xBF58476D1CE4E5B9
 _M2 = 0x94D049BB133111EB
 
-# Scale bytes are drawn uniformly over the 49 positive E4M3 encodings 0x18 (2^-4) .. 0x48 (4).
+# Scale bytes are drawn uniformly over the 49 positive E4M3 encodings 0x18 (2^-4) .. 0x48 (4)
+# ("config", the benchmark configurations), or over all 254 non-NaN E4M3 encodings -- zero,
+# subnormals, both signs, up to 448 -- ("all_finite", range tests).
 SCALE_BYTE_LO = 0x18
 SCALE_BYTE_COUNT = 49
+SCALE_KINDS = ("config", "all_finite")
 
 # Record streams.
 STREAM_CODES = 0
@@ -110,7 +113,7 @@ def global_value(H: int, global_mode: int = 0) -> np.float32:
 
 
 def record_bytes(seed: int, layer: int, expert: int, lay: RecordLayout,
-                 global_mode: int = 0) -> np.ndarray:
+                 global_mode: int = 0, scale_kind: str = "config") -> np.ndarray:
     """The lay.record_bytes bytes of record (layer, expert) as uint8 (no stride padding)."""
     out = np.empty(lay.record_bytes, dtype=np.uint8)
     n_code_bytes = 3 * lay.I * lay.H // 2
@@ -121,19 +124,26 @@ def record_bytes(seed: int, layer: int, expert: int, lay: RecordLayout,
     out[0:n_code_bytes] = words.astype('<u8').view(np.uint8)
     ks = stream_key(seed, layer, expert, STREAM_SCALES)
     h = counter_words(ks, n_scale_bytes) & np.uint64(0xFFFFFFFF)
-    sc = (h * np.uint64(SCALE_BYTE_COUNT)) >> np.uint64(32)
-    out[n_code_bytes:n_code_bytes + n_scale_bytes] = (sc + np.uint64(SCALE_BYTE_LO)).astype(np.uint8)
+    if scale_kind == "config":
+        sc = ((h * np.uint64(SCALE_BYTE_COUNT)) >> np.uint64(32)) + np.uint64(SCALE_BYTE_LO)
+    elif scale_kind == "all_finite":
+        i = (h * np.uint64(254)) >> np.uint64(32)            # 0 .. 253 -> 0x00..0x7E, 0x80..0xFE
+        sc = np.where(i < 127, i, i + np.uint64(1))
+    else:
+        raise ValueError(scale_kind)
+    out[n_code_bytes:n_code_bytes + n_scale_bytes] = sc.astype(np.uint8)
     g = np.full(3, global_value(lay.H, global_mode), dtype='<f4')
     out[lay.global_off[0]:lay.global_off[0] + 12] = g.view(np.uint8)
     return out
 
 
-def bank_host(seed: int, layer: int, lay: RecordLayout, global_mode: int = 0) -> np.ndarray:
+def bank_host(seed: int, layer: int, lay: RecordLayout, global_mode: int = 0,
+              scale_kind: str = "config") -> np.ndarray:
     """A whole bank on the host (E * record_stride bytes, padding zero); small banks only."""
     buf = np.zeros(lay.bank_bytes, dtype=np.uint8)
     for e in range(lay.E):
         o = e * lay.record_stride
-        buf[o:o + lay.record_bytes] = record_bytes(seed, layer, e, lay, global_mode)
+        buf[o:o + lay.record_bytes] = record_bytes(seed, layer, e, lay, global_mode, scale_kind)
     return buf
 
 
@@ -190,6 +200,17 @@ def make_x(cfg: LayerConfig, seed: int | None = None, layer: int = 0) -> np.ndar
     s = cfg.seed if seed is None else seed
     x = _rng(s, layer, _TAG_X).standard_normal((cfg.T, cfg.H), dtype=np.float32)
     return to_bf16_bits(x)
+
+
+def make_x_wide(T: int, H: int, exps, seed: int = 0, heavy: bool = False) -> np.ndarray:
+    """Activations [T, H] as BF16 bit patterns whose scale differs per token: token t is
+    N(0, 1) * 2^exps[t % len(exps)] (with heavy, a standard Cauchy draw instead of N(0, 1), so
+    that a few entries of a row are far larger than the rest), rounded to BF16."""
+    rng = _rng(seed, 0, _TAG_X)
+    base = rng.standard_cauchy((T, H)) if heavy else rng.standard_normal((T, H))
+    e = np.asarray([exps[t % len(exps)] for t in range(T)], dtype=np.float64)
+    v = np.clip(base * np.exp2(e)[:, None], -3.0e38, 3.0e38)
+    return to_bf16_bits(v)
 
 
 def make_logits(cfg: LayerConfig, seed: int | None = None, layer: int = 0,

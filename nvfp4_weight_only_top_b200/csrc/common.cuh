@@ -203,6 +203,60 @@ __device__ __forceinline__ void mma_16816(float c[4], const uint32_t a[4], uint3
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// ---------------------------------------------------------------- power-of-two prescale
+//
+// The decode kernels multiply NVFP4 weights with the activations in f16 (packed f16 FMAs, or
+// mma.sync with f16 operands).  BF16 activations and f32 mid values span far more than f16, so
+// every activation vector (one token's x, one routed row's h) is first multiplied by an exact
+// power of two 2^s taken from its largest magnitude: s = min(136 - emax, 126), with emax the
+// largest biased exponent (the 8-bit field that f32 and BF16 share), puts max |v| 2^s in
+// [2^9, 2^10) (below 1 for vectors whose maximum is under 2^-126).
+//  * A sum of 8 products e2m1 x v (|e2m1| <= 6) then stays below 48 x 2^10 = 49152 < 65504.
+//  * Values down to 2^-23 of the vector's maximum stay normal f16 (11 significant bits); below
+//    that they lose bits as f16 subnormals, and below 2^-34 of the maximum they become zero.
+//    Every BF16 value times 2^126 is at least 2^-7, so x never underflows for that reason.
+//  * Results are multiplied by 2^-s in f32, which is exact unless the result itself leaves
+//    the normal f32 range, so the outcome is that of the unscaled arithmetic wherever f16 would
+//    have held the unscaled values.
+// s lies in [-119, 126], so 2^s and 2^-s are both normal f32 values.
+
+// Largest |bf16| bit pattern (sign cleared) of the two halves of a packed pair: magnitudes of
+// finite values order like their patterns, and inf / NaN compare above every finite value.
+__device__ __forceinline__ uint32_t bf16x2_abs_max_bits(uint32_t v) {
+  const uint32_t a = v & 0x7FFF7FFFu;
+  return max(a & 0xFFFFu, a >> 16);
+}
+__device__ __forceinline__ uint32_t f32_abs_bits(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
+
+// s from the largest |bf16| pattern / the largest |f32| pattern.
+__device__ __forceinline__ int prescale_shift_bf16(uint32_t max_abs_bits) {
+  return min(136 - (int)(max_abs_bits >> 7), 126);
+}
+__device__ __forceinline__ int prescale_shift_f32(uint32_t max_abs_bits) {
+  return min(136 - (int)(max_abs_bits >> 23), 126);
+}
+
+// 2^s for s in [-126, 127].
+__device__ __forceinline__ float exp2_int(int s) { return __int_as_float((s + 127) << 23); }
+
+// Two BF16 values (a packed pair) times the power of two f, as a BF16 pair.  Exact unless a
+// scaled value falls below the normal BF16 range, which only happens to values that lie more
+// than 2^-126 below the largest of their vector (f16 flushes those to zero anyway).
+__device__ __forceinline__ uint32_t bf16x2_scaled(uint32_t v, float f) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
+      : "=r"(r)
+      : "f"(bf16_bits_to_f32(v >> 16) * f), "f"(bf16_bits_to_f32(v & 0xFFFFu) * f));
+  return r;
+}
+__device__ __forceinline__ uint4 bf16x8_scaled(uint4 v, float f) {
+  return make_uint4(bf16x2_scaled(v.x, f), bf16x2_scaled(v.y, f), bf16x2_scaled(v.z, f), bf16x2_scaled(v.w, f));
+}
+__device__ __forceinline__ uint32_t bf16x8_abs_max_bits(uint4 v) {
+  return max(max(bf16x2_abs_max_bits(v.x), bf16x2_abs_max_bits(v.y)),
+             max(bf16x2_abs_max_bits(v.z), bf16x2_abs_max_bits(v.w)));
+}
+
 // SwiGLU of one pair: silu(g) * u = g / (1 + e^-g) * u, in f32.
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 

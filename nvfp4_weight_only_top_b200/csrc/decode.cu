@@ -52,33 +52,56 @@ struct DecodeParams {
 
 __host__ __device__ inline int xs_pitch(int K) { return K * 2 + 64; }   // = 64 (mod 128)
 __host__ __device__ inline int off_red(int K, int xrows) { return (xrows * xs_pitch(K) + 127) & ~127; }
-__host__ __device__ inline int smem_total(int K, int xrows) { return off_red(K, xrows) + 2 * kNW * 32 * 16; }
+// + the prescale shifts of the group's activation rows (8 ints).
+__host__ __device__ inline int smem_total(int K, int xrows) { return off_red(K, xrows) + 2 * kNW * 32 * 16 + 32; }
 
 // Stage the group's activations as f16 in fragment order: inside each 128-wide K unit the 8
-// values K0 .. K0+7 with K0 = 32*t + 8*i go to 16-byte chunk 4*i + t.
+// values K0 .. K0+7 with K0 = 32*t + 8*i go to 16-byte chunk 4*i + t.  Row n is stored times
+// 2^xsh[n], its power-of-two prescale into f16, taken first from its largest magnitude (one warp
+// per row); callers bracket the call with CTA barriers.
 template <bool GATEUP>
-__device__ void fill_xs(const DecodeParams& p, uint8_t* xs, int row0, int nrows) {
+__device__ void fill_xs(const DecodeParams& p, uint8_t* xs, int* xsh, int row0, int nrows) {
   const int cpr = p.K / 8;  // chunks of 8 values per row
   const int pitch = xs_pitch(p.K);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int n = warp; n < nrows; n += kNW) {
+    uint32_t m = 0;
+    if (GATEUP) {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.xin) +
+                                                        (size_t)(p.perm[row0 + n] / p.k) * p.K);
+      for (int c = lane; c < cpr; c += 32) m = max(m, bf16x8_abs_max_bits(__ldg(src + c)));
+    } else {
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.xin) + (size_t)(row0 + n) * p.K);
+      for (int c = lane; c < 2 * cpr; c += 32) {
+        const float4 a = __ldg(src + c);
+        m = max(m, max(max(f32_abs_bits(a.x), f32_abs_bits(a.y)), max(f32_abs_bits(a.z), f32_abs_bits(a.w))));
+      }
+    }
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if (lane == 0) xsh[n] = GATEUP ? prescale_shift_bf16(m) : prescale_shift_f32(m);
+  }
+  named_bar_sync(1, kThreads);
   for (int c = threadIdx.x; c < p.xrows * cpr; c += kThreads) {
     const int n = c / cpr, kk = (c - n * cpr) * 8;
     const int u = kk >> 7, q = kk & 127;
     uint4* dst = reinterpret_cast<uint4*>(xs + n * pitch + u * 256 + (((q & 31) >> 3) * 4 + (q >> 5)) * 16);
     uint4 v = make_uint4(0, 0, 0, 0);
     if (n < nrows) {
+      const float f = exp2_int(xsh[n]);
       if (GATEUP) {
         const int t = p.perm[row0 + n] / p.k;
         const uint4 b = __ldg(reinterpret_cast<const uint4*>(
             static_cast<const uint16_t*>(p.xin) + (size_t)t * p.K + kk));
-        v.x = pack_f16x2(bf16_bits_to_f32(b.x & 0xFFFF), bf16_bits_to_f32(b.x >> 16));
-        v.y = pack_f16x2(bf16_bits_to_f32(b.y & 0xFFFF), bf16_bits_to_f32(b.y >> 16));
-        v.z = pack_f16x2(bf16_bits_to_f32(b.z & 0xFFFF), bf16_bits_to_f32(b.z >> 16));
-        v.w = pack_f16x2(bf16_bits_to_f32(b.w & 0xFFFF), bf16_bits_to_f32(b.w >> 16));
+        v.x = pack_f16x2(bf16_bits_to_f32(b.x & 0xFFFF) * f, bf16_bits_to_f32(b.x >> 16) * f);
+        v.y = pack_f16x2(bf16_bits_to_f32(b.y & 0xFFFF) * f, bf16_bits_to_f32(b.y >> 16) * f);
+        v.z = pack_f16x2(bf16_bits_to_f32(b.z & 0xFFFF) * f, bf16_bits_to_f32(b.z >> 16) * f);
+        v.w = pack_f16x2(bf16_bits_to_f32(b.w & 0xFFFF) * f, bf16_bits_to_f32(b.w >> 16) * f);
       } else {
         const float4* src = reinterpret_cast<const float4*>(
             static_cast<const float*>(p.xin) + (size_t)(row0 + n) * p.K + kk);
         const float4 a = src[0], b = src[1];
-        v = make_uint4(pack_f16x2(a.x, a.y), pack_f16x2(a.z, a.w), pack_f16x2(b.x, b.y), pack_f16x2(b.z, b.w));
+        v = make_uint4(pack_f16x2(a.x * f, a.y * f), pack_f16x2(a.z * f, a.w * f), pack_f16x2(b.x * f, b.y * f),
+                       pack_f16x2(b.z * f, b.w * f));
       }
     }
     *dst = v;
@@ -118,6 +141,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* xs = smem;
   float4* red = reinterpret_cast<float4*>(smem + off_red(p.K, p.xrows));
+  int* xsh = reinterpret_cast<int*>(red + 2 * kNW * 32);     // [8] prescale shifts of the group's rows
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tid4 = lane & 3;
   const int tiles = GATEUP ? p.N / 8 : p.N / 16;
@@ -184,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
         nrows = grp.z;
         gm0 = global_mult(*reinterpret_cast<const float*>(c.rec + p.global_off[0]), p.global_mode);
         gm1 = GATEUP ? global_mult(*reinterpret_cast<const float*>(c.rec + p.global_off[1]), p.global_mode) : 0.0f;
-        fill_xs<GATEUP>(p, xs, row0, nrows);
+        fill_xs<GATEUP>(p, xs, xsh, row0, nrows);
         named_bar_sync(1, kThreads);
         cur_g = c.g;
       }
@@ -230,12 +254,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
         for (int cc = 0; cc < 2; ++cc) {
           const int n = 2 * tid4 + cc;
           if (n < nrows) {
+            const float un = exp2_int(-xsh[n]);             // undo the row's prescale
             if (GATEUP) {
-              p.out[(size_t)(row0 + n) * p.N + c.tile * 8 + gid] = silu_mul(cs[cc] * gm0, cs[2 + cc] * gm1);
+              p.out[(size_t)(row0 + n) * p.N + c.tile * 8 + gid] = silu_mul(cs[cc] * un * gm0, cs[2 + cc] * un * gm1);
             } else {
               float* o = p.out + (size_t)(row0 + n) * p.N;
-              o[c.tile * 16 + gid] = cs[cc] * gm0;
-              o[c.tile * 16 + gid + 8] = cs[2 + cc] * gm0;
+              o[c.tile * 16 + gid] = cs[cc] * un * gm0;
+              o[c.tile * 16 + gid + 8] = cs[2 + cc] * un * gm0;
             }
           }
         }

@@ -102,6 +102,9 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
   float* s_w = reinterpret_cast<float*>(s_ids + kMaxK);
   float* s_gm = s_w + kMaxK;                                // [3][kMaxK]
   int* s_ok = reinterpret_cast<int*>(s_gm + 3 * kMaxK);
+  // After s_ok and the kMaxLast blocks to combine: largest |x| pattern per warp ([0, 9)) and
+  // largest |h| pattern per consumer warp and down slot ([16 + 2 w + slot]).
+  uint32_t* s_amax = reinterpret_cast<uint32_t*>(s_ok + 1 + kMaxLast);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k = p.k;
@@ -125,30 +128,46 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
   // Every CTA routes the token itself.  Expert e's rank is the number of experts ahead of it
   // in the order (logit desc, index asc) -- the order of the warp router -- counted by one
   // thread per expert against all E keys; the experts of rank < k fill slots 0 .. k-1.
+  // The logit and this thread's share of x are loaded together.  x goes to shared memory once
+  // per CTA, already multiplied by the power of two 2^shx of its prescale into f16 (shx from the
+  // largest |x|, reduced across the CTA while the routing keys are ranked), 16-byte chunk c of
+  // 32-input unit u at chunk c ^ ((u >> 1) & 3) of the unit, so that the lanes of a warp, which
+  // read consecutive units, hit different banks.
+  constexpr int kXPer = (H / 8 + kThreads1 - 1) / kThreads1;
+  uint4 xv[kXPer];
   {
-    // The logit and this thread's share of x are loaded together; x goes to shared memory once
-    // per CTA, 16-byte chunk c of 32-input unit u at chunk c ^ ((u >> 1) & 3) of the unit, so
-    // that the lanes of a warp, which read consecutive units, hit different banks.
     const int e = threadIdx.x;
     const float lg = (e < kMaxRankE && e < p.E) ? __ldg(p.logits + e) : 0.0f;
-    constexpr int kXPer = (H / 8 + kThreads1 - 1) / kThreads1;
-    uint4 xv[kXPer];
+    uint32_t m = 0;
 #pragma unroll
     for (int t = 0; t < kXPer; ++t) {
       const int i = (int)threadIdx.x + t * kThreads1;
-      if (i < H / 8) xv[t] = __ldg(reinterpret_cast<const uint4*>(p.x) + i);
+      if (i < H / 8) {
+        xv[t] = __ldg(reinterpret_cast<const uint4*>(p.x) + i);
+        m = max(m, bf16x8_abs_max_bits(xv[t]));
+      }
     }
     if (e < kMaxRankE) s_key[e] = e < p.E ? ((uint64_t)rank_key(lg) << 32) | (uint32_t)(0xFFFFFFFFu - e) : 0ull;
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if (lane == 0) s_amax[warp] = m;
+  }
+  __syncthreads();
+  int shx;                                                  // prescale shift of x
+  {
+    uint32_t m = 0;
+#pragma unroll
+    for (int w = 0; w <= kNW; ++w) m = max(m, s_amax[w]);
+    shx = prescale_shift_bf16(m);
+    const float f = exp2_int(shx);
 #pragma unroll
     for (int t = 0; t < kXPer; ++t) {
       const int i = (int)threadIdx.x + t * kThreads1;
       if (i < H / 8) {
         const int u = i >> 2, c = i & 3;
-        reinterpret_cast<uint4*>(sx)[4 * u + (c ^ ((u >> 1) & 3))] = xv[t];
+        reinterpret_cast<uint4*>(sx)[4 * u + (c ^ ((u >> 1) & 3))] = bf16x8_scaled(xv[t], f);
       }
     }
   }
-  __syncthreads();
   if (threadIdx.x < p.E) {
     const uint64_t me = s_key[threadIdx.x];
     int ahead = 0;
@@ -233,6 +252,7 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
     bool ok = true;
     // Phase 1: gate/up.  Warp w takes row r0 + w of both matrices; lane l its units
     // l + 32 u (u < UG) of the row, with x at those K positions held in registers.
+    // x 2^shx enters the f16 products; the gate and up sums are multiplied back by 2^-shx.
     uint32_t xr[UG][16];
 #pragma unroll
     for (int u = 0; u < UG; ++u) {
@@ -285,7 +305,10 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
           break;
         }
       }
-      if (lane == 0) p.h[(size_t)j * I + r] = silu_mul(accG * s_gm[j], accU * s_gm[kMaxK + j]);
+      if (lane == 0) {
+        const float xun = exp2_int(-shx);
+        p.h[(size_t)j * I + r] = silu_mul(accG * xun * s_gm[j], accU * xun * s_gm[kMaxK + j]);
+      }
     }
     // Publish this CTA's gate/up stages per slot, then wait for the slots of its down rows.
     named_bar_sync(1, 32 * kNW);
@@ -308,6 +331,7 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
     // rather than once per warp: every CTA reads the same few KB, so per-warp loads would
     // pile onto the same L2 lines.
     const int jlo = lo2 / (H / kRows2);
+    int sh0 = 0, sh1 = 0;                                   // prescale shifts of h, slots jlo, jlo + 1
     if (ok && hi2 > lo2) {
       // All of a thread's loads are issued before any store, so their latencies overlap.
       constexpr int kPer = (2 * I / 4 + 32 * kNW - 1) / (32 * kNW);
@@ -319,6 +343,37 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
         const int i = (int)threadIdx.x + t * 32 * kNW;
         if (i < n4) v[t] = __ldcg(src + i);
       }
+      // h enters the f16 products as h 2^sh per slot (sh from the slot's largest magnitude,
+      // collected across the consumer warps first); the down sums are multiplied back by 2^-sh.
+      uint32_t m0 = 0, m1 = 0;
+#pragma unroll
+      for (int t = 0; t < kPer; ++t) {
+        const int i = (int)threadIdx.x + t * 32 * kNW;
+        if (i < n4) {
+          const uint32_t a = max(max(f32_abs_bits(v[t].x), f32_abs_bits(v[t].y)),
+                                 max(f32_abs_bits(v[t].z), f32_abs_bits(v[t].w)));
+          if (i < I / 4)
+            m0 = max(m0, a);
+          else
+            m1 = max(m1, a);
+        }
+      }
+      m0 = __reduce_max_sync(0xFFFFFFFFu, m0);
+      m1 = __reduce_max_sync(0xFFFFFFFFu, m1);
+      if (lane == 0) {
+        s_amax[16 + 2 * warp] = m0;
+        s_amax[16 + 2 * warp + 1] = m1;
+      }
+      named_bar_sync(1, 32 * kNW);
+      m0 = m1 = 0;
+#pragma unroll
+      for (int w = 0; w < kNW; ++w) {
+        m0 = max(m0, s_amax[16 + 2 * w]);
+        m1 = max(m1, s_amax[16 + 2 * w + 1]);
+      }
+      sh0 = prescale_shift_f32(m0);
+      sh1 = prescale_shift_f32(m1);
+      const float f0 = exp2_int(sh0), f1 = exp2_int(sh1);
       // Chunk c of unit u (32 floats) of a slot is stored at chunk c ^ (u & 7) of the unit
       // (bank spread for the per-lane reads below).
 #pragma unroll
@@ -326,7 +381,9 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
         const int i = (int)threadIdx.x + t * 32 * kNW;
         if (i < n4) {
           const int sl = i / (I / 4), w = i - sl * (I / 4), u = w >> 3, c = w & 7;
-          reinterpret_cast<float4*>(sh)[sl * (I / 4) + 8 * u + (c ^ (u & 7))] = v[t];
+          const float f = sl ? f1 : f0;
+          reinterpret_cast<float4*>(sh)[sl * (I / 4) + 8 * u + (c ^ (u & 7))] =
+              make_float4(v[t].x * f, v[t].y * f, v[t].z * f, v[t].w * f);
         }
       }
     }
@@ -338,6 +395,7 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
     // changes).
     uint32_t hr[UD][16];
     int hj = -1;
+    int shh = 0;                                            // prescale shift of the h in hr
     for (; q < cnt && ok; ++q) {
       const int s = q % kRing;
       const int u0 = lo2 + (q - cnt1), j = u0 / (H / kRows2), r0 = (u0 - j * (H / kRows2)) * kRows2 + 4 * warp;
@@ -351,6 +409,7 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
       if (j != hj) {
         hj = j;
         const float* hp = sh + (size_t)(j - jlo) * I;
+        shh = j == jlo ? sh0 : sh1;
 #pragma unroll
         for (int u = 0; u < UD; ++u) {
           const int ku = (lane + 32 * u) % kUnits2;
@@ -399,7 +458,7 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
         for (int i = 0; i < 4; ++i) acc[i] += __shfl_xor_sync(0xFFFFFFFFu, acc[i], off);
       if (lane < 4) {
         const float v = lane == 0 ? acc[0] : lane == 1 ? acc[1] : lane == 2 ? acc[2] : acc[3];
-        p.y[(size_t)j * H + r0 + lane] = v * s_gm[2 * kMaxK + j];
+        p.y[(size_t)j * H + r0 + lane] = v * exp2_int(-shh) * s_gm[2 * kMaxK + j];
       }
     }
     // Combine.  Block b = rows 32b .. 32b+31: one down stage per slot, so k contributions.
@@ -461,7 +520,8 @@ int launch_d1(const D1Params& p, int num_sms, cudaStream_t s) {
   constexpr int kStage2 = 4 * kNW * I / 2 + 4 * kNW * I / 16;
   constexpr int kStage = kStage1 > kStage2 ? kStage1 : kStage2;
   const int smem =
-      kRing * kStage + H * 2 + 2 * I * 4 + (2 * kRing + 1) * 8 + kMaxRankE * 8 + 5 * kMaxK * 4 + 4 + 4 * kMaxLast;
+      kRing * kStage + H * 2 + 2 * I * 4 + (2 * kRing + 1) * 8 + kMaxRankE * 8 + 5 * kMaxK * 4 + 4 + 4 * kMaxLast +
+      4 * 32;
   auto kern = decode1_kernel<UG, UD>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return -(int)err;

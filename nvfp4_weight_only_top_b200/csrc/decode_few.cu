@@ -88,6 +88,9 @@ __global__ void __launch_bounds__(kThreads1, 1) decode_few_kernel(const DNParams
   float* s_gm = reinterpret_cast<float*>(s_st + kMaxSlots); // [3][kMaxSlots] global multipliers
   int* s_ok = reinterpret_cast<int*>(s_gm + 3 * kMaxSlots);
   int* s_last = s_ok + 1;                                   // [kMaxLast] (token, block)s to combine
+  // Largest |x| pattern per warp and x buffer ([2 w + b]) and largest |h| pattern per consumer
+  // warp and down slot ([32 + 2 w + slot]).
+  uint32_t* s_amax = reinterpret_cast<uint32_t*>(s_last + kMaxLast);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k = p.k, T = p.T, R = T * k;
@@ -119,13 +122,51 @@ __global__ void __launch_bounds__(kThreads1, 1) decode_few_kernel(const DNParams
       s_st[r] = pr / k;
     }
     __syncthreads();
-    // x of the tokens of slots ra and rb, bank-spread as in the single-token case.
-    for (int i = threadIdx.x; i < 2 * (H / 8); i += blockDim.x) {
+    // x of the tokens of slots ra and rb (buffers b = 0, 1), bank-spread as in the single-token
+    // case and multiplied by the power of two 2^shx[b] of its prescale into f16 (from the
+    // token's largest |x|, reduced across the CTA first).
+    constexpr int kXPer = (2 * (H / 8) + kThreads1 - 1) / kThreads1;
+    uint4 xv[kXPer];
+    uint32_t m0 = 0, m1 = 0;
+#pragma unroll
+    for (int t = 0; t < kXPer; ++t) {
+      const int i = (int)threadIdx.x + t * kThreads1;
       const int b = i / (H / 8), ii = i - b * (H / 8);
-      if (b == 1 && rb == ra) break;
-      const int u = ii >> 2, c = ii & 3;
-      reinterpret_cast<uint4*>(sx + b * H)[4 * u + (c ^ ((u >> 1) & 3))] =
-          __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)s_st[b ? rb : ra] * H) + ii);
+      if (i < 2 * (H / 8) && !(b == 1 && rb == ra)) {
+        xv[t] = __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)s_st[b ? rb : ra] * H) + ii);
+        if (b == 0)
+          m0 = max(m0, bf16x8_abs_max_bits(xv[t]));
+        else
+          m1 = max(m1, bf16x8_abs_max_bits(xv[t]));
+      }
+    }
+    m0 = __reduce_max_sync(0xFFFFFFFFu, m0);
+    m1 = __reduce_max_sync(0xFFFFFFFFu, m1);
+    if (lane == 0) {
+      s_amax[2 * warp] = m0;
+      s_amax[2 * warp + 1] = m1;
+    }
+    __syncthreads();
+    m0 = m1 = 0;
+#pragma unroll
+    for (int w = 0; w <= kNW; ++w) {
+      m0 = max(m0, s_amax[2 * w]);
+      m1 = max(m1, s_amax[2 * w + 1]);
+    }
+    const int sx0 = prescale_shift_bf16(m0), sx1 = prescale_shift_bf16(m1);
+    const float f0 = exp2_int(sx0), f1 = exp2_int(sx1);
+    if (threadIdx.x == 0) {                                 // read back by the gate/up epilogue
+      s_amax[20] = (uint32_t)sx0;
+      s_amax[21] = (uint32_t)sx1;
+    }
+#pragma unroll
+    for (int t = 0; t < kXPer; ++t) {
+      const int i = (int)threadIdx.x + t * kThreads1;
+      const int b = i / (H / 8), ii = i - b * (H / 8);
+      if (i < 2 * (H / 8) && !(b == 1 && rb == ra)) {
+        const int u = ii >> 2, c = ii & 3;
+        reinterpret_cast<uint4*>(sx + b * H)[4 * u + (c ^ ((u >> 1) & 3))] = bf16x8_scaled(xv[t], b ? f1 : f0);
+      }
     }
     __syncthreads();
   }
@@ -245,7 +286,10 @@ __global__ void __launch_bounds__(kThreads1, 1) decode_few_kernel(const DNParams
           break;
         }
       }
-      if (lane == 0) p.h[(size_t)j * I + r] = silu_mul(accG * s_gm[j], accU * s_gm[kMaxSlots + j]);
+      if (lane == 0) {
+        const float xun = exp2_int(-(int)s_amax[20 + (seg == 1 && rb != ra ? 1 : 0)]);
+        p.h[(size_t)j * I + r] = silu_mul(accG * xun * s_gm[j], accU * xun * s_gm[kMaxSlots + j]);
+      }
     }
     }
     // Publish this CTA's gate/up stages per slot, then wait for the slots of its down rows.
@@ -280,6 +324,35 @@ __global__ void __launch_bounds__(kThreads1, 1) decode_few_kernel(const DNParams
         const int i = (int)threadIdx.x + t * 32 * kNW;
         if (i < n4) v[t] = __ldcg(src + i);
       }
+      // h enters the f16 products as h 2^sh per slot (sh from the slot's largest magnitude,
+      // collected across the consumer warps first); the down sums are multiplied back by 2^-sh.
+      uint32_t m0 = 0, m1 = 0;
+#pragma unroll
+      for (int t = 0; t < kPer; ++t) {
+        const int i = (int)threadIdx.x + t * 32 * kNW;
+        if (i < n4) {
+          const uint32_t a = max(max(f32_abs_bits(v[t].x), f32_abs_bits(v[t].y)),
+                                 max(f32_abs_bits(v[t].z), f32_abs_bits(v[t].w)));
+          if (i < I / 4)
+            m0 = max(m0, a);
+          else
+            m1 = max(m1, a);
+        }
+      }
+      m0 = __reduce_max_sync(0xFFFFFFFFu, m0);
+      m1 = __reduce_max_sync(0xFFFFFFFFu, m1);
+      if (lane == 0) {
+        s_amax[32 + 2 * warp] = m0;
+        s_amax[32 + 2 * warp + 1] = m1;
+      }
+      named_bar_sync(1, 32 * kNW);
+      m0 = m1 = 0;
+#pragma unroll
+      for (int w = 0; w < kNW; ++w) {
+        m0 = max(m0, s_amax[32 + 2 * w]);
+        m1 = max(m1, s_amax[32 + 2 * w + 1]);
+      }
+      const float f0 = exp2_int(prescale_shift_f32(m0)), f1 = exp2_int(prescale_shift_f32(m1));
       // Chunk c of unit u (32 floats) of a slot is stored at chunk c ^ (u & 7) of the unit
       // (bank spread for the per-lane reads below).
 #pragma unroll
@@ -287,7 +360,9 @@ __global__ void __launch_bounds__(kThreads1, 1) decode_few_kernel(const DNParams
         const int i = (int)threadIdx.x + t * 32 * kNW;
         if (i < n4) {
           const int sl = i / (I / 4), w = i - sl * (I / 4), u = w >> 3, c = w & 7;
-          reinterpret_cast<float4*>(sh)[sl * (I / 4) + 8 * u + (c ^ (u & 7))] = v[t];
+          const float f = sl ? f1 : f0;
+          reinterpret_cast<float4*>(sh)[sl * (I / 4) + 8 * u + (c ^ (u & 7))] =
+              make_float4(v[t].x * f, v[t].y * f, v[t].z * f, v[t].w * f);
         }
       }
     }
@@ -299,6 +374,7 @@ __global__ void __launch_bounds__(kThreads1, 1) decode_few_kernel(const DNParams
     // changes).
     uint32_t hr[UD][16];
     int hj = -1;
+    int shh = 0;                                            // prescale shift of the h in hr
     for (; q < cnt && ok; ++q) {
       const int s = q % kRing;
       const int u0 = lo2 + (q - cnt1), j = u0 / (H / kRows2), r0 = (u0 - j * (H / kRows2)) * kRows2 + 4 * warp;
@@ -312,6 +388,10 @@ __global__ void __launch_bounds__(kThreads1, 1) decode_few_kernel(const DNParams
       if (j != hj) {
         hj = j;
         const float* hp = sh + (size_t)(j - jlo) * I;
+        uint32_t m = 0;
+#pragma unroll
+        for (int w = 0; w < kNW; ++w) m = max(m, s_amax[32 + 2 * w + (j - jlo)]);
+        shh = prescale_shift_f32(m);
 #pragma unroll
         for (int u = 0; u < UD; ++u) {
           const int ku = (lane + 32 * u) % kUnits2;
@@ -360,7 +440,7 @@ __global__ void __launch_bounds__(kThreads1, 1) decode_few_kernel(const DNParams
         for (int i = 0; i < 4; ++i) acc[i] += __shfl_xor_sync(0xFFFFFFFFu, acc[i], off);
       if (lane < 4) {
         const float v = lane == 0 ? acc[0] : lane == 1 ? acc[1] : lane == 2 ? acc[2] : acc[3];
-        p.y[(size_t)j * H + r0 + lane] = v * s_gm[2 * kMaxSlots + j];
+        p.y[(size_t)j * H + r0 + lane] = v * exp2_int(-shh) * s_gm[2 * kMaxSlots + j];
       }
     }
     // Combine.  Block (t, b) = rows 32b .. 32b+31 of token t: one down stage for each of the
@@ -424,7 +504,8 @@ int launch_dn(const DNParams& p, int num_sms, cudaStream_t s) {
   constexpr int kStage1 = 2 * (kNW * H / 2 + kNW * H / 16);
   constexpr int kStage2 = 4 * kNW * I / 2 + 4 * kNW * I / 16;
   constexpr int kStage = kStage1 > kStage2 ? kStage1 : kStage2;
-  const int smem = kRing * kStage + 2 * H * 2 + 2 * I * 4 + (2 * kRing + 1) * 8 + 5 * kMaxSlots * 4 + 4 + 4 * kMaxLast;
+  const int smem =
+      kRing * kStage + 2 * H * 2 + 2 * I * 4 + (2 * kRing + 1) * 8 + 5 * kMaxSlots * 4 + 4 + 4 * kMaxLast + 4 * 48;
   auto kern = decode_few_kernel<UG, UD>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return -(int)err;

@@ -87,34 +87,56 @@ __device__ __forceinline__ float2 f16x2_to_float2(uint32_t v) {
 // Stores the group's activations as f16 at the lane's own K positions in the warp's slab of
 // shared memory.  Slot (m, q) of lane l -- the 8 values at K = kpos[m] + 8q .. +7 -- lives at
 // 16-byte chunk (4m + q) * 32 + l, so a warp-wide 128-bit read of one slot is conflict-free.
-// Each lane reads back only what it wrote itself.
+// Each lane reads back only what it wrote itself.  The values are stored times 2^s, the
+// power-of-two prescale into f16 taken from the row's largest magnitude (the lanes of the warp
+// together cover the whole row: a first pass finds it); returns s.
 template <int NX, bool GATEUP>
-__device__ __forceinline__ void load_x(const RowParams& p, int prow, const int (&kpos)[NX], uint4* slab, int lane) {
+__device__ __forceinline__ int load_x(const RowParams& p, int prow, const int (&kpos)[NX], uint4* slab, int lane) {
   if (GATEUP) {
     const int t = __ldg(&p.perm[prow]) / p.k;
     const uint16_t* xrow = static_cast<const uint16_t*>(p.xin) + (size_t)t * p.K;
+    uint32_t mx = 0;
+#pragma unroll 1
+    for (int m = 0; m < NX; ++m)
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        mx = max(mx, bf16x8_abs_max_bits(__ldg(reinterpret_cast<const uint4*>(xrow + kpos[m] + 8 * q))));
+    const int sh = prescale_shift_bf16(__reduce_max_sync(0xFFFFFFFFu, mx));
+    const float f = exp2_int(sh);
 #pragma unroll
     for (int m = 0; m < NX; ++m)
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const uint4 b = __ldg(reinterpret_cast<const uint4*>(xrow + kpos[m] + 8 * q));
         slab[(4 * m + q) * 32 + lane] =
-            make_uint4(pack_f16x2(bf16_bits_to_f32(b.x & 0xFFFF), bf16_bits_to_f32(b.x >> 16)),
-                       pack_f16x2(bf16_bits_to_f32(b.y & 0xFFFF), bf16_bits_to_f32(b.y >> 16)),
-                       pack_f16x2(bf16_bits_to_f32(b.z & 0xFFFF), bf16_bits_to_f32(b.z >> 16)),
-                       pack_f16x2(bf16_bits_to_f32(b.w & 0xFFFF), bf16_bits_to_f32(b.w >> 16)));
+            make_uint4(pack_f16x2(bf16_bits_to_f32(b.x & 0xFFFF) * f, bf16_bits_to_f32(b.x >> 16) * f),
+                       pack_f16x2(bf16_bits_to_f32(b.y & 0xFFFF) * f, bf16_bits_to_f32(b.y >> 16) * f),
+                       pack_f16x2(bf16_bits_to_f32(b.z & 0xFFFF) * f, bf16_bits_to_f32(b.z >> 16) * f),
+                       pack_f16x2(bf16_bits_to_f32(b.w & 0xFFFF) * f, bf16_bits_to_f32(b.w >> 16) * f));
       }
+    return sh;
   } else {
     const float* hp = static_cast<const float*>(p.xin) + (size_t)prow * p.K;
+    uint32_t mx = 0;
+#pragma unroll 1
+    for (int m = 0; m < NX; ++m)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(hp + kpos[m] + 4 * q));
+        mx = max(mx, max(max(f32_abs_bits(a.x), f32_abs_bits(a.y)), max(f32_abs_bits(a.z), f32_abs_bits(a.w))));
+      }
+    const int sh = prescale_shift_f32(__reduce_max_sync(0xFFFFFFFFu, mx));
+    const float f = exp2_int(sh);
 #pragma unroll
     for (int m = 0; m < NX; ++m)
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float4 a = __ldg(reinterpret_cast<const float4*>(hp + kpos[m] + 8 * q));
         const float4 b = __ldg(reinterpret_cast<const float4*>(hp + kpos[m] + 8 * q + 4));
-        slab[(4 * m + q) * 32 + lane] =
-            make_uint4(pack_f16x2(a.x, a.y), pack_f16x2(a.z, a.w), pack_f16x2(b.x, b.y), pack_f16x2(b.z, b.w));
+        slab[(4 * m + q) * 32 + lane] = make_uint4(pack_f16x2(a.x * f, a.y * f), pack_f16x2(a.z * f, a.w * f),
+                                                   pack_f16x2(b.x * f, b.y * f), pack_f16x2(b.z * f, b.w * f));
       }
+    return sh;
   }
 }
 
@@ -184,15 +206,15 @@ __global__ void __launch_bounds__(32 * WARPS, 1) rows_kernel(const RowParams p) 
 
   extern __shared__ __align__(16) uint4 x_slabs[];
   uint4* slab = x_slabs + (threadIdx.x >> 5) * (NX * 4 * 32);   // this warp's activations
-  int cur_g = -1;
-  float gmA = 0.0f, gmB = 0.0f;
+  int cur_g = -1, xsh = 0;          // current group, prescale shift of its activations
+  float gmA = 0.0f, gmB = 0.0f;     // global multipliers
 
   auto compute = [&](const Cursor& c, const RowFrag<UPL>& f) {
     if (c.g != cur_g) {
       cur_g = c.g;
       gmA = global_mult(__ldg(reinterpret_cast<const float*>(c.rec + p.global_off[0])), p.global_mode);
       gmB = global_mult(__ldg(reinterpret_cast<const float*>(c.rec + p.global_off[1])), p.global_mode);
-      load_x<NX, GATEUP>(p, c.prow, kpos, slab, lane);
+      xsh = load_x<NX, GATEUP>(p, c.prow, kpos, slab, lane);
       __syncwarp();
     }
     float accA = 0.0f, accB = 0.0f;
@@ -229,10 +251,12 @@ __global__ void __launch_bounds__(32 * WARPS, 1) rows_kernel(const RowParams p) 
       accA += __shfl_xor_sync(0xFFFFFFFFu, accA, off);
       accB += __shfl_xor_sync(0xFFFFFFFFu, accB, off);
     }
+    const float un = exp2_int(-xsh);
     if (GATEUP) {
-      if (lane == 0) p.out[(size_t)c.prow * p.out_stride + c.t] = silu_mul(accA * gmA, accB * gmB);
+      if (lane == 0) p.out[(size_t)c.prow * p.out_stride + c.t] = silu_mul(accA * un * gmA, accB * un * gmB);
     } else if (lane < 2) {
-      p.out[(size_t)c.prow * p.out_stride + (lane == 0 ? row_a(c.t) : row_b(c.t))] = lane == 0 ? accA * gmA : accB * gmB;
+      p.out[(size_t)c.prow * p.out_stride + (lane == 0 ? row_a(c.t) : row_b(c.t))] =
+          lane == 0 ? accA * un * gmA : accB * un * gmB;
     }
   };
 
