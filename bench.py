@@ -1,12 +1,18 @@
 """Benchmark of the NVFP4 weight-only routed-expert MoE layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+    python bench.py --ncu-case NAME --calls N        (plain calls for ncu captures)
 
 One step = one MoE layer call (router -> permute -> expert gate/up + SwiGLU -> down -> combine)
-over one batch of synthetic input resident in HBM.  Default workload: decode, batch 1
-(E=256, k=8, H=5120, I=2560, T=1; ~177 MB of NVFP4 expert records read per step).  Rank 0
-prints one JSON line.  Under torchrun each rank runs an independent replica (no collective
-on the data path; "replicas only"); timing is the max over ranks.
+over one batch of synthetic input resident in HBM (for the 24-layer stack, the whole stack).
+Without --config the run measures every full-size workload: decode, batch 1 (E=256, k=8,
+H=5120, I=2560, T=1; ~177 MB of NVFP4 expert records per step) is the headline of the JSON
+line, and decode T=64 with Zipf routing, prefill T=8192 and the 24-layer verify stack (T=16)
+follow under "workloads", each with its own timing, roofline, kernel shares, clocks and
+end-to-end figure (--steps K applies to the headline; the others take the same share of their
+default step counts).  Rank 0 prints one JSON line.  Under torchrun each rank runs an
+independent replica (no collective on the data path; "replicas only"); timing is the max over
+ranks.
 
 --impl reference times the FP64 CPU oracle (the only reference implementation that exists
 for this method) on the host cores, on a bounded sample of the same workload.
@@ -44,7 +50,13 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
-    ap.add_argument("--config", default="decode_t1", choices=[c for c in moe_inputs.CONFIGS if c != "tiny"])
+    ap.add_argument("--config", default=None, choices=[c for c in moe_inputs.CONFIGS if c != "tiny"],
+                    help="one workload only (default: decode_t1 as the headline, then every other "
+                         "full-size workload in the same line)")
+    ap.add_argument("--ncu-case", default=None, choices=["decode_t1_e16", "decode_t16_e16", "decode_t64_e16",
+                                                        "prefill_t4096_e16"],
+                    help="plain layer calls on a small bank for ncu captures (no timing, no graph)")
+    ap.add_argument("--calls", type=int, default=4, help="layer calls of --ncu-case")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=20.0,
@@ -53,6 +65,8 @@ def parse():
 
 
 DEFAULT_STEPS = {"decode_t1": 20000, "decode_t64_zipf": 2000, "prefill_t8192": 50, "verify24_t16": 100}
+# Fewest steps of a workload measured after the headline (about 50 ms of timed work or more).
+MIN_STEPS = {"decode_t1": 1000, "decode_t64_zipf": 40, "prefill_t8192": 10, "verify24_t16": 5}
 
 
 def load_peaks():
@@ -161,8 +175,18 @@ def replay_stats(replay_ms: list, steps_per_replay: int) -> dict:
     return {"median": med, "best": per[0], "worst": per[-1]}
 
 
-def cpu_oracle_baseline(cfg, budget_s: float = 20.0, max_tokens: int = 64):
-    """Times the FP64 oracle (as it stands) on one host core over a bounded token sample."""
+def _oracle_pool(n: int):
+    """A spawn-context process pool of n oracle workers (never forked after CUDA init)."""
+    import multiprocessing
+    return multiprocessing.get_context("spawn").Pool(n)
+
+
+def cpu_oracle_baseline(cfg, budget_s: float = 20.0, max_tokens: int = 64, cores: int = 1):
+    """Times the FP64 oracle (as it stands) on the host over a bounded token sample.
+
+    cores = 1: one process with one BLAS thread.  cores > 1: the oracle's per-expert work is
+    spread over a spawn process pool of that many single-threaded workers through its map_fn
+    argument (the arithmetic is unchanged)."""
     from threadpoolctl import threadpool_limits
     import oracle
     xb = moe_inputs.make_x(cfg)
@@ -171,20 +195,33 @@ def cpu_oracle_baseline(cfg, budget_s: float = 20.0, max_tokens: int = 64):
     else:
         lg_sets = [moe_inputs.make_logits(cfg, layer=0)]
     src = oracle.GeneratedRecords(cfg.seed, 0, cfg.E, cfg.H, cfg.I)
-    tokens_done, t0, i = 0, time.perf_counter(), 0
-    with threadpool_limits(limits=1):
-        while True:
-            lg = lg_sets[i % len(lg_sets)]
-            t = i % cfg.T
-            oracle.layer_forward(xb, lg, cfg.k, src, tokens=[t])
-            tokens_done += 1
-            i += 1
-            if time.perf_counter() - t0 > budget_s * 0.5 or i >= max_tokens:
-                break
-    dt = time.perf_counter() - t0
-    return {"value": tokens_done / dt, "unit": "tok/s", "cores": 1, "kind": "oracle", "tokens": tokens_done,
-            "sample": f"{tokens_done} token(s) of {cfg.name}, each through the FP64 oracle "
-                      f"(decode of its {cfg.k} expert records + SwiGLU + combine), {dt:.1f} s"}
+    pool = _oracle_pool(cores) if cores > 1 else None
+    map_fn = (lambda fn, jobs: pool.map(fn, list(jobs), chunksize=1)) if pool else map
+    # Tokens per oracle call: one at a time on one core; with a pool, enough tokens per call to
+    # give every worker expert records to decode.
+    per_call = 1 if cores == 1 else max(1, min(cfg.T, (cores + cfg.k - 1) // cfg.k))
+    tokens_done, i = 0, 0
+    try:
+        if pool:                                       # start the workers outside the timed span
+            pool.map(abs, range(cores))
+        t0 = time.perf_counter()
+        with threadpool_limits(limits=1):
+            while True:
+                lg = lg_sets[i % len(lg_sets)]
+                toks = [(tokens_done + j) % cfg.T for j in range(per_call)]
+                oracle.layer_forward(xb, lg, cfg.k, src, tokens=toks, map_fn=map_fn)
+                tokens_done += per_call
+                i += 1
+                if time.perf_counter() - t0 > budget_s * 0.5 or tokens_done >= max_tokens:
+                    break
+        dt = time.perf_counter() - t0
+    finally:
+        if pool:
+            pool.terminate()
+    how = "one process, one BLAS thread" if cores == 1 else f"{cores} single-threaded worker processes"
+    return {"value": tokens_done / dt, "unit": "tok/s", "cores": cores, "kind": "oracle", "tokens": tokens_done,
+            "sample": f"{tokens_done} token(s) of {cfg.name}, {per_call} per oracle call (decode of the routed "
+                      f"expert records + SwiGLU + combine in FP64), {dt:.1f} s, {how}"}
 
 
 def run_reference(args):
@@ -195,7 +232,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    cfg = moe_inputs.CONFIGS[args.config]
+    cfg = moe_inputs.CONFIGS[args.config or HEADLINE]
     steps = args.steps if args.steps is not None else 2
     warm = args.warmup if args.warmup is not None else 0
     if warm > 0:                         # one untimed token (imports, first-touch of the records)
@@ -218,19 +255,12 @@ def workload_config(cfg):
             "layers": cfg.layers, "global_batch": cfg.T, "parallelism": "replicas"}
 
 
-def main():
-    args = parse()
-    if args.impl == "reference":
-        run_reference(args)
-        return
+def measure(cfg, args, ws, rank, local, steps, warm):
+    """Times one workload; returns its record (rank 0) or None (other ranks)."""
     import torch
     import nvfp4_weight_only_top_b200 as moe
     from moe_inputs import device as mdev
 
-    ws, rank, local = dist_init()
-    cfg = moe_inputs.CONFIGS[args.config]
-    steps = args.steps if args.steps is not None else DEFAULT_STEPS[cfg.name]
-    warm = args.warmup if args.warmup is not None else max(3, min(200, steps // 10))
     lay = cfg.layout
     s = torch.cuda.Stream()          # graphs are captured on a non-default stream
     torch.cuda.set_stream(s)
@@ -275,7 +305,9 @@ def main():
     for i in range(warm):
         step(i)
     torch.cuda.synchronize()
-    gsteps = min(GRAPH_STEPS, steps) if cfg.layers == 1 else 1
+    # steps per graph replay: the largest divisor of the step count up to GRAPH_STEPS, so that
+    # exactly `steps` steps are timed
+    gsteps = max(d for d in range(1, min(GRAPH_STEPS, steps) + 1) if steps % d == 0) if cfg.layers == 1 else 1
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=s):
         for i in range(gsteps):
@@ -304,6 +336,7 @@ def main():
     ms_step = ms / steps_eff
     tokens = cfg.T * steps_eff * ws
     value = tokens / (ms / 1000.0)
+    del graph
 
     # ---- per-kernel durations: a second graph of the same steps with kernel-bracketing events
     moe.moe_nvfp4_profile_begin()
@@ -317,12 +350,13 @@ def main():
     prof = moe.moe_nvfp4_profile_end()
     del pgraph
 
-    # ---- end to end through the host-buffer entry point (pinned host memory)
-    e2e = None
+    # ---- end to end from pinned host memory, through the library's public calls
+    xh = torch.from_numpy(xb.view(np.int16)).pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
     if cfg.layers == 1:
-        xh = torch.from_numpy(xb.view(np.int16)).pin_memory()
+        # moe_nvfp4_forward_host: the copies in, the layer, the copy out and the synchronisation
+        # all happen inside the call.
         lgh = [torch.from_numpy(lg_np[i]).pin_memory() for i in range(nsets)]
-        oh = torch.empty_like(xh).pin_memory()
         n_e2e = min(steps_eff, 2000 if cfg.T <= 64 else 20)
         # The caller's host arrays (numpy views of the pinned buffers), made once, as a caller
         # holding its activations in host memory would.
@@ -338,17 +372,44 @@ def main():
             moe.moe_nvfp4_forward_host(xa, la[i % nsets], banks[0], cfg.k, out_host=oa)
         f1.record(s)
         torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(ws, f0.elapsed_time(f1))
-        e2e = {"value": cfg.T * n_e2e * ws / (e2e_ms / 1000.0), "unit": "tok/s",
-               "h2d_bytes_per_step": cfg.T * cfg.H * 2 + cfg.T * cfg.E * 4,
-               "d2h_bytes_per_step": cfg.T * cfg.H * 2, "steps": n_e2e,
-               "api": "moe_nvfp4_forward_host (pinned host x/logits/out, copies and sync inside)"}
+        api = "moe_nvfp4_forward_host (pinned host x/logits/out, copies and sync inside)"
+        h2d = cfg.T * cfg.H * 2 + cfg.T * cfg.E * 4
+    else:
+        # The stack: every step copies x and the layers' router logits in from pinned host
+        # memory, runs the layers through moe_nvfp4_forward_ex (residual included) and copies the
+        # last layer's x back, then synchronises.
+        lgh = torch.from_numpy(lg_np[:cfg.layers]).pin_memory()
+        n_e2e = min(steps_eff, 20)
+        xd, lgd = torch.empty_like(x), torch.empty_like(logits[:cfg.layers])
+
+        def e2e_step():
+            xd.copy_(xh.view(torch.bfloat16), non_blocking=True)
+            lgd.copy_(lgh, non_blocking=True)
+            cur = xd
+            for l in range(cfg.layers):
+                moe.moe_nvfp4_forward_ex(cur, lgd[l], banks[l], cfg.k, out=out, x_next=xs[l + 1], workspace=wsbuf)
+                cur = xs[l + 1]
+            oh.view(torch.bfloat16).copy_(cur, non_blocking=True)
+            s.synchronize()
+
+        for _ in range(min(warm, 3)):
+            e2e_step()
+        barrier(ws)
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(s)
+        for _ in range(n_e2e):
+            e2e_step()
+        f1.record(s)
+        torch.cuda.synchronize()
+        api = f"moe_nvfp4_forward_ex x {cfg.layers} layers (pinned host x and logits in, x out, sync per step)"
+        h2d = cfg.T * cfg.H * 2 + cfg.layers * cfg.T * cfg.E * 4
+    e2e_ms = max_over_ranks(ws, f0.elapsed_time(f1))
+    e2e = {"value": cfg.T * n_e2e * ws / (e2e_ms / 1000.0), "unit": "tok/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": cfg.T * cfg.H * 2, "steps": n_e2e, "api": api}
 
     if rank != 0:
-        if ws > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
-        return
+        return None
 
     # ---- roofline of the dominant kernel
     hbm, tf_burst, tf_sus, peak_kind = load_peaks()
@@ -371,13 +432,13 @@ def main():
         achieved = flops / (dom_ms / 1000.0) / 1e12
         pb = {"prefill_gateup": avg_touched * 2 * proj_bytes(cfg.I, cfg.H) + R * cfg.H * 2 + R * cfg.I * 2,
               "prefill_down": avg_touched * proj_bytes(cfg.H, cfg.I) + R * cfg.I * 2 + R * cfg.H * 4}[dom]
-        # The kernel is timed inside a long back-to-back loop under the power cap, so the
-        # sustained dense BF16 rate is its denominator; the burst fraction is kept beside it.
-        roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": tf_sus, "unit": "TFLOP/s",
-                    "frac": achieved / tf_sus, "frac_of_burst": achieved / tf_burst,
-                    "peak_source": f"{peak_kind} dense BF16 cuBLAS, sustained loop (MEASURED_PEAKS.json; the "
-                                   "timed region is a long back-to-back loop); the kernel computes BF16 x BF16 -> "
-                                   "F32 on tcgen05",
+        # The timed region of this workload lasts well under a second, so the burst dense BF16
+        # rate is the denominator; the fraction of the sustained (power-capped) rate is kept
+        # beside it.
+        roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s",
+                    "frac": achieved / tf_burst, "frac_of_sustained": achieved / tf_sus, "peak_sustained": tf_sus,
+                    "peak_source": f"{peak_kind} dense BF16 cuBLAS, burst (MEASURED_PEAKS.json); the kernel "
+                                   "computes BF16 x BF16 -> F32 on tcgen05",
                     "traffic": kernel_traffic(dom, cfg.name), "algorithmic_flops_per_launch": flops,
                     "algorithmic_bytes_per_launch": pb, "avg_launch_us": dom_ms * 1000.0}
     else:
@@ -390,7 +451,7 @@ def main():
                     "traffic": kernel_traffic(dom, cfg.name), "algorithmic_bytes_per_launch": dom_bytes,
                     "avg_launch_us": dom_ms * 1000.0}
     expert_bytes = avg_touched * (2 * proj_bytes(cfg.I, cfg.H) + proj_bytes(cfg.H, cfg.I)) * per_step_layers
-    line = {
+    rec = {
         "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": ws, "steps": steps_eff, "warmup": warm,
         "ms_per_step": ms_step,
         "ms_per_step_spread": dict(spread, replays=reps, steps_per_replay=gsteps),
@@ -401,6 +462,8 @@ def main():
                                       % (L2_WINDOW - 1) if cfg.name == "decode_t1" else " over rotating logit sets"),
                        graph=f"{gsteps} step(s) per CUDA graph replay"),
         "decode_expert_hbm_gbs": expert_bytes / (ms_step / 1000.0) / 1e9,
+        "decode_expert_hbm_frac": expert_bytes / (ms_step / 1000.0) / 1e9 / hbm,
+        "touched_experts_per_layer": avg_touched,
         "roofline": roofline,
         "kernels_ms_per_step": {k: v[0] / gsteps for k, v in kinds.items()},
         "kernel_share": {k: v[0] / total_ms for k, v in kinds.items()},
@@ -408,12 +471,197 @@ def main():
         "e2e": e2e,
     }
     if cfg.T * cfg.k > 8 * cfg.E:
-        line["layer_tflops"] = 2.0 * R * 3 * cfg.H * cfg.I * per_step_layers / (ms_step / 1000.0) / 1e12
+        tf = 2.0 * R * 3 * cfg.H * cfg.I * per_step_layers / (ms_step / 1000.0) / 1e12
+        rec["layer_tflops"] = tf
+        rec["layer_tflops_frac"] = tf / tf_burst
     if ck is not None:
-        line["clocks"] = ck
-    if ws == 1:
-        line["cpu_baseline"] = cpu_oracle_baseline(cfg)
-    print(json.dumps(line), flush=True)
+        rec["clocks"] = ck
+    return rec
+
+
+def measure_encoder(experts: int = 16, reps: int = 5) -> dict:
+    """NVFP4 encoding of `experts` full-size BF16 experts (gate and up [2560, 5120], down
+    [5120, 2560]) into bank records; HBM-bound.  The algorithmic minimum is one read of the BF16
+    weights and one write of the records (2.5625 B per weight); the kernels read the weights twice
+    (the per-projection maximum first, then the blocks)."""
+    import torch
+    import nvfp4_weight_only_top_b200 as moe
+    H, I = 5120, 2560
+    g = torch.Generator(device="cuda").manual_seed(0)
+    ws = [torch.randn((experts, I, H), generator=g, device="cuda").mul_(0.02).to(torch.bfloat16),
+          torch.randn((experts, I, H), generator=g, device="cuda").mul_(0.02).to(torch.bfloat16),
+          torch.randn((experts, H, I), generator=g, device="cuda").mul_(0.02).to(torch.bfloat16)]
+    lay = moe.record_layout(H, I)
+    buf = torch.empty(experts * lay["record_stride"], dtype=torch.uint8, device="cuda")
+
+    def run():
+        for p, w in enumerate(ws):
+            moe.moe_nvfp4_encode(w, buf, lay["record_stride"], lay["codes_off"][p], lay["scales_off"][p],
+                                 lay["global_off"][p], 1)
+    run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    weights = experts * 3 * H * I
+    hbm, _, _, kind = load_peaks()
+    algo = weights * (2 + 0.5625)
+    moved = weights * (2 * 2 + 0.5625)
+    del ws, buf
+    return {"experts": experts, "ms_per_call": ms, "weights_per_s": weights / (ms / 1e3),
+            "launches": 4 * 3,
+            "roofline": {"bound": "hbm", "achieved": algo / (ms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
+                         "frac": algo / (ms / 1e3) / 1e9 / hbm, "peak_source": f"{kind} HBM copy bandwidth",
+                         "algorithmic_bytes_per_call": algo, "bytes_moved_per_call": moved,
+                         "moved_gbs": moved / (ms / 1e3) / 1e9}}
+
+
+def measure_pack(E: int = 16, slots: int = 8, calls: int = 24) -> dict:
+    """A synthetic streaming pack of one full-size layer (E records of 22,118,412 B at a 4 KiB
+    stride) written to a temporary directory on the host: sha256 verification rate on the host
+    cores, the rate of a whole-layer load (file -> pinned staging -> HBM), and single-token layer
+    calls through an expert-row cache of `slots` slots (cold: every selected expert loaded; warm:
+    every selected expert resident)."""
+    import shutil
+    import tempfile
+    import torch
+    import nvfp4_weight_only_top_b200 as moe
+    from moe_inputs import pack as mpack
+    H, I, k = 5120, 2560, 8
+    d = tempfile.mkdtemp(prefix="moe_pack_")
+    try:
+        mpack.write_pack(d, layers=1, E=E, H=H, I=I, seed=0)
+        p = moe.Pack(os.path.join(d, "expert-manifest.json"))
+        rb = p.info["record_bytes"]
+        t0 = time.perf_counter()
+        p.verify(threads=0)
+        t_ver = time.perf_counter() - t0
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        buf, bank = p.load_bank(0)
+        torch.cuda.synchronize()
+        t_load = time.perf_counter() - t0
+        del buf
+        rows = moe.Rows(p, 0, slots)
+        rng = np.random.default_rng(0)
+        x = torch.from_numpy(moe_inputs.gen.to_bf16_bits(rng.standard_normal((1, H)).astype(np.float32))
+                             .view(np.int16)).view(torch.bfloat16).cuda()
+        lg_cold = [torch.from_numpy(rng.standard_normal((1, E)).astype(np.float32)).cuda() for _ in range(calls)]
+        t0 = time.perf_counter()
+        for lg in lg_cold:
+            rows.forward(x, lg, k)
+        torch.cuda.synchronize()
+        t_mixed = (time.perf_counter() - t0) / calls
+        st = rows.stats()
+        lg_warm = lg_cold[-1]
+        rows.forward(x, lg_warm, k)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(calls):
+            rows.forward(x, lg_warm, k)
+        torch.cuda.synchronize()
+        t_warm = (time.perf_counter() - t0) / calls
+        rows.destroy()
+        p.close()
+        return {"experts": E, "record_bytes": rb, "verify_gbs": E * rb / t_ver / 1e9, "verify_threads": os.cpu_count(),
+                "load_layer_gbs": E * rb / t_load / 1e9, "load_layer_ms": t_load * 1e3,
+                "rows": {"slots": slots, "k": k, "calls": calls, "ms_per_call_random_routing": t_mixed * 1e3,
+                         "hits": st["hits"], "misses": st["misses"], "gb_loaded": st["bytes_loaded"] / 1e9,
+                         "ms_per_call_resident": t_warm * 1e3},
+                "timing": "host wall clock around synchronised calls (the loads include disk or page-cache reads)"}
+    finally:
+        shutil.rmtree(d, ignore_errors=True)
+
+
+# Workloads of the default run: the headline first, then the other full-size configurations.
+HEADLINE = "decode_t1"
+FULL_RUN = ["decode_t1", "decode_t64_zipf", "prefill_t8192", "verify24_t16"]
+
+
+def ncu_case(case: str, calls: int) -> None:
+    """Plain layer calls (no CUDA graph, one stream) on a small bank, for ncu captures.
+
+    Cases (full-size records H=5120, I=2560, 16 experts resident = 354 MB, above the 126 MB L2):
+    decode_t1_e16 (T=1, each call routes to 8 experts the previous call did not use),
+    decode_t16_e16 (T=16), decode_t64_e16 (T=64), prefill_t4096_e16 (T=4096, tensor-core path).
+    """
+    import torch
+    import nvfp4_weight_only_top_b200 as moe
+    from moe_inputs import device as mdev
+    T, path = NCU_CASES[case]
+    E, k, H, I = 16, 8, 5120, 2560
+    lay = moe_inputs.record_layout(E, H, I)
+    buf = mdev.bank_tensor(lay, 0, 0)
+    bank = moe.make_bank(buf.data_ptr(), E, H, I, lay.record_stride, lay.codes_off, lay.scales_off,
+                         lay.global_off, 0)
+    cfg = moe_inputs.LayerConfig(case, E, k, H, I, T)
+    x = torch.from_numpy(moe_inputs.make_x(cfg).view(np.int16)).view(torch.bfloat16).cuda()
+    if T == 1:
+        lg = torch.from_numpy(moe_inputs.disjoint_routing_logits(E, k, calls, 2)).cuda()
+    else:
+        lg = torch.from_numpy(np.stack([moe_inputs.make_logits(cfg, layer=i) for i in range(calls)])).cuda()
+    p = moe.PATH_DECODE if path == "decode" else moe.PATH_PREFILL
+    for i in range(calls):
+        moe.moe_nvfp4_forward_ex(x, lg[i], bank, k, path=p)
+    torch.cuda.synchronize()
+    assert moe.moe_nvfp4_device_status() == 0
+    print(f"{case}: {calls} calls ok")
+
+
+NCU_CASES = {"decode_t1_e16": (1, "decode"), "decode_t16_e16": (16, "decode"), "decode_t64_e16": (64, "decode"),
+             "prefill_t4096_e16": (4096, "prefill")}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    if args.ncu_case:
+        ncu_case(args.ncu_case, args.calls)
+        return
+    import torch
+
+    ws, rank, local = dist_init()
+    names = [args.config] if args.config else FULL_RUN
+    recs = {}
+    for name in names:
+        cfg = moe_inputs.CONFIGS[name]
+        if args.steps is not None and name == names[0]:
+            steps = args.steps
+        elif args.steps is not None:
+            # the same share of each workload's default steps as the headline was given, but at
+            # least MIN_STEPS
+            steps = max(MIN_STEPS[name], round(DEFAULT_STEPS[name] * args.steps / DEFAULT_STEPS[names[0]]))
+        else:
+            steps = DEFAULT_STEPS[name]
+        warm = args.warmup if args.warmup is not None else max(3, min(200, steps // 10))
+        recs[name] = measure(cfg, args, ws, rank, local, steps, warm)
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()                 # free this workload's banks before the next
+    comps = {}
+    if not args.config and rank == 0:
+        comps["encode"] = measure_encoder()
+        torch.cuda.empty_cache()
+        comps["pack"] = measure_pack()
+        torch.cuda.empty_cache()
+    if rank == 0:
+        line = recs[names[0]]
+        if len(names) > 1:
+            line["workloads"] = {n: recs[n] for n in names[1:]}
+        if comps:
+            line["components"] = comps
+        if ws == 1:
+            cfg = moe_inputs.CONFIGS[names[0]]
+            cores = os.cpu_count() or 1
+            one = cpu_oracle_baseline(cfg, budget_s=args.ref_budget)
+            every = cpu_oracle_baseline(cfg, budget_s=args.ref_budget, max_tokens=8 * cores, cores=cores)
+            line["cpu_baseline"] = dict(one, all_cores=every)
+        print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

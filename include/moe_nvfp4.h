@@ -50,6 +50,8 @@ extern "C" {
 #define MOE_NVFP4_ERR_WORKSPACE   (-4)  /* caller workspace too small, or growth refused
                                            during stream capture                             */
 #define MOE_NVFP4_ERR_TIMEOUT     (-5)  /* a bounded device-side wait gave up (device status) */
+#define MOE_NVFP4_ERR_IO          (-6)  /* a pack file could not be opened or read            */
+#define MOE_NVFP4_ERR_INTEGRITY   (-7)  /* a pack record's sha256 differs from its manifest    */
 
 /*
  * Expert-GEMM path selection for moe_nvfp4_forward_ex.
@@ -60,8 +62,11 @@ extern "C" {
  *     kernel over the routed rows (two launches);
  *   otherwise: router kernel(s), grouped GEMV/GEMM kernels, combine.
  *   The persistent kernels take completion counters from 64 library-owned counter sets per
- *   device and kernel, one per call in turn: at most 64 such calls may be in flight at once on
- *   one device.
+ *   device and kernel, one per call in turn, chosen on the host when the call is made (and so
+ *   fixed inside a captured CUDA graph).  Two such calls whose GPU work overlaps -- calls on
+ *   different streams with no ordering between them, concurrent replays of one graph, or a
+ *   graph replay beside an eager call -- may share a set and return wrong results: order them
+ *   on one stream (calls and replays in one stream run one after another).
  * PREFILL (tcgen05 tensor cores, BF16 x BF16 -> F32): H and I multiples of 256.
  */
 #define MOE_NVFP4_PATH_AUTO    0
@@ -115,6 +120,9 @@ int moe_nvfp4_forward(const void* x_dev, const float* logits_dev, int64_t T,
  *  path           MOE_NVFP4_PATH_*; AUTO picks the prefill path when T*k > 8*E and H and I
  *                 are multiples of 256, else the decode path.
  * With a caller workspace nothing is allocated, so the call can be captured in a CUDA graph.
+ * When the call's work has completed, the caller workspace starts with the routing result of
+ * the call, on every path: ids [T, k] int32 at byte 0 and the softmax weights w [T, k] f32 at
+ * byte 256 * ceil(T*k*4 / 256), both as moe_nvfp4_route describes them.
  */
 int moe_nvfp4_forward_ex(const void* x_dev, const float* logits_dev, int64_t T,
                          const moe_nvfp4_bank* bank, int32_t k, void* out_dev,
@@ -164,6 +172,111 @@ int moe_nvfp4_forward_noalloc(const void* x_dev, const float* logits_dev, int64_
 int moe_nvfp4_route(const float* logits_dev, int64_t T, int32_t E, int32_t k, int32_t* ids_dev,
                     float* w_dev, int32_t* counts_dev, int32_t* offsets_dev, int32_t* perm_dev,
                     int32_t* inv_dev, void* stream);
+
+/*
+ * NVFP4 encoder: turns BF16 weights into the bank's NVFP4 parts, so that BF16 experts can feed
+ * the layer.  w_dev holds n projections [n, out_features, in_features] BF16, row-major (rows =
+ * outputs); projection i is written to dst_dev + i * dst_stride: its E2M1 codes at + codes_off
+ * ([out, in/8] little-endian u32 words, low nibble first), its E4M3 block scales at + scales_off
+ * ([out, in/16] bytes, one per 16 inputs of a row) and its f32 global at + global_off -- with
+ * the bank's record layout, one call writes one part role (gate, up or down) of n experts.
+ * The rule (pages "Beam 1.0 501B-A23B, streaming pack, NVFP4 experts / MLX 8-bit residents",
+ * section "What this pack holds", whose MLX block scale is e4m3(s) x (g / 2688), and "Running
+ * Beam-1.0 (501B) on workstation GPUs", data-free NVFP4A16 quantization): amax = max |w| of the
+ * projection, s2 = f32(amax / 2688); block scale = the E4M3 value nearest to
+ * f32(amax_block / f32(6 s2)) (ties to even, saturating at 448); code = the E2M1 value nearest
+ * to f32(w / f32(e4m3 x s2)) (ties to even, saturating at 6) with the sign bit of w, magnitude
+ * 0 where the block scale is 0; every step one f32 operation rounded to nearest even.  The
+ * stored global is s2 (global_mode 0) or g = amax (global_mode 1, the streaming pack's
+ * convention: f32(g / 2688) is then exactly s2).  A projection of zeros stores 0 everywhere.
+ * Inputs must be finite.  Requirements: in_features a multiple of 16; w_dev, dst_dev,
+ * dst_stride and codes_off multiples of 16, global_off of 4; the three parts must not overlap
+ * and (for n > 1) must lie inside dst_stride.  Nothing is allocated (the global slot holds the
+ * running amax until the last of the call's four kernels).  n = 0 returns OK.
+ */
+int moe_nvfp4_encode(const void* w_dev, int64_t n, int32_t out_features, int32_t in_features,
+                     int32_t global_mode, void* dst_dev, uint64_t dst_stride, uint64_t codes_off,
+                     uint64_t scales_off, uint64_t global_off, void* stream);
+
+/*
+ * Streaming packs (page "Beam 1.0 501B-A23B, streaming pack, NVFP4 experts / MLX 8-bit
+ * residents", sections "What this pack holds" and "How to run").  experts.bin holds one record
+ * per (layer, expert), each starting at a multiple of 4 KiB; expert-manifest.json names the
+ * format (mlx-stream-nvfp4-expert-bank-v1) and layout (nvfp4-gud-9part), the source pin, the 9
+ * parts of a record, and the offset, length and sha256 of each record, plus the projections
+ * whose global scale is inexact (global_scale_inexact).  The page prints these fields but not
+ * the JSON schema; this library reads top-level keys "format", "layout", "layers", "experts",
+ * "hidden", "intermediate", "record_bytes", "record_stride", "parts" (objects with "name" in
+ * gate|up|down . codes|scales|global, "offset", "length" inside a record), "records" (objects
+ * with "layer", "expert", "offset", "length", "sha256" as 64 hex digits) and
+ * "global_scale_inexact" (a list).  The pack's globals follow the page's convention: a bank
+ * built from it has global_mode 1 (multiplier f32(g / 2688)).
+ *
+ * moe_nvfp4_pack_open    parses manifest_path and opens bin_path (NULL: experts.bin beside the
+ *                        manifest); checks the format and layout names, the part sizes against
+ *                        hidden and intermediate, 4 KiB-aligned record offsets inside the file.
+ *                        *pack receives an opaque handle (host memory owned by the library until
+ *                        moe_nvfp4_pack_close).  Needs no GPU.
+ * moe_nvfp4_pack_get_info fills the geometry (below).
+ * moe_nvfp4_pack_verify  recomputes the sha256 of every record of `layer` (-1: all layers) on
+ *                        `threads` host threads (0: one per core); *bad receives the number of
+ *                        records whose digest differs, and MOE_NVFP4_ERR_INTEGRITY is returned
+ *                        if any does.  Needs no GPU.
+ * moe_nvfp4_pack_load    copies the records (layer, experts[i]) for i < n (experts NULL: every
+ *                        expert of the layer in order, n ignored) to dst_dev + i * dst_stride:
+ *                        file -> pinned staging buffers (a ring, reused once its copy is done)
+ *                        -> cudaMemcpyAsync on `stream`; with verify != 0 each record's sha256 is
+ *                        checked before its copy and a mismatch stops the load with
+ *                        MOE_NVFP4_ERR_INTEGRITY.  dst_stride >= record_bytes, multiple of 16.
+ *                        Returns once every copy is enqueued.
+ */
+typedef struct moe_nvfp4_pack_info {
+  int32_t layers, experts, hidden, intermediate;
+  uint64_t record_bytes, record_stride;           /* record size and spacing in experts.bin */
+  uint64_t codes_off[3], scales_off[3], global_off[3];  /* gate, up, down parts in a record */
+  int32_t global_mode;                            /* 1: the pack stores g, multiplier f32(g/2688) */
+  int32_t inexact_globals;                        /* entries of global_scale_inexact           */
+} moe_nvfp4_pack_info;
+
+int moe_nvfp4_pack_open(const char* manifest_path, const char* bin_path, void** pack);
+int moe_nvfp4_pack_get_info(const void* pack, moe_nvfp4_pack_info* info);
+int moe_nvfp4_pack_verify(void* pack, int32_t layer, int32_t threads, int64_t* bad);
+int moe_nvfp4_pack_load(void* pack, int32_t layer, const int32_t* experts_host, int32_t n, void* dst_dev,
+                        uint64_t dst_stride, int32_t verify, void* stream);
+int moe_nvfp4_pack_close(void* pack);
+
+/* SHA-256 (FIPS 180-4) of len bytes of host memory into digest_host[32]; the digest the pack
+ * loader checks records with.  Needs no GPU. */
+int moe_nvfp4_sha256(const void* data_host, uint64_t len, uint8_t* digest_host);
+
+/*
+ * Expert rows: a bounded cache of one layer's expert records on the GPU, fed from a pack (the
+ * page's "rows": the expert slots the GPU keeps per routed layer, filled from experts.bin as the
+ * router selects experts).  A layer whose experts do not all fit in device memory runs through
+ * its rows:
+ *  moe_nvfp4_rows_create   allocates `slots` record slots on the current device (slots <= E,
+ *                          <= 256 for the single-token kernel), a copy stream and pinned staging.
+ *  moe_nvfp4_rows_forward  the layer on x_dev [T, H] / logits_dev [T, E] (finite logits) into
+ *                          out_dev [T, H]: routes on the GPU, reads back which experts were
+ *                          selected (one synchronisation of `stream`), loads the missing ones
+ *                          into free slots or the least recently used slots that this call does
+ *                          not need (file -> pinned staging -> the cache's copy stream, which
+ *                          `stream` then waits for), and runs the layer on the slots: each
+ *                          token's logits are mapped onto the slots (selected experts keep their
+ *                          logit, every other slot gets -inf), so the routing, the weights and
+ *                          the output are those of the full layer.  A call that selects more
+ *                          experts than there are slots returns MOE_NVFP4_ERR_UNSUPPORTED.
+ *                          One stream at a time per cache; not capturable (it synchronises).
+ *  moe_nvfp4_rows_stats    hits and misses (selected experts found resident / loaded) and bytes
+ *                          loaded since creation.
+ *  moe_nvfp4_rows_destroy  frees the cache (synchronises its streams).
+ * The pack must stay open while a cache made from it exists.
+ */
+int moe_nvfp4_rows_create(void* pack, int32_t layer, int32_t slots, void** rows);
+int moe_nvfp4_rows_forward(void* rows, const void* x_dev, const float* logits_dev, int64_t T, int32_t k,
+                           void* out_dev, void* stream);
+int moe_nvfp4_rows_stats(const void* rows, int64_t* hits, int64_t* misses, int64_t* bytes_loaded);
+int moe_nvfp4_rows_destroy(void* rows);
 
 /* Bytes of caller workspace moe_nvfp4_forward_ex needs for these sizes and path (AUTO
  * gives the size of the path AUTO would take).  Returns 0 for invalid sizes. */

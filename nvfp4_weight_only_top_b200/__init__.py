@@ -11,7 +11,7 @@ import ctypes
 import numpy as np
 
 from . import _abi
-from ._abi import Bank, MoeError, PATH_AUTO, PATH_DECODE, PATH_PREFILL  # noqa: F401
+from ._abi import Bank, MoeError, PackInfo, PATH_AUTO, PATH_DECODE, PATH_PREFILL  # noqa: F401
 
 _LIB = None
 
@@ -31,6 +31,43 @@ def _check(rc: int) -> None:
 
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(name: str, t, dtype, shape, device: bool = True) -> None:
+    """Raises ValueError unless t is a C-contiguous tensor of this dtype and shape (and, with
+    device, on the current CUDA device).  The C library takes raw pointers and the sizes of the
+    bank descriptor, so a mismatch would read or write out of bounds."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a torch tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device and (not t.is_cuda or t.device.index != torch.cuda.current_device()):
+        raise ValueError(f"{name} must be on the current CUDA device (it is on {t.device})")
+
+
+def _layer_args(x, logits, bank: Bank, out, x_next=None, workspace=None) -> int:
+    """Checks the tensors of a layer call against the bank (layouts first, then devices);
+    returns T."""
+    import torch
+    if not isinstance(x, torch.Tensor) or x.dim() != 2:
+        raise ValueError("x must be a 2-D torch tensor [T, H]")
+    T = int(x.shape[0])
+    need = [("x", x, torch.bfloat16, (T, bank.hidden)), ("logits", logits, torch.float32, (T, bank.num_experts)),
+            ("out", out, torch.bfloat16, (T, bank.hidden))]
+    if x_next is not None:
+        need.append(("x_next", x_next, torch.bfloat16, (T, bank.hidden)))
+    if workspace is not None:
+        need.append(("workspace", workspace, workspace.dtype, tuple(workspace.shape)))
+    for args in need:
+        _need(*args, device=False)
+    for args in need:
+        _need(*args)
+    return T
 
 
 def _stream(stream):
@@ -55,9 +92,9 @@ def make_bank(base_ptr: int, num_experts: int, hidden: int, intermediate: int, r
 def moe_nvfp4_forward(x, logits, bank: Bank, k: int, out=None, stream=None):
     """out [T, H] bf16 = MoE(x [T, H] bf16, logits [T, E] f32) on the current device."""
     import torch
-    T = x.shape[0]
-    if out is None:
+    if out is None and isinstance(x, torch.Tensor):
         out = torch.empty_like(x)
+    T = _layer_args(x, logits, bank, out)
     _check(lib().moe_nvfp4_forward(_ptr(x), _ptr(logits), T, ctypes.byref(bank), k, _ptr(out),
                                    _stream(stream)))
     return out
@@ -67,9 +104,9 @@ def moe_nvfp4_forward_ex(x, logits, bank: Bank, k: int, out=None, x_next=None, w
                          path: int = PATH_AUTO, stream=None):
     """As moe_nvfp4_forward, with optional residual output, caller workspace and path."""
     import torch
-    T = x.shape[0]
-    if out is None:
+    if out is None and isinstance(x, torch.Tensor):
         out = torch.empty_like(x)
+    T = _layer_args(x, logits, bank, out, x_next, workspace)
     wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().moe_nvfp4_forward_ex(_ptr(x), _ptr(logits), T, ctypes.byref(bank), k, _ptr(out),
                                       _ptr(x_next), _ptr(workspace), wsb, path, _stream(stream)))
@@ -83,9 +120,10 @@ def moe_nvfp4_forward_noalloc(x, logits, bank: Bank, k: int, out=None, stream=No
     that the call itself allocates nothing on the Python side either.
     """
     import torch
-    if out is None:
+    if out is None and isinstance(x, torch.Tensor):
         out = torch.empty_like(x)
-    _check(lib().moe_nvfp4_forward_noalloc(_ptr(x), _ptr(logits), x.shape[0], ctypes.byref(bank), k, _ptr(out),
+    T = _layer_args(x, logits, bank, out)
+    _check(lib().moe_nvfp4_forward_noalloc(_ptr(x), _ptr(logits), T, ctypes.byref(bank), k, _ptr(out),
                                            _stream(stream)))
     return out
 
@@ -99,6 +137,10 @@ def moe_nvfp4_forward_host(x_host: np.ndarray, logits_host: np.ndarray, bank: Ba
     """
     x_host = np.ascontiguousarray(x_host, dtype=np.uint16)
     logits_host = np.ascontiguousarray(logits_host, dtype=np.float32)
+    if x_host.ndim != 2 or x_host.shape[1] != bank.hidden:
+        raise ValueError(f"x_host has shape {x_host.shape}, expected [T, {bank.hidden}]")
+    if logits_host.shape != (x_host.shape[0], bank.num_experts):
+        raise ValueError(f"logits_host has shape {logits_host.shape}, expected {(x_host.shape[0], bank.num_experts)}")
     if out_host is None:
         out_host = np.empty_like(x_host)
     elif out_host.dtype != np.uint16 or not out_host.flags.c_contiguous or out_host.shape != x_host.shape:
@@ -113,7 +155,10 @@ def moe_nvfp4_forward_host(x_host: np.ndarray, logits_host: np.ndarray, bank: Ba
 def moe_nvfp4_route(logits, k: int, stream=None) -> dict:
     """Routing only: ids, w, counts, offsets, perm, inv (int32 / f32 CUDA tensors)."""
     import torch
-    T, E = logits.shape
+    if not isinstance(logits, torch.Tensor) or logits.dim() != 2:
+        raise ValueError("logits must be a 2-D torch tensor [T, E]")
+    T, E = (int(v) for v in logits.shape)
+    _need("logits", logits, torch.float32, (T, E))
     dev = logits.device
     r = dict(ids=torch.empty((T, k), dtype=torch.int32, device=dev),
              w=torch.empty((T, k), dtype=torch.float32, device=dev),
@@ -124,6 +169,148 @@ def moe_nvfp4_route(logits, k: int, stream=None) -> dict:
     _check(lib().moe_nvfp4_route(_ptr(logits), T, E, k, _ptr(r["ids"]), _ptr(r["w"]), _ptr(r["counts"]),
                                  _ptr(r["offsets"]), _ptr(r["perm"]), _ptr(r["inv"]), _stream(stream)))
     return r
+
+
+def moe_nvfp4_encode(w, dst, dst_stride: int, codes_off: int, scales_off: int, global_off: int,
+                     global_mode: int = 0, stream=None) -> None:
+    """NVFP4-encode n projections w [n, out, in] (bf16 CUDA tensor) into the uint8 CUDA tensor dst:
+    projection i's codes, block scales and global at byte i * dst_stride + the part offsets."""
+    import torch
+    if not isinstance(w, torch.Tensor) or w.dim() != 3:
+        raise ValueError("w must be a 3-D torch tensor [n, out, in]")
+    n, out_f, in_f = (int(v) for v in w.shape)
+    if not isinstance(dst, torch.Tensor) or dst.dim() != 1:
+        raise ValueError("dst must be a 1-D torch uint8 tensor")
+    end = max(codes_off + out_f * in_f // 2, scales_off + out_f * in_f // 16, global_off + 4)
+    need = (n - 1) * dst_stride + end if n else 0
+    if dst.numel() < need:
+        raise ValueError(f"dst holds {dst.numel()} bytes; {need} are needed")
+    for args in (("w", w, torch.bfloat16, (n, out_f, in_f)), ("dst", dst, torch.uint8, (dst.numel(),))):
+        _need(*args, device=False)
+    for args in (("w", w, torch.bfloat16, (n, out_f, in_f)), ("dst", dst, torch.uint8, (dst.numel(),))):
+        _need(*args)
+    _check(lib().moe_nvfp4_encode(_ptr(w), n, out_f, in_f, global_mode, _ptr(dst), dst_stride, codes_off,
+                                  scales_off, global_off, _stream(stream)))
+
+
+def record_layout(hidden: int, intermediate: int, align: int = 4096) -> dict:
+    """The library's expert record: gate, up, down codes, then their block scales, then three f32
+    globals, each part 16-byte aligned; records `align` bytes apart (4 KiB, as in the streaming
+    pack: 22,118,412 B records every 22,122,496 B at hidden 5,120, intermediate 2,560)."""
+    c = hidden * intermediate // 2
+    sc = hidden * intermediate // 16
+    g0 = 3 * c + 3 * sc
+    rec = g0 + 12
+    return {"record_bytes": rec, "record_stride": -(-rec // align) * align,
+            "codes_off": (0, c, 2 * c), "scales_off": (3 * c, 3 * c + sc, 3 * c + 2 * sc),
+            "global_off": (g0, g0 + 4, g0 + 8)}
+
+
+def encode_bank(gate, up, down, global_mode: int = 0, stream=None):
+    """A device bank from BF16 expert weights: gate and up [E, I, H], down [E, H, I] (bf16 CUDA
+    tensors).  Returns (uint8 CUDA tensor holding the records, moe_nvfp4_bank)."""
+    import torch
+    E, I, H = (int(v) for v in gate.shape)
+    if tuple(up.shape) != (E, I, H) or tuple(down.shape) != (E, H, I):
+        raise ValueError("gate and up must be [E, I, H] and down [E, H, I]")
+    lay = record_layout(H, I)
+    buf = torch.zeros(E * lay["record_stride"], dtype=torch.uint8, device=gate.device)
+    for p, w in enumerate((gate, up, down)):
+        moe_nvfp4_encode(w, buf, lay["record_stride"], lay["codes_off"][p], lay["scales_off"][p],
+                         lay["global_off"][p], global_mode, stream)
+    bank = make_bank(buf.data_ptr(), E, H, I, lay["record_stride"], lay["codes_off"], lay["scales_off"],
+                     lay["global_off"], global_mode)
+    return buf, bank
+
+
+def moe_nvfp4_sha256(data: bytes) -> bytes:
+    """SHA-256 digest of host bytes (the digest the pack loader checks records with)."""
+    buf = (ctypes.c_uint8 * 32)()
+    src = ctypes.create_string_buffer(bytes(data), len(data)) if len(data) else None
+    _check(lib().moe_nvfp4_sha256(src, len(data), buf))
+    return bytes(buf)
+
+
+class Pack:
+    """An open streaming pack (moe_nvfp4_pack_open): experts.bin records and their manifest."""
+
+    def __init__(self, manifest_path: str, bin_path: str | None = None):
+        h = ctypes.c_void_p()
+        _check(lib().moe_nvfp4_pack_open(manifest_path.encode(), bin_path.encode() if bin_path else None,
+                                         ctypes.byref(h)))
+        self.handle = h
+        info = PackInfo()
+        _check(lib().moe_nvfp4_pack_get_info(h, ctypes.byref(info)))
+        self.info = {name: (list(getattr(info, name)) if name.endswith("_off") else getattr(info, name))
+                     for name, _ in PackInfo._fields_}
+
+    def verify(self, layer: int = -1, threads: int = 0) -> int:
+        """sha256 check of the records of a layer (-1: all); returns the number that differ
+        (raises MoeError with code ERR_INTEGRITY if any does)."""
+        bad = ctypes.c_int64()
+        rc = lib().moe_nvfp4_pack_verify(self.handle, layer, threads, ctypes.byref(bad))
+        if rc == _abi.ERR_INTEGRITY:
+            raise MoeError(rc, lib().moe_nvfp4_last_error().decode() + f" ({bad.value} bad)")
+        _check(rc)
+        return int(bad.value)
+
+    def load(self, layer: int, dst, experts=None, dst_stride: int | None = None, verify: bool = False,
+             stream=None) -> None:
+        """Copies records (layer, experts[i]) (all experts if None) into the uint8 CUDA tensor dst,
+        record i at byte i * dst_stride (default: the pack's record stride)."""
+        import torch
+        stride = int(dst_stride or self.info["record_stride"])
+        n = self.info["experts"] if experts is None else len(experts)
+        if n and dst.numel() < (n - 1) * stride + self.info["record_bytes"]:
+            raise ValueError("dst is too small for the records")
+        _need("dst", dst, torch.uint8, (dst.numel(),))
+        arr = None if experts is None else (ctypes.c_int32 * n)(*[int(e) for e in experts])
+        _check(lib().moe_nvfp4_pack_load(self.handle, layer, arr, n, _ptr(dst), stride, int(verify), _stream(stream)))
+
+    def load_bank(self, layer: int, verify: bool = False, stream=None):
+        """A whole layer resident on the current device: (uint8 tensor, moe_nvfp4_bank)."""
+        import torch
+        i = self.info
+        buf = torch.empty(i["experts"] * i["record_stride"], dtype=torch.uint8, device="cuda")
+        self.load(layer, buf, verify=verify, stream=stream)
+        bank = make_bank(buf.data_ptr(), i["experts"], i["hidden"], i["intermediate"], i["record_stride"],
+                         i["codes_off"], i["scales_off"], i["global_off"], i["global_mode"])
+        return buf, bank
+
+    def close(self) -> None:
+        if self.handle:
+            lib().moe_nvfp4_pack_close(self.handle)
+            self.handle = None
+
+
+class Rows:
+    """A bounded GPU cache of one layer's expert records fed from a pack (moe_nvfp4_rows_*)."""
+
+    def __init__(self, pack: Pack, layer: int, slots: int):
+        h = ctypes.c_void_p()
+        _check(lib().moe_nvfp4_rows_create(pack.handle, layer, slots, ctypes.byref(h)))
+        self.handle, self.pack = h, pack
+
+    def forward(self, x, logits, k: int, out=None, stream=None):
+        import torch
+        i = self.pack.info
+        if out is None and isinstance(x, torch.Tensor):
+            out = torch.empty_like(x)
+        bank = Bank()
+        bank.hidden, bank.num_experts = i["hidden"], i["experts"]
+        T = _layer_args(x, logits, bank, out)
+        _check(lib().moe_nvfp4_rows_forward(self.handle, _ptr(x), _ptr(logits), T, k, _ptr(out), _stream(stream)))
+        return out
+
+    def stats(self) -> dict:
+        h, m, b = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        _check(lib().moe_nvfp4_rows_stats(self.handle, ctypes.byref(h), ctypes.byref(m), ctypes.byref(b)))
+        return {"hits": h.value, "misses": m.value, "bytes_loaded": b.value}
+
+    def destroy(self) -> None:
+        if self.handle:
+            lib().moe_nvfp4_rows_destroy(self.handle)
+            self.handle = None
 
 
 def moe_nvfp4_workspace_bytes(T: int, E: int, k: int, H: int, I: int, path: int = PATH_AUTO) -> int:

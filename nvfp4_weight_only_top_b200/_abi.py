@@ -18,6 +18,8 @@ ERR_UNSUPPORTED = -2
 ERR_CUDA = -3
 ERR_WORKSPACE = -4
 ERR_TIMEOUT = -5
+ERR_IO = -6
+ERR_INTEGRITY = -7
 
 PATH_AUTO = 0
 PATH_DECODE = 1
@@ -40,7 +42,7 @@ class Bank(ctypes.Structure):
 
 
 # Every symbol include/moe_nvfp4.h declares, with its argument and return types.
-_vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+_vp, _i32, _i64, _sz, _u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint64
 _BANKP = ctypes.POINTER(Bank)
 SIGNATURES = {
     "moe_nvfp4_forward": (ctypes.c_int, [_vp, _vp, _i64, _BANKP, _i32, _vp, _vp]),
@@ -49,6 +51,17 @@ SIGNATURES = {
     "moe_nvfp4_forward_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _BANKP, _i32, _vp, _vp]),
     "moe_nvfp4_route": (ctypes.c_int, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_nvfp4_workspace_bytes": (ctypes.c_size_t, [_i64, _i32, _i32, _i32, _i32, _i32]),
+    "moe_nvfp4_encode": (ctypes.c_int, [_vp, _i64, _i32, _i32, _i32, _vp, _u64, _u64, _u64, _u64, _vp]),
+    "moe_nvfp4_pack_open": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_char_p, ctypes.POINTER(_vp)]),
+    "moe_nvfp4_pack_get_info": (ctypes.c_int, [_vp, _vp]),
+    "moe_nvfp4_pack_verify": (ctypes.c_int, [_vp, _i32, _i32, ctypes.POINTER(_i64)]),
+    "moe_nvfp4_pack_load": (ctypes.c_int, [_vp, _i32, _vp, _i32, _vp, _u64, _i32, _vp]),
+    "moe_nvfp4_pack_close": (ctypes.c_int, [_vp]),
+    "moe_nvfp4_sha256": (ctypes.c_int, [_vp, _u64, _vp]),
+    "moe_nvfp4_rows_create": (ctypes.c_int, [_vp, _i32, _i32, ctypes.POINTER(_vp)]),
+    "moe_nvfp4_rows_forward": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i32, _vp, _vp]),
+    "moe_nvfp4_rows_stats": (ctypes.c_int, [_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i64)]),
+    "moe_nvfp4_rows_destroy": (ctypes.c_int, [_vp]),
     "moe_nvfp4_last_error": (ctypes.c_char_p, []),
     "moe_nvfp4_device_status": (ctypes.c_int, []),
     "moe_nvfp4_last_launch_count": (ctypes.c_int, []),
@@ -58,6 +71,23 @@ SIGNATURES = {
 
 KERNEL_KINDS = ["route", "decode_gateup", "decode_down", "combine", "prefill_gather",
                 "prefill_gateup", "prefill_down", "decode_fused"]
+
+
+class PackInfo(ctypes.Structure):
+    """moe_nvfp4_pack_info."""
+    _fields_ = [
+        ("layers", ctypes.c_int32),
+        ("experts", ctypes.c_int32),
+        ("hidden", ctypes.c_int32),
+        ("intermediate", ctypes.c_int32),
+        ("record_bytes", ctypes.c_uint64),
+        ("record_stride", ctypes.c_uint64),
+        ("codes_off", ctypes.c_uint64 * 3),
+        ("scales_off", ctypes.c_uint64 * 3),
+        ("global_off", ctypes.c_uint64 * 3),
+        ("global_mode", ctypes.c_int32),
+        ("inexact_globals", ctypes.c_int32),
+    ]
 
 
 def load(path: str = LIB_PATH) -> ctypes.CDLL:

@@ -98,4 +98,16 @@ int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const
 int launch_prefill_down(const BankView& bank, const void* hb, int64_t R, const RouteBufs& rb, float* y,
                         unsigned* tile_ctr, int num_sms, cudaStream_t s);
 
+// NVFP4 encoder: n projections [n, out_f, in_f] of BF16 weights -> codes, block scales and the
+// stored global of projection i at dst + i * stride + {codes_off, scales_off, global_off}.
+// Returns the number of kernels launched or a negative cudaError_t.
+int launch_encode(const uint16_t* w, int64_t n, int out_f, int in_f, int global_mode, uint8_t* dst, uint64_t stride,
+                  uint64_t codes_off, uint64_t scales_off, uint64_t global_off, int num_sms, cudaStream_t s);
+
+// C-ABI bridge (moe_nvfp4.cu): status and message of the calling host thread, the current
+// device (sm_100 check, SM count).
+int api_fail(int code, const char* msg);
+int api_cuda_fail(int err, const char* what);
+int api_device(int* dev, int* sms);
+
 }  // namespace moe

@@ -2,10 +2,12 @@
 // management and the launch sequence (route -> expert GEMMs -> combine).
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <memory>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -56,7 +58,9 @@ struct HostStage {
   void* out = nullptr;
   size_t x_bytes = 0, logits_bytes = 0, out_bytes = 0;
 };
-std::vector<HostStage> g_stage;
+// One record per device, held by pointer so that growing the vector for another device never
+// moves a record a caller is using.
+std::vector<std::unique_ptr<HostStage>> g_stage;
 
 int current_device(int* dev, DeviceInfo* info) {
   cudaError_t e = cudaGetDevice(dev);
@@ -67,6 +71,7 @@ int current_device(int* dev, DeviceInfo* info) {
     g_ws.resize(*dev + 1);
     g_stage.resize(*dev + 1);
   }
+  if (!g_stage[*dev]) g_stage[*dev].reset(new HostStage());
   DeviceInfo& d = g_info[*dev];
   if (d.sms == 0) {
     cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, *dev);
@@ -463,6 +468,23 @@ int noalloc_scratch(int dev, void** out) {
 
 }  // namespace
 
+// Bridge for the other translation units of the C ABI (pack.cu): error reporting and the
+// current device's checks, with the same semantics as the entry points here.
+namespace moe {
+
+int api_fail(int code, const char* msg) { return fail(code, "%s", msg); }
+
+int api_cuda_fail(int err, const char* what) { return cuda_fail((cudaError_t)err, what); }
+
+int api_device(int* dev, int* sms) {
+  DeviceInfo info;
+  const int rc = current_device(dev, &info);
+  if (rc == MOE_NVFP4_OK) *sms = info.sms;
+  return rc;
+}
+
+}  // namespace moe
+
 extern "C" {
 
 int moe_nvfp4_forward(const void* x_dev, const float* logits_dev, int64_t T, const moe_nvfp4_bank* bank, int32_t k,
@@ -492,7 +514,7 @@ int moe_nvfp4_forward_host(const void* x_host, const float* logits_host, int64_t
   HostStage* st;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    st = &g_stage[dev];
+    st = g_stage[dev].get();
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (xb > st->x_bytes || lb > st->logits_bytes || xb > st->out_bytes) {
@@ -594,6 +616,46 @@ int moe_nvfp4_forward_noalloc(const void* x_dev, const float* logits_dev, int64_
   if ((rc = noalloc_scratch(dev, &scratch))) return rc;
   return forward_impl(x_dev, logits_dev, T, bank, k, out_dev, nullptr, scratch, kNoAllocBytes,
                       MOE_NVFP4_PATH_AUTO, stream);
+}
+
+int moe_nvfp4_encode(const void* w_dev, int64_t n, int32_t out_features, int32_t in_features, int32_t global_mode,
+                     void* dst_dev, uint64_t dst_stride, uint64_t codes_off, uint64_t scales_off, uint64_t global_off,
+                     void* stream) {
+  t_last_launches = 0;
+  if (n < 0) return fail(MOE_NVFP4_ERR_INVALID_ARG, "n = %lld is negative", (long long)n);
+  if (out_features < 1 || in_features < 16 || in_features % 16)
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "shape [%d, %d]: out must be >= 1 and in a positive multiple of 16",
+                out_features, in_features);
+  if (global_mode != 0 && global_mode != 1)
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "global_mode %d is not 0 or 1", global_mode);
+  const uint64_t weights = (uint64_t)out_features * (uint64_t)in_features;
+  const uint64_t cb = weights / 2, sb = weights / 16;
+  if (codes_off % 16 || global_off % 4 || dst_stride % 16)
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "codes_off and dst_stride must be multiples of 16, global_off of 4");
+  auto overlap = [](uint64_t a, uint64_t al, uint64_t b, uint64_t bl) { return a < b + bl && b < a + al; };
+  if (overlap(codes_off, cb, scales_off, sb) || overlap(codes_off, cb, global_off, 4) ||
+      overlap(scales_off, sb, global_off, 4))
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "the codes, scales and global parts overlap");
+  const uint64_t end = std::max(codes_off + cb, std::max(scales_off + sb, global_off + 4));
+  if (n > 1 && end > dst_stride)
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "a projection's parts (%llu bytes) do not fit in dst_stride %llu",
+                (unsigned long long)end, (unsigned long long)dst_stride);
+  int dev, rc;
+  DeviceInfo info;
+  if ((rc = current_device(&dev, &info))) return rc;
+  if (n == 0) return MOE_NVFP4_OK;
+  if (!w_dev || !dst_dev) return fail(MOE_NVFP4_ERR_INVALID_ARG, "w and dst must not be NULL");
+  if (!aligned(w_dev, 16) || !aligned(dst_dev, 16))
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "w and dst must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int launches = 0;
+  if ((rc = after_launch(moe::launch_encode(static_cast<const uint16_t*>(w_dev), n, out_features, in_features,
+                                            global_mode, static_cast<uint8_t*>(dst_dev), dst_stride, codes_off,
+                                            scales_off, global_off, info.sms, s),
+                         s, "encode", &launches)))
+    return rc;
+  t_last_launches = launches;
+  return MOE_NVFP4_OK;
 }
 
 int moe_nvfp4_last_launch_count(void) { return t_last_launches; }

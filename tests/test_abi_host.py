@@ -150,3 +150,80 @@ def test_forward_host_passes_the_callers_buffers(monkeypatch):
     assert got.shape == x.shape and got.dtype == np.uint16 and calls[-1][1] != lg.ctypes.data
     with pytest.raises(ValueError):
         moe.moe_nvfp4_forward_host(x, lg, _bank(), 2, out_host=np.empty((2, 256), np.uint16), stream=Stream())
+
+
+# The Python binding checks tensors against the bank before calling the C library, which only
+# sees raw pointers: a wrong width, dtype, layout or device would otherwise read or write out of
+# bounds.  These run on the CPU: every check fires before any CUDA call.
+def _cpu(shape, dtype):
+    import torch
+    return torch.zeros(shape, dtype=dtype)
+
+
+@pytest.mark.parametrize("which,bad,msg", [
+    ("x", ("shape", (4, 128)), "x has shape"),
+    ("x", ("dtype", "float16"), "x has dtype"),
+    ("logits", ("shape", (4, 15)), "logits has shape"),
+    ("logits", ("dtype", "float64"), "logits has dtype"),
+    ("out", ("shape", (3, 256)), "out has shape"),
+    ("x", ("strided", None), "x must be contiguous"),
+    ("x", ("cpu", None), "x must be on the current CUDA device"),
+])
+def test_binding_rejects_mismatched_tensors(which, bad, msg):
+    import torch
+    bank = _bank()
+    t = dict(x=_cpu((4, 256), torch.bfloat16), logits=_cpu((4, 16), torch.float32), out=_cpu((4, 256), torch.bfloat16))
+    kind, val = bad
+    if kind == "shape":
+        t[which] = _cpu(val, t[which].dtype)
+    elif kind == "dtype":
+        t[which] = _cpu(tuple(t[which].shape), getattr(torch, val))
+    elif kind == "strided":
+        t[which] = _cpu((256, 4), t[which].dtype).t()
+    for fn in (lambda: moe.moe_nvfp4_forward(t["x"], t["logits"], bank, 2, out=t["out"]),
+               lambda: moe.moe_nvfp4_forward_ex(t["x"], t["logits"], bank, 2, out=t["out"]),
+               lambda: moe.moe_nvfp4_forward_noalloc(t["x"], t["logits"], bank, 2, out=t["out"])):
+        with pytest.raises(ValueError, match=msg):
+            fn()
+
+
+def test_binding_rejects_mismatched_residual_and_route_inputs():
+    import torch
+    bank = _bank()
+    x, lg, out = _cpu((4, 256), torch.bfloat16), _cpu((4, 16), torch.float32), _cpu((4, 256), torch.bfloat16)
+    with pytest.raises(ValueError, match="x_next has shape"):
+        moe.moe_nvfp4_forward_ex(x, lg, bank, 2, out=out, x_next=_cpu((4, 255), torch.bfloat16))
+    with pytest.raises(ValueError, match="logits has dtype"):
+        moe.moe_nvfp4_route(_cpu((4, 16), torch.float16), 2)
+    with pytest.raises(ValueError, match="logits must be a 2-D"):
+        moe.moe_nvfp4_route(_cpu((16,), torch.float32), 2)
+
+
+def test_binding_rejects_mismatched_host_arrays():
+    bank = _bank()
+    x = np.zeros((4, 256), dtype=np.uint16)
+    with pytest.raises(ValueError, match="x_host has shape"):
+        moe.moe_nvfp4_forward_host(np.zeros((4, 128), dtype=np.uint16), np.zeros((4, 16), np.float32), bank, 2)
+    with pytest.raises(ValueError, match="logits_host has shape"):
+        moe.moe_nvfp4_forward_host(x, np.zeros((4, 17), np.float32), bank, 2)
+    with pytest.raises(ValueError, match="out_host must be"):
+        moe.moe_nvfp4_forward_host(x, np.zeros((4, 16), np.float32), bank, 2, out_host=np.zeros((4, 255), np.uint16))
+
+
+def _enc(n=2, out_f=8, in_f=64, mode=0, w=0x20000, dst=0x40000, stride=4096, co=0, so=256, go=320):
+    lib = moe.lib()
+    return lib.moe_nvfp4_encode(ctypes.c_void_p(w), n, out_f, in_f, mode, ctypes.c_void_p(dst), stride, co, so, go,
+                                None)
+
+
+@pytest.mark.parametrize("kw", [dict(n=-1), dict(in_f=24), dict(in_f=0), dict(out_f=0), dict(mode=2),
+                                dict(co=8), dict(stride=4008), dict(go=322), dict(so=16),    # codes overlap scales
+                                dict(go=0), dict(stride=256, n=3)])                            # parts beyond the stride
+def test_encode_rejects_bad_arguments_on_the_host(kw):
+    assert _enc(**kw) == _abi.ERR_INVALID_ARG
+    assert moe.moe_nvfp4_last_error() != ""
+
+
+def test_encode_without_a_device_is_unsupported():
+    assert _enc() == _abi.ERR_UNSUPPORTED
+    assert moe.moe_nvfp4_last_launch_count() == 0

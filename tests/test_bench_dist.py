@@ -95,3 +95,22 @@ def test_committed_traffic_summaries_resolve():
         v = bench.kernel_traffic(d["kind"], d["workload"])
         assert v is None or v == d["dram_bytes_per_launch"]
     assert bench.kernel_traffic("no_such_kernel", "decode_t1") is None
+
+
+def test_default_run_covers_every_full_size_workload():
+    import bench
+    import moe_inputs
+    assert bench.FULL_RUN[0] == bench.HEADLINE
+    assert set(bench.FULL_RUN) == {n for n in moe_inputs.CONFIGS if n != "tiny"}
+    for n in bench.FULL_RUN:
+        assert bench.MIN_STEPS[n] <= bench.DEFAULT_STEPS[n]
+
+
+def test_cpu_baseline_on_a_process_pool_reports_its_cores():
+    import bench
+    import moe_inputs
+    cfg = moe_inputs.CONFIGS["tiny"]
+    one = bench.cpu_oracle_baseline(cfg, budget_s=2.0, max_tokens=4)
+    two = bench.cpu_oracle_baseline(cfg, budget_s=2.0, max_tokens=4, cores=2)
+    assert one["cores"] == 1 and two["cores"] == 2 and one["tokens"] >= 1 and two["tokens"] >= 1
+    assert one["kind"] == two["kind"] == "oracle" and one["value"] > 0 and two["value"] > 0
