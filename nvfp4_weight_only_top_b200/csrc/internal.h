@@ -67,6 +67,16 @@ int launch_combine(const float* y, const float* w, const int32_t* inv, int64_t T
 
 size_t decode_smem_bytes(int K, int xrows, bool gateup);
 
+// Decode of larger batches on the router's groups (up to 8 routed rows of one expert, group_rows
+// 8, singles kept in the groups): persistent gate/up + SwiGLU and down kernels (bulk-TMA stage
+// ring, mma.sync with the group's activations as N = 8).  h [R, I] and y [R, H] f32 in permuted
+// row order, as the combine kernel reads them.
+bool grouped_supported(int H, int I);
+int launch_grouped_gateup(const BankView& bank, const uint16_t* x, int k, const RouteBufs& rb, float* h, int num_sms,
+                          cudaStream_t s);
+int launch_grouped_down(const BankView& bank, const float* h, const RouteBufs& rb, float* y, int num_sms,
+                        cudaStream_t s);
+
 // Decode of a single token: route, gate/up, down and combine in one persistent kernel.  h [k, I]
 // and y [k, H] are f32 scratch; its completion counters come from a library-owned pool of
 // self-clearing counter sets on device dev (the current device).

@@ -161,6 +161,20 @@ moe::BankView view_of(const moe_nvfp4_bank* b) {
   return v;
 }
 
+// Decode kernels for more than one token, for comparisons: MOE_NVFP4_DECODE=grouped takes the
+// grouped kernels for every T > 1 that their shapes allow, =rows the older row and mma.sync group
+// kernels; unset, 2..16 tokens take the few-token kernel and larger batches the grouped kernels.
+enum { kDecodeDefault = 0, kDecodeGrouped = 1, kDecodeRows = 2 };
+int decode_kernel_choice() {
+  static const int v = [] {
+    const char* s = getenv("MOE_NVFP4_DECODE");
+    if (s && strcmp(s, "grouped") == 0) return (int)kDecodeGrouped;
+    if (s && strcmp(s, "rows") == 0) return (int)kDecodeRows;
+    return (int)kDecodeDefault;
+  }();
+  return v;
+}
+
 bool sync_each_kernel() {
   static const bool on = [] {
     const char* s = getenv("MOE_NVFP4_SYNC");
@@ -386,7 +400,7 @@ int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
     t_last_launches = launches;
     return MOE_NVFP4_OK;
   }
-  if (moe::decode_few_supported(H, I, k, (int)T, info.sms)) {
+  if (moe::decode_few_supported(H, I, k, (int)T, info.sms) && decode_kernel_choice() == kDecodeDefault) {
     // A few tokens: the router, then one persistent kernel over one slot per routed row in the
     // router's permutation order (expert order).
     prof_before(MOE_NVFP4_KERNEL_ROUTE, s);
@@ -398,6 +412,30 @@ int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
                                                   reinterpret_cast<float*>(w8 + L.y), rb.ids, rb.w, rb.perm, rb.inv,
                                                   dev, info.sms, s),
                            s, "fused few-token decode", &launches)))
+      return rc;
+    t_last_launches = launches;
+    return MOE_NVFP4_OK;
+  }
+  if (moe::grouped_supported(H, I) && decode_kernel_choice() != kDecodeRows) {
+    // Larger batches: the router's groups of up to 8 rows of one expert (single rows included),
+    // the persistent gate/up and down kernels, then the combine.
+    rb.group_rows = 8;
+    rb.split_singles = 0;
+    float* h = reinterpret_cast<float*>(w8 + L.h);
+    float* y = reinterpret_cast<float*>(w8 + L.y);
+    prof_before(MOE_NVFP4_KERNEL_ROUTE, s);
+    if ((rc = after_launch(moe::launch_route(logits, T, E, k, rb, s), s, "route", &launches))) return rc;
+    prof_before(MOE_NVFP4_KERNEL_DECODE_GATEUP, s);
+    if ((rc = after_launch(moe::launch_grouped_gateup(bv, static_cast<const uint16_t*>(x), k, rb, h, info.sms, s), s,
+                           "grouped gate/up", &launches)))
+      return rc;
+    prof_before(MOE_NVFP4_KERNEL_DECODE_DOWN, s);
+    if ((rc = after_launch(moe::launch_grouped_down(bv, h, rb, y, info.sms, s), s, "grouped down", &launches)))
+      return rc;
+    prof_before(MOE_NVFP4_KERNEL_COMBINE, s);
+    if ((rc = after_launch(moe::launch_combine(y, rb.w, rb.inv, T, k, H, static_cast<const uint16_t*>(x),
+                                               static_cast<uint16_t*>(out), static_cast<uint16_t*>(x_next), s),
+                           s, "combine", &launches)))
       return rc;
     t_last_launches = launches;
     return MOE_NVFP4_OK;
