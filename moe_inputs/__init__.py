@@ -15,6 +15,7 @@ from .gen import (  # noqa: F401
     make_x,
     make_x_wide,
     make_logits,
+    make_act_scales,
     sample_tokens,
     disjoint_routing_logits,
     global_value,

@@ -182,7 +182,7 @@ CONFIGS = {
     "verify24_t16": LayerConfig("verify24_t16", 256, 8, 5120, 2560, 16, 24),
 }
 
-_TAG_X, _TAG_LOGITS, _TAG_PERM, _TAG_SAMPLE, _TAG_ROT = 1, 2, 3, 4, 5
+_TAG_X, _TAG_LOGITS, _TAG_PERM, _TAG_SAMPLE, _TAG_ROT, _TAG_ACT = 1, 2, 3, 4, 5, 6
 
 
 def _rng(seed: int, layer: int, tag: int) -> np.random.Generator:
@@ -211,6 +211,23 @@ def make_x_wide(T: int, H: int, exps, seed: int = 0, heavy: bool = False) -> np.
     e = np.asarray([exps[t % len(exps)] for t in range(T)], dtype=np.float64)
     v = np.clip(base * np.exp2(e)[:, None], -3.0e38, 3.0e38)
     return to_bf16_bits(v)
+
+
+# Largest magnitudes the W4A4 input multipliers are set for: about the row maxima of this
+# generator's x (N(0, 1) rows of a few thousand entries: ~3.8 at H = 5120) and of the mid values
+# its weights give (~3 at H = 5120, I = 2560; the global scale 1/(6 sqrt(H)) keeps them similar
+# across sizes), with some margin.
+ACT_X_RANGE = 4.5
+ACT_H_RANGE = 4.0
+
+
+def make_act_scales(E: int, seed: int = 0, layer: int = 0) -> np.ndarray:
+    """W4A4 input multipliers [E, 2] f32, a stand-in for a release's static activation scales:
+    per expert s_x = ACT_X_RANGE 2^u / 2688 (gate/up input) and s_h = ACT_H_RANGE 2^v / 2688
+    (down input), u and v uniform in [-1/4, 1/4], so that a few of the largest values saturate."""
+    uv = _rng(seed, layer, _TAG_ACT).uniform(-0.25, 0.25, size=(E, 2))
+    rng_ = np.array([ACT_X_RANGE, ACT_H_RANGE])[None, :]
+    return (rng_ * np.exp2(uv) / 2688.0).astype(np.float32)
 
 
 def make_logits(cfg: LayerConfig, seed: int | None = None, layer: int = 0,

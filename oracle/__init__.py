@@ -38,6 +38,7 @@ from .moe import (  # noqa: F401
     permute,
     silu,
     expert_forward,
+    expert_forward_w4a4,
     layer_forward,
     bf16_bits_to_f64,
     round_to_bf16_bits,
@@ -49,5 +50,9 @@ from .encode import (  # noqa: F401
     e4m3_round,
     tensor_global,
     encode_projection,
+    encode_f32,
+    quantize_rows,
+    quantize_static,
+    decode_blocks,
     pack_codes,
 )

@@ -69,12 +69,16 @@ def e4m3_round(v: np.ndarray) -> np.ndarray:
     return _nearest_even_on_grid(v.astype(np.float64), _E4M3_MAG).astype(np.uint8)
 
 
-def tensor_global(w_bits: np.ndarray):
-    """(amax, s2) of a BF16 tensor: amax = max |w|, s2 = f32(amax / 2688) (0 for a zero tensor)."""
-    w = (np.asarray(w_bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+def _global_of(w: np.ndarray):
+    """(amax, s2) of f32 values: amax = max |w|, s2 = f32(amax / 2688) (0 for a zero tensor)."""
     amax = _F32(np.max(np.abs(w))) if w.size else _F32(0.0)
     s2 = _F32(amax / _F32(2688.0)) if amax > 0 else _F32(0.0)
     return amax, s2
+
+
+def tensor_global(w_bits: np.ndarray):
+    """(amax, s2) of a BF16 tensor: amax = max |w|, s2 = f32(amax / 2688) (0 for a zero tensor)."""
+    return _global_of((np.asarray(w_bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32))
 
 
 def encode_projection(w_bits: np.ndarray, global_mode: int = 0):
@@ -84,27 +88,80 @@ def encode_projection(w_bits: np.ndarray, global_mode: int = 0):
     f32): with global_mode 0 the stored global is s2, with 1 it is g = amax.
     """
     w_bits = np.asarray(w_bits, dtype=np.uint16)
-    out_f, in_f = w_bits.shape
+    return encode_f32((w_bits.astype(np.uint32) << 16).view(np.float32), global_mode)
+
+
+def _encode_blocks(w: np.ndarray, s2):
+    """Steps 2 and 3 for f32 values [rows, n] with a positive f32 multiplier s2 per row (an array
+    broadcast over the rows): (codes [rows, n], block scale bytes [rows, n/16])."""
+    rows, n = w.shape
+    blocks = w.reshape(rows, n // 16, 16)
+    s2 = np.asarray(s2, dtype=np.float32).reshape(-1, 1)
+    amax_b = np.max(np.abs(blocks), axis=2).astype(np.float32)                  # [rows, blocks]
+    denom = (_F32(6.0) * s2).astype(np.float32)
+    scales = e4m3_round((amax_b / denom).astype(np.float32))                    # f32 quotient
+    eff = (E4M3_VALUES[scales].astype(np.float32) * s2).astype(np.float32)      # f32 product
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = (blocks / eff[:, :, None]).astype(np.float32)                       # f32 quotient
+    r = np.where(eff[:, :, None] > 0, r, np.copysign(_F32(0.0), blocks))
+    return e2m1_round(r).reshape(rows, n), scales
+
+
+def encode_f32(w: np.ndarray, global_mode: int = 0):
+    """The same encoding of f32 values [out, in] (one tensor)."""
+    w = np.asarray(w, dtype=np.float32)
+    out_f, in_f = w.shape
     assert in_f % 16 == 0
-    w = (w_bits.astype(np.uint32) << 16).view(np.float32)
     assert np.all(np.isfinite(w)), "inputs must be finite"
-    amax, s2 = tensor_global(w_bits)
-    blocks = w.reshape(out_f, in_f // 16, 16)
-    codes = np.zeros((out_f, in_f // 16, 16), dtype=np.uint8)
-    scales = np.zeros((out_f, in_f // 16), dtype=np.uint8)
+    amax, s2 = _global_of(w)
     if s2 > 0:
-        amax_b = np.max(np.abs(blocks), axis=2).astype(np.float32)              # [out, blocks]
-        denom = _F32(_F32(6.0) * s2)
-        scales = e4m3_round((amax_b / denom).astype(np.float32))                # f32 quotient
-        eff = (E4M3_VALUES[scales].astype(np.float32) * s2).astype(np.float32)  # f32 product
-        with np.errstate(divide="ignore", invalid="ignore"):
-            r = (blocks / eff[:, :, None]).astype(np.float32)                   # f32 quotient
-        r = np.where(eff[:, :, None] > 0, r, np.copysign(_F32(0.0), blocks))
-        codes = e2m1_round(r)
+        codes, scales = _encode_blocks(w, np.full(out_f, s2, np.float32))
     else:
-        codes = (np.signbit(blocks).astype(np.uint8) << 3)
+        codes = (np.signbit(w).astype(np.uint8) << 3)
+        scales = np.zeros((out_f, in_f // 16), dtype=np.uint8)
     stored = s2 if global_mode == 0 else amax
-    return codes.reshape(out_f, in_f), scales, _F32(stored)
+    return codes, scales, _F32(stored)
+
+
+def decode_blocks(codes: np.ndarray, scales: np.ndarray, s2) -> np.ndarray:
+    """Exact FP64 values e2m1(code) x e4m3(block scale) x s2 of codes [rows, n] (one value per
+    byte), scale bytes [rows, n/16] and a multiplier per row (or one for all rows)."""
+    codes = np.asarray(codes)
+    rows, n = codes.shape
+    s2 = np.broadcast_to(np.asarray(s2, dtype=np.float32).astype(np.float64).reshape(-1), (rows,))
+    v = E2M1_VALUES[codes].reshape(rows, n // 16, 16) * E4M3_VALUES[np.asarray(scales)][:, :, None]
+    return v.reshape(rows, n) * s2[:, None]
+
+
+def quantize_rows(v: np.ndarray):
+    """Each row of f32 values [rows, n] encoded on its own (the row is the tensor: its amax sets
+    its multiplier s2), returned as (codes [rows, n], scales [rows, n/16], s2 [rows] f32,
+    decoded values [rows, n] in FP64, exact)."""
+    v = np.asarray(v, dtype=np.float32)
+    rows, n = v.shape
+    codes = np.empty((rows, n), np.uint8)
+    scales = np.empty((rows, n // 16), np.uint8)
+    g = np.empty(rows, np.float32)
+    for r in range(rows):
+        c, s, gg = encode_f32(v[r:r + 1], 0)
+        codes[r], scales[r], g[r] = c[0], s[0], gg
+    return codes, scales, g, decode_blocks(codes, scales, g)
+
+
+def quantize_static(v: np.ndarray, s2):
+    """NVFP4 activations with a given multiplier: rows of f32 values [rows, n] (n a multiple of
+    16), each row with its positive f32 multiplier s2 (one per row, or one for all), encoded by
+    steps 2 and 3 above (block scales and codes found from the values, the multiplier fixed in
+    advance -- values beyond 6 x 448 x s2 saturate).  Returns (codes [rows, n], scale bytes
+    [rows, n/16], decoded values [rows, n] in FP64, exact)."""
+    v = np.asarray(v, dtype=np.float32)
+    rows, n = v.shape
+    assert n % 16 == 0
+    assert np.all(np.isfinite(v)), "inputs must be finite"
+    s2 = np.broadcast_to(np.asarray(s2, dtype=np.float32).reshape(-1), (rows,)).copy()
+    assert np.all(s2 > 0) and np.all(np.isfinite(s2)), "multipliers must be positive and finite"
+    codes, scales = _encode_blocks(v, s2)
+    return codes, scales, decode_blocks(codes, scales, s2)
 
 
 def pack_codes(codes: np.ndarray) -> np.ndarray:

@@ -25,6 +25,8 @@ from __future__ import annotations
 
 import numpy as np
 
+from . import encode as _encode
+
 
 def route(logits: np.ndarray, k: int):
     """Top-k experts per token and their softmax weights.
@@ -75,6 +77,22 @@ def expert_forward(Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray, X: np.ndarray
     return A @ Wd.T
 
 
+def expert_forward_w4a4(Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray, X: np.ndarray, s_x, s_h,
+                        H_rows=None):
+    """The expert with NVFP4 activations (W4A4) on rows X [n, H] (exact input values): X is
+    quantized with the multiplier s_x (quantize_static) before the gate and up projections; the
+    mid values h = silu(g) * u, computed in FP64 from the quantized rows, are rounded to f32 (the
+    precision in which they are quantized) and quantized with s_h before the down projection.
+    H_rows [n, I], if given, replaces the f32 h rows (teacher forcing: a test feeds the h that
+    the GPU computed).  Returns (h f32 [n, I] before quantization, Y [n, H] FP64)."""
+    Xq = _encode.quantize_static(np.asarray(X, dtype=np.float32), s_x)[2]
+    G = Xq @ Wg.T
+    U = Xq @ Wu.T
+    h = (silu(G) * U).astype(np.float32) if H_rows is None else np.asarray(H_rows, dtype=np.float32)
+    hq = _encode.quantize_static(h, s_h)[2]
+    return h, hq @ Wd.T
+
+
 def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
@@ -102,13 +120,15 @@ def residual_add(x_bits: np.ndarray, out_bits: np.ndarray) -> np.ndarray:
 
 
 def _expert_job(job):
-    get_weights, e, X = job
+    get_weights, e, X = job[:3]
     Wg, Wu, Wd = get_weights(e)
-    return expert_forward(Wg, Wu, Wd, X)
+    if len(job) == 3:
+        return expert_forward(Wg, Wu, Wd, X)
+    return expert_forward_w4a4(Wg, Wu, Wd, X, *job[3:])
 
 
 def layer_forward(x_bits: np.ndarray, logits: np.ndarray, k: int, get_weights,
-                  tokens=None, want_rows: bool = False, map_fn=map):
+                  tokens=None, want_rows: bool = False, map_fn=map, act_scales=None, h_rows=None):
     """One MoE layer.
 
     x_bits [T, H] BF16 bit patterns, logits [T, E] f32, get_weights(e) -> (Wg, Wu, Wd) FP64.
@@ -117,21 +137,41 @@ def layer_forward(x_bits: np.ndarray, logits: np.ndarray, k: int, get_weights,
     with want_rows also y [len(tokens), k, H], the expert outputs before the combine.
     map_fn maps the per-expert work (decode the record, run the expert on its rows); a process
     pool's map spreads it over host cores without changing any arithmetic.
+    act_scales [E, 2] f32 selects the W4A4 variant (expert_forward_w4a4): a routed row of expert e
+    quantizes its token's x with the multiplier act_scales[e, 0] and its mid values with
+    act_scales[e, 1]; the result then also holds h [len(tokens), k, I] (f32, before
+    quantization).  h_rows [T, k, I] (optional) replaces the mid values of every routed row
+    (teacher forcing).
     """
     T, E = np.asarray(logits).shape
     ids, w = route(logits, k)
     counts, offsets, perm, inv = permute(ids, E)
     toks = np.arange(T) if tokens is None else np.asarray(tokens)
     x = bf16_bits_to_f64(x_bits)
+    w4a4 = act_scales is not None
+    if w4a4:
+        act_scales = np.asarray(act_scales, dtype=np.float32).reshape(E, 2)
     H = x.shape[1]
     y = np.zeros((len(toks), k, H))
+    hs = None
     by_expert: dict = {}
     for ti, t in enumerate(toks):
         for j in range(k):
             by_expert.setdefault(int(ids[t, j]), []).append((ti, int(t), j))
     experts = sorted(by_expert)
     jobs = [(get_weights, e, x[[t for (_, t, _) in by_expert[e]]]) for e in experts]
-    for e, Y in zip(experts, map_fn(_expert_job, jobs)):
+    if w4a4:
+        jobs = [job + (act_scales[e, 0], act_scales[e, 1],
+                       None if h_rows is None else np.stack([h_rows[t, j] for (_, t, j) in by_expert[e]]))
+                for e, job in zip(experts, jobs)]
+    for e, res in zip(experts, map_fn(_expert_job, jobs)):
+        Y = res
+        if w4a4:
+            h, Y = res
+            if hs is None:
+                hs = np.zeros((len(toks), k, h.shape[1]), np.float32)
+            for r, (ti, _, j) in enumerate(by_expert[e]):
+                hs[ti, j] = h[r]
         for r, (ti, _, j) in enumerate(by_expert[e]):
             y[ti, j] = Y[r]
     out = np.zeros((len(toks), H))
@@ -139,6 +179,8 @@ def layer_forward(x_bits: np.ndarray, logits: np.ndarray, k: int, get_weights,
         out += w[toks, j][:, None] * y[:, j]
     res = dict(ids=ids, w=w, counts=counts, offsets=offsets, perm=perm, inv=inv, out=out,
                tokens=toks)
+    if w4a4:
+        res["h"] = hs
     if want_rows:
         res["y"] = y
     return res

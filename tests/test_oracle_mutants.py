@@ -3,7 +3,7 @@
 Every mutant is a one-place edit of the oracle's source -- a dropped term, a wrong sign,
 index, bias or operand order, a swapped role -- executed into a fresh namespace and patched
 over the oracle's public names for the duration of one test.  The pins of
-``test_oracle_nvfp4`` and ``test_oracle_layer`` are then run in order (parametrised cases
+``test_oracle_nvfp4``, ``test_oracle_layer``, ``test_oracle_encode`` and ``test_oracle_w4a4`` are then run in order (parametrised cases
 expanded) until one fails; a mutant that no pin kills fails this test.  Tests of the input
 generator are skipped: they do not look at the oracle.
 """
@@ -21,7 +21,7 @@ import oracle.moe
 import oracle.nvfp4
 import oracle.sources
 
-PIN_MODULES = ("test_oracle_nvfp4", "test_oracle_layer", "test_oracle_encode")
+PIN_MODULES = ("test_oracle_nvfp4", "test_oracle_layer", "test_oracle_encode", "test_oracle_w4a4")
 
 # (label, oracle module, exact source text, replacement)
 MUTANTS = [
@@ -96,7 +96,7 @@ MUTANTS = [
     ("rounding ties go to odd", "encode", "(hi % 2 == 0)", "(hi % 2 == 1)"),
     ("global over 448", "encode", "amax / _F32(2688.0)", "amax / _F32(448.0)"),
     ("global from the first element", "encode", "_F32(np.max(np.abs(w)))", "_F32(np.abs(w).reshape(-1)[0])"),
-    ("block scale not divided by 6", "encode", "denom = _F32(_F32(6.0) * s2)", "denom = s2"),
+    ("block scale not divided by 6", "encode", "denom = (_F32(6.0) * s2)", "denom = (s2)"),
     ("block amax signed", "encode", "np.max(np.abs(blocks), axis=2)", "np.max(blocks, axis=2)"),
     ("block amax along rows", "encode", "amax_b = np.max(np.abs(blocks), axis=2)",
      "amax_b = np.repeat(np.max(np.abs(blocks), axis=(0, 2))[None, :], blocks.shape[0], axis=0)"),
@@ -106,6 +106,20 @@ MUTANTS = [
     ("packed high nibble first", "encode", "(pairs[:, :, 0] | (pairs[:, :, 1] << 4))", "(pairs[:, :, 1] | (pairs[:, :, 0] << 4))"),
     ("effective scale without the global", "encode", "eff = (E4M3_VALUES[scales].astype(np.float32) * s2)",
      "eff = (E4M3_VALUES[scales].astype(np.float32) * 1.0)"),
+    # --- W4A4 (NVFP4 activations)
+    ("W4A4 activations left unquantized", "moe", "Xq = _encode.quantize_static(np.asarray(X, dtype=np.float32), s_x)[2]",
+     "Xq = X"),
+    ("W4A4 mid values left unquantized", "moe", "hq = _encode.quantize_static(h, s_h)[2]", "hq = h.astype(np.float64)"),
+    ("W4A4 down input with the gate/up multiplier", "moe", "act_scales[e, 0], act_scales[e, 1],",
+     "act_scales[e, 0], act_scales[e, 0],"),
+    ("W4A4 multipliers by slot instead of expert", "moe", "act_scales[e, 0], act_scales[e, 1],",
+     "act_scales[0, 0], act_scales[0, 1],"),
+    ("W4A4 teacher forcing ignored", "moe", "None if h_rows is None else np.stack(", "None if True else np.stack("),
+    ("static multiplier of another row", "encode", "(rows,)).copy()\n    assert np.all(s2 > 0)",
+     "(rows,))[::-1].copy()\n    assert np.all(s2 > 0)"),
+    ("static quantizer decodes without the multiplier", "encode", "return v.reshape(rows, n) * s2[:, None]",
+     "return v.reshape(rows, n)"),
+    ("static scale divides by 448", "encode", "denom = (_F32(6.0) * s2)", "denom = (_F32(448.0) * s2)"),
 ]
 
 
