@@ -54,7 +54,7 @@ def parse():
                     help="one workload only (default: decode_t1 as the headline, then every other "
                          "full-size workload in the same line)")
     ap.add_argument("--ncu-case", default=None, choices=["decode_t1_e16", "decode_t16_e16", "decode_t64_e16",
-                                                        "prefill_t4096_e16"],
+                                                        "prefill_t4096_e16", "decode_t64z_e64", "w4a4_t4096_e16"],
                     help="plain layer calls on a small bank for ncu captures (no timing, no graph)")
     ap.add_argument("--calls", type=int, default=4, help="layer calls of --ncu-case")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -362,17 +362,33 @@ def measure(cfg, args, ws, rank, local, steps, warm):
         # holding its activations in host memory would.
         xa, oa = xh.numpy().view(np.uint16), oh.numpy().view(np.uint16)
         la = [t.numpy() for t in lgh]
+        # The C entry point with its arguments built once (as a C caller holds them), and the
+        # Python binding (argument checks and marshalling on every call) for comparison.
+        import ctypes
+        lib = moe.lib()
+        cargs = [(ctypes.c_void_p(xa.ctypes.data), ctypes.c_void_p(l.ctypes.data), cfg.T, ctypes.byref(banks[0]),
+                  cfg.k, ctypes.c_void_p(oa.ctypes.data), ctypes.c_void_p(s.cuda_stream)) for l in la]
         for i in range(min(warm, 20)):
-            moe.moe_nvfp4_forward_host(xa, la[i % nsets], banks[0], cfg.k, out_host=oa)
+            moe.moe_nvfp4_forward_host(xa, la[i % nsets], banks[0], cfg.k, out_host=oa, stream=s)
         barrier(ws)
         torch.cuda.synchronize()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(s)
         for i in range(n_e2e):
-            moe.moe_nvfp4_forward_host(xa, la[i % nsets], banks[0], cfg.k, out_host=oa)
+            rc = lib.moe_nvfp4_forward_host(*cargs[i % nsets])
         f1.record(s)
         torch.cuda.synchronize()
-        api = "moe_nvfp4_forward_host (pinned host x/logits/out, copies and sync inside)"
+        if rc != 0:
+            raise RuntimeError(moe.moe_nvfp4_last_error())
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(s)
+        for i in range(n_e2e):
+            moe.moe_nvfp4_forward_host(xa, la[i % nsets], banks[0], cfg.k, out_host=oa, stream=s)
+        g1.record(s)
+        torch.cuda.synchronize()
+        py_ms = max_over_ranks(ws, g0.elapsed_time(g1))
+        api = ("moe_nvfp4_forward_host, the C entry point (pinned host x/logits/out; one staging copy in, the "
+               "layer, the copy out and the synchronisation inside)")
         h2d = cfg.T * cfg.H * 2 + cfg.T * cfg.E * 4
     else:
         # The stack: every step copies x and the layers' router logits in from pinned host
@@ -406,7 +422,11 @@ def measure(cfg, args, ws, rank, local, steps, warm):
         h2d = cfg.T * cfg.H * 2 + cfg.layers * cfg.T * cfg.E * 4
     e2e_ms = max_over_ranks(ws, f0.elapsed_time(f1))
     e2e = {"value": cfg.T * n_e2e * ws / (e2e_ms / 1000.0), "unit": "tok/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": cfg.T * cfg.H * 2, "steps": n_e2e, "api": api}
+           "d2h_bytes_per_step": cfg.T * cfg.H * 2, "steps": n_e2e, "api": api,
+           "ms_per_step": e2e_ms / n_e2e}
+    if cfg.layers == 1:
+        e2e["python_binding"] = {"value": cfg.T * n_e2e * ws / (py_ms / 1000.0), "unit": "tok/s",
+                                 "ms_per_step": py_ms / n_e2e}
 
     if rank != 0:
         return None
@@ -477,6 +497,89 @@ def measure(cfg, args, ws, rank, local, steps, warm):
     if ck is not None:
         rec["clocks"] = ck
     return rec
+
+
+FP4_OVER_BF16 = 4.0    # nominal dense FP4 / BF16 tensor rates of B200 (9 / 2.25 PFLOP/s)
+
+
+def measure_w4a4(cfg, steps: int, warm: int) -> dict:
+    """The W4A4 variant (NVFP4 activations, tcgen05 kind::mxf4nvf4) on one full-size workload:
+    device time per layer call in a CUDA graph, per-kernel times, and the roofline of its top
+    kernel against the FP4 dense peak (the measured BF16 peak x the nominal FP4/BF16 ratio)."""
+    import torch
+    import nvfp4_weight_only_top_b200 as moe
+    from moe_inputs import device as mdev
+    lay = cfg.layout
+    s = torch.cuda.Stream()
+    torch.cuda.set_stream(s)
+    buf = mdev.bank_tensor(lay, cfg.seed, 0)
+    bank = moe.make_bank(buf.data_ptr(), lay.E, lay.H, lay.I, lay.record_stride, lay.codes_off, lay.scales_off,
+                         lay.global_off, 0)
+    x = torch.from_numpy(moe_inputs.make_x(cfg).view(np.int16)).view(torch.bfloat16).cuda()
+    logits = torch.from_numpy(np.stack([moe_inputs.make_logits(cfg, layer=i) for i in range(2)])).cuda()
+    act = torch.from_numpy(moe_inputs.make_act_scales(cfg.E, seed=cfg.seed)).cuda()
+    out = torch.empty_like(x)
+    wsbuf = torch.empty(moe.moe_nvfp4_workspace_bytes(cfg.T, cfg.E, cfg.k, cfg.H, cfg.I, moe.PATH_PREFILL),
+                        dtype=torch.uint8, device="cuda")
+
+    def step(i):
+        moe.moe_nvfp4_forward_w4a4(x, logits[i % 2], bank, act, cfg.k, out=out, workspace=wsbuf)
+
+    for i in range(warm):
+        step(i)
+    torch.cuda.synchronize()
+    gsteps = max(d for d in range(1, min(GRAPH_STEPS, steps) + 1) if steps % d == 0)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        for i in range(gsteps):
+            step(i)
+    launches = moe.moe_nvfp4_last_launch_count()
+    graph.replay()
+    torch.cuda.synchronize()
+    reps = max(1, steps // gsteps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms_step = e0.elapsed_time(e1) / (reps * gsteps)
+    del graph
+    moe.moe_nvfp4_profile_begin()
+    pgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(pgraph, stream=s):
+        for i in range(gsteps):
+            step(i)
+    for _ in range(3):
+        pgraph.replay()
+    torch.cuda.synchronize()
+    prof = moe.moe_nvfp4_profile_end()
+    del pgraph
+    assert moe.moe_nvfp4_device_status() == 0
+    hbm, tf_burst, tf_sus, peak_kind = load_peaks()
+    R = cfg.T * cfg.k
+    dom = max(("w4a4_gateup", "w4a4_down"), key=lambda k_: prof.get(k_, (0.0, 1))[0])
+    dom_ms = prof[dom][0] / prof[dom][1]
+    flops = 2.0 * R * cfg.H * 2 * cfg.I if dom == "w4a4_gateup" else 2.0 * R * cfg.I * cfg.H
+    achieved = flops / (dom_ms / 1000.0) / 1e12
+    fp4_peak = tf_burst * FP4_OVER_BF16
+    total = sum(v[0] for v in prof.values())
+    layer_tf = 2.0 * R * 3 * cfg.H * cfg.I / (ms_step / 1000.0) / 1e12
+    return {"metric": "MoE-layer tok/s (W4A4: NVFP4 weights and activations)", "value": cfg.T / (ms_step / 1000.0),
+            "unit": "tok/s", "ms_per_step": ms_step, "steps": reps * gsteps, "warmup": warm, "dtype": "e2m1",
+            "config": dict(workload_config(cfg), activations="NVFP4 (per-expert static input multipliers, "
+                           "block scales from the values)"),
+            "layer_tflops": layer_tf, "layer_tflops_frac_fp4": layer_tf / fp4_peak,
+            "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": fp4_peak,
+                         "unit": "TFLOP/s", "frac": achieved / fp4_peak,
+                         "peak_source": f"{peak_kind} dense BF16 cuBLAS burst x {FP4_OVER_BF16:g} (nominal dense "
+                                        "FP4/BF16 ratio); the kernel computes E2M1 x E2M1 with UE4M3 block "
+                                        "scales -> F32 on tcgen05",
+                         "traffic": kernel_traffic(dom, cfg.name), "algorithmic_flops_per_launch": flops,
+                         "avg_launch_us": dom_ms * 1000.0},
+            "kernels_ms_per_step": {k_: v[0] / gsteps for k_, v in prof.items()},
+            "kernel_share": {k_: v[0] / total for k_, v in prof.items()},
+            "gpu_launches": launches * reps * gsteps}
 
 
 def measure_encoder(experts: int = 16, reps: int = 5) -> dict:
@@ -587,33 +690,40 @@ def ncu_case(case: str, calls: int) -> None:
 
     Cases (full-size records H=5120, I=2560, 16 experts resident = 354 MB, above the 126 MB L2):
     decode_t1_e16 (T=1, each call routes to 8 experts the previous call did not use),
-    decode_t16_e16 (T=16), decode_t64_e16 (T=64), prefill_t4096_e16 (T=4096, tensor-core path).
+    decode_t16_e16 (T=16), decode_t64_e16 (T=64), prefill_t4096_e16 (T=4096, tensor-core path);
+    decode_t64z_e64: T=64 with Zipf routing over 64 resident experts (1.4 GB);
+    w4a4_t4096_e16: T=4096 on the W4A4 path (NVFP4 activations).
     """
     import torch
     import nvfp4_weight_only_top_b200 as moe
     from moe_inputs import device as mdev
     T, path = NCU_CASES[case]
-    E, k, H, I = 16, 8, 5120, 2560
+    E, k, H, I = (64 if case.endswith("e64") else 16), 8, 5120, 2560
     lay = moe_inputs.record_layout(E, H, I)
     buf = mdev.bank_tensor(lay, 0, 0)
     bank = moe.make_bank(buf.data_ptr(), E, H, I, lay.record_stride, lay.codes_off, lay.scales_off,
                          lay.global_off, 0)
-    cfg = moe_inputs.LayerConfig(case, E, k, H, I, T)
+    cfg = moe_inputs.LayerConfig(case, E, k, H, I, T, 1, "zipf" if "z_" in case else "normal")
     x = torch.from_numpy(moe_inputs.make_x(cfg).view(np.int16)).view(torch.bfloat16).cuda()
     if T == 1:
         lg = torch.from_numpy(moe_inputs.disjoint_routing_logits(E, k, calls, 2)).cuda()
     else:
         lg = torch.from_numpy(np.stack([moe_inputs.make_logits(cfg, layer=i) for i in range(calls)])).cuda()
     p = moe.PATH_DECODE if path == "decode" else moe.PATH_PREFILL
+    act = torch.from_numpy(moe_inputs.make_act_scales(E)).cuda()
     for i in range(calls):
-        moe.moe_nvfp4_forward_ex(x, lg[i], bank, k, path=p)
+        if path == "w4a4":
+            moe.moe_nvfp4_forward_w4a4(x, lg[i], bank, act, k)
+        else:
+            moe.moe_nvfp4_forward_ex(x, lg[i], bank, k, path=p)
     torch.cuda.synchronize()
     assert moe.moe_nvfp4_device_status() == 0
     print(f"{case}: {calls} calls ok")
 
 
 NCU_CASES = {"decode_t1_e16": (1, "decode"), "decode_t16_e16": (16, "decode"), "decode_t64_e16": (64, "decode"),
-             "prefill_t4096_e16": (4096, "prefill")}
+             "prefill_t4096_e16": (4096, "prefill"), "decode_t64z_e64": (64, "decode"),
+             "w4a4_t4096_e16": (4096, "w4a4")}
 
 
 def main():
@@ -643,6 +753,11 @@ def main():
         recs[name] = measure(cfg, args, ws, rank, local, steps, warm)
         torch.cuda.synchronize()
         torch.cuda.empty_cache()                 # free this workload's banks before the next
+    variants = {}
+    if (not args.config or args.config == "prefill_t8192") and rank == 0:
+        cfg = moe_inputs.CONFIGS["prefill_t8192"]
+        variants["w4a4_prefill_t8192"] = measure_w4a4(cfg, MIN_STEPS["prefill_t8192"] * 2, 3)
+        torch.cuda.empty_cache()
     comps = {}
     if not args.config and rank == 0:
         comps["encode"] = measure_encoder()
@@ -653,6 +768,8 @@ def main():
         line = recs[names[0]]
         if len(names) > 1:
             line["workloads"] = {n: recs[n] for n in names[1:]}
+        if variants:
+            line["variants"] = variants
         if comps:
             line["components"] = comps
         if ws == 1:

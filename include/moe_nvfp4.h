@@ -130,6 +130,46 @@ int moe_nvfp4_forward_ex(const void* x_dev, const float* logits_dev, int64_t T,
                          int32_t path, void* stream);
 
 /*
+ * W4A4 variant of the layer: NVFP4 weights and NVFP4 activations on the block-scaled tensor
+ * cores.  Source: page "Beam-1.0-501B-A23B, EXL3 3-bit ...", section "Fidelity" (the official
+ * NVFP4 release served on Blackwell with FP4 activations, against the weights-only build); page
+ * "Beam 1.0 501B-A23B, streaming pack, NVFP4 experts / MLX 8-bit residents", section "What this
+ * pack holds" (the release's activation scales, which the BF16-activation build leaves unused).
+ *
+ * act_scales_dev [E][2] f32, positive and finite (not checked on the device): for a routed row
+ * of expert e, x is quantized to NVFP4 with act_scales[e][0] as its global multiplier s, and the
+ * mid values h = silu(g) * u, formed in f32, with act_scales[e][1].  Per block of 16 values the
+ * block scale is the E4M3 value nearest to f32(amax / f32(6 s)) and each code the E2M1 value
+ * nearest to f32(v / f32(e4m3 x s)), ties to even, saturating at 448 and 6, with the value's sign
+ * bit (the encoder's rule, moe_nvfp4_encode, with s fixed in advance).  g, u and y accumulate in
+ * f32 on the tensor cores; y is scaled by the weight global and s and combined as in
+ * moe_nvfp4_forward.  The bank's block-scale bytes must be below 0x80 (the tensor cores read them
+ * as unsigned E4M3; every encoder output is); this is not checked.  H and I must be multiples of
+ * 256 (else MOE_NVFP4_ERR_UNSUPPORTED).
+ *
+ * x_next_dev as in moe_nvfp4_forward_ex.  workspace_dev: NULL for the internal workspace, else
+ * at least moe_nvfp4_workspace_bytes(T, E, k, H, I, MOE_NVFP4_PATH_PREFILL) bytes, 256-byte
+ * aligned; afterwards it starts with the routing result as moe_nvfp4_forward_ex describes.
+ * taps (may be NULL, and so may each member; codes and scales come in pairs): the quantized
+ * activations and the mid values of every routed slot t*k + j, written in addition to the
+ * layer's own work, for inspection and tests.  Codes hold two E2M1 values per byte, the lower
+ * index in the low nibble; scales are E4M3 bytes, one per 16 values.  Each must be 16-byte
+ * aligned.
+ */
+typedef struct moe_nvfp4_w4a4_taps {
+  uint8_t* x_codes_dev;   /* [T*k, H/2]  quantized x of the slot                 */
+  uint8_t* x_scales_dev;  /* [T*k, H/16]                                        */
+  float* h_dev;           /* [T*k, I]    f32 mid values before quantization      */
+  uint8_t* h_codes_dev;   /* [T*k, I/2]  quantized mid values                    */
+  uint8_t* h_scales_dev;  /* [T*k, I/16]                                        */
+} moe_nvfp4_w4a4_taps;
+
+int moe_nvfp4_forward_w4a4(const void* x_dev, const float* logits_dev, int64_t T,
+                           const moe_nvfp4_bank* bank, const float* act_scales_dev, int32_t k,
+                           void* out_dev, void* x_next_dev, void* workspace_dev,
+                           size_t workspace_bytes, const moe_nvfp4_w4a4_taps* taps, void* stream);
+
+/*
  * End-to-end call with host tensors: copies x_host [T, H] BF16 and logits_host [T, E] f32 to
  * the device, runs the layer on the resident bank, copies out [T, H] BF16 back to out_host and
  * synchronises `stream` before returning.  Host buffers may be pageable or pinned (pinned
@@ -306,7 +346,10 @@ int moe_nvfp4_last_launch_count(void);
 #define MOE_NVFP4_KERNEL_PREFILL_GATEUP 5
 #define MOE_NVFP4_KERNEL_PREFILL_DOWN   6
 #define MOE_NVFP4_KERNEL_DECODE_FUSED   7  /* single-token decode: the whole layer in one kernel */
-#define MOE_NVFP4_KERNEL_KINDS          8
+#define MOE_NVFP4_KERNEL_W4A4_QUANT     8  /* W4A4: quantize the routed rows of x            */
+#define MOE_NVFP4_KERNEL_W4A4_GATEUP    9
+#define MOE_NVFP4_KERNEL_W4A4_DOWN     10
+#define MOE_NVFP4_KERNEL_KINDS         11
 
 /*
  * Kernel timing for benchmarks.  Between moe_nvfp4_profile_begin() and

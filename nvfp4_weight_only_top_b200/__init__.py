@@ -50,9 +50,9 @@ def _need(name: str, t, dtype, shape, device: bool = True) -> None:
         raise ValueError(f"{name} must be on the current CUDA device (it is on {t.device})")
 
 
-def _layer_args(x, logits, bank: Bank, out, x_next=None, workspace=None) -> int:
-    """Checks the tensors of a layer call against the bank (layouts first, then devices);
-    returns T."""
+def _layer_args(x, logits, bank: Bank, out, x_next=None, workspace=None, extra=()) -> int:
+    """Checks the tensors of a layer call against the bank, and the (name, tensor, dtype, shape)
+    entries of extra (layouts first, then devices); returns T."""
     import torch
     if not isinstance(x, torch.Tensor) or x.dim() != 2:
         raise ValueError("x must be a 2-D torch tensor [T, H]")
@@ -63,6 +63,7 @@ def _layer_args(x, logits, bank: Bank, out, x_next=None, workspace=None) -> int:
         need.append(("x_next", x_next, torch.bfloat16, (T, bank.hidden)))
     if workspace is not None:
         need.append(("workspace", workspace, workspace.dtype, tuple(workspace.shape)))
+    need.extend(extra(T) if callable(extra) else extra)
     for args in need:
         _need(*args, device=False)
     for args in need:
@@ -110,6 +111,39 @@ def moe_nvfp4_forward_ex(x, logits, bank: Bank, k: int, out=None, x_next=None, w
     wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().moe_nvfp4_forward_ex(_ptr(x), _ptr(logits), T, ctypes.byref(bank), k, _ptr(out),
                                       _ptr(x_next), _ptr(workspace), wsb, path, _stream(stream)))
+    return out
+
+
+def moe_nvfp4_forward_w4a4(x, logits, bank: Bank, act_scales, k: int, out=None, x_next=None, workspace=None,
+                           taps: dict | None = None, stream=None):
+    """The W4A4 variant (NVFP4 activations): act_scales [E, 2] f32 device tensor holds each
+    expert's input multipliers of gate/up and of down.  taps, if given, maps any of "x_codes"
+    [T*k, H/2] u8, "x_scales" [T*k, H/16] u8, "h" [T*k, I] f32, "h_codes" [T*k, I/2] u8 and
+    "h_scales" [T*k, I/16] u8 (device tensors) to outputs filled in slot order."""
+    import torch
+    if out is None and isinstance(x, torch.Tensor):
+        out = torch.empty_like(x)
+    H, I = bank.hidden, bank.intermediate
+    for name in (taps or {}):
+        if name not in ("x_codes", "x_scales", "h", "h_codes", "h_scales"):
+            raise ValueError(f"unknown tap {name!r}")
+
+    def extra(T):
+        R = T * k
+        shapes = {"x_codes": (torch.uint8, (R, H // 2)), "x_scales": (torch.uint8, (R, H // 16)),
+                  "h": (torch.float32, (R, I)), "h_codes": (torch.uint8, (R, I // 2)),
+                  "h_scales": (torch.uint8, (R, I // 16))}
+        return [("act_scales", act_scales, torch.float32, (bank.num_experts, 2))] + \
+               [(f"taps[{n!r}]", t, *shapes[n]) for n, t in (taps or {}).items()]
+
+    T = _layer_args(x, logits, bank, out, x_next, workspace, extra)
+    tp = _abi.W4A4Taps()
+    for name, t in (taps or {}).items():
+        setattr(tp, name + "_dev", t.data_ptr())
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().moe_nvfp4_forward_w4a4(_ptr(x), _ptr(logits), T, ctypes.byref(bank), _ptr(act_scales), k,
+                                        _ptr(out), _ptr(x_next), _ptr(workspace), wsb, ctypes.byref(tp),
+                                        _stream(stream)))
     return out
 
 

@@ -44,9 +44,24 @@ class Bank(ctypes.Structure):
 # Every symbol include/moe_nvfp4.h declares, with its argument and return types.
 _vp, _i32, _i64, _sz, _u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint64
 _BANKP = ctypes.POINTER(Bank)
+
+
+class W4A4Taps(ctypes.Structure):
+    """moe_nvfp4_w4a4_taps."""
+    _fields_ = [
+        ("x_codes_dev", ctypes.c_void_p),
+        ("x_scales_dev", ctypes.c_void_p),
+        ("h_dev", ctypes.c_void_p),
+        ("h_codes_dev", ctypes.c_void_p),
+        ("h_scales_dev", ctypes.c_void_p),
+    ]
+
+
+_TAPSP = ctypes.POINTER(W4A4Taps)
 SIGNATURES = {
     "moe_nvfp4_forward": (ctypes.c_int, [_vp, _vp, _i64, _BANKP, _i32, _vp, _vp]),
     "moe_nvfp4_forward_ex": (ctypes.c_int, [_vp, _vp, _i64, _BANKP, _i32, _vp, _vp, _vp, _sz, _i32, _vp]),
+    "moe_nvfp4_forward_w4a4": (ctypes.c_int, [_vp, _vp, _i64, _BANKP, _vp, _i32, _vp, _vp, _vp, _sz, _TAPSP, _vp]),
     "moe_nvfp4_forward_host": (ctypes.c_int, [_vp, _vp, _i64, _BANKP, _i32, _vp, _vp]),
     "moe_nvfp4_forward_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _BANKP, _i32, _vp, _vp]),
     "moe_nvfp4_route": (ctypes.c_int, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -70,7 +85,7 @@ SIGNATURES = {
 }
 
 KERNEL_KINDS = ["route", "decode_gateup", "decode_down", "combine", "prefill_gather",
-                "prefill_gateup", "prefill_down", "decode_fused"]
+                "prefill_gateup", "prefill_down", "decode_fused", "w4a4_quant", "w4a4_gateup", "w4a4_down"]
 
 
 class PackInfo(ctypes.Structure):

@@ -258,6 +258,69 @@ __device__ __forceinline__ uint32_t bf16x8_abs_max_bits(uint4 v) {
 }
 
 // SwiGLU of one pair: silu(g) * u = g / (1 + e^-g) * u, in f32.
+// ---------------------------------------------------------------- NVFP4 encoding
+// Every decision (a scale byte, a code) is taken on an f32 quotient rounded to nearest even.
+
+// E4M3 byte of a non-negative f32, nearest even, saturating at 448.
+__device__ __forceinline__ uint32_t f32_to_e4m3_byte(float v) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
+  return r & 0xFFu;
+}
+
+// Value of an E4M3 byte (exact: every E4M3 value is an f16 value).
+__device__ __forceinline__ float e4m3_byte_to_f32(uint32_t b) {
+  const uint32_t h2 = e4m3x2_to_f16x2((uint16_t)b);
+  float f;
+  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.f32.f16 %0, lo;\n\t}" : "=f"(f) : "r"(h2));
+  return f;
+}
+
+// Eight E2M1 magnitude codes (element i in bits 4i .. 4i+3, bit 4i+3 clear) of non-negative f32
+// values, nearest magnitude, ties to even, saturating at 6.
+__device__ __forceinline__ uint32_t e2m1x8_mag(const float (&a)[8]) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+      : "=r"(r)
+      : "f"(a[0]), "f"(a[1]), "f"(a[2]), "f"(a[3]), "f"(a[4]), "f"(a[5]), "f"(a[6]), "f"(a[7]));
+  return r & 0x77777777u;
+}
+
+// Encodes one block of 16 f32 values with the positive multiplier s2: the block scale is the E4M3
+// value nearest to f32(amax / f32(6 s2)) (ties to even, saturating at 448), each code the E2M1
+// value nearest to f32(v / f32(e4m3 x s2)) (ties to even, saturating at 6) with the sign bit of
+// v; a block whose f32(e4m3 x s2) is 0 keeps only the signs.  Codes of elements 0..7 go to lo,
+// 8..15 to hi (element i at bits 4(i % 8)); returns the scale byte.
+__device__ __forceinline__ uint32_t nvfp4_encode16(const float (&v)[16], float s2, uint32_t& lo, uint32_t& hi) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t scale = f32_to_e4m3_byte(__fdiv_rn(amax, __fmul_rn(6.0f, s2)));
+  const float eff = __fmul_rn(e4m3_byte_to_f32(scale), s2);
+  lo = 0;
+  hi = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    lo |= (__float_as_uint(v[i]) >> 31) << (4 * i + 3);
+    hi |= (__float_as_uint(v[8 + i]) >> 31) << (4 * i + 3);
+  }
+  if (eff > 0.0f) {
+    float r[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r[i] = fabsf(__fdiv_rn(v[i], eff));
+    lo |= e2m1x8_mag(r);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r[i] = fabsf(__fdiv_rn(v[8 + i], eff));
+    hi |= e2m1x8_mag(r);
+  }
+  return scale;
+}
+
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
 // SwiGLU with the hardware exponential and fast division (a few ulp; used where the result is

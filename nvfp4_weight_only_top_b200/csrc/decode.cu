@@ -301,8 +301,7 @@ template <bool GATEUP>
 int launch(const DecodeParams& p, int num_sms, cudaStream_t s) {
   const int bytes = smem_total(p.K, p.xrows);
   if (bytes > kSmemLimit) return -(int)cudaErrorInvalidValue;
-  cudaError_t err = cudaFuncSetAttribute(decode_kernel<GATEUP>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(decode_kernel<GATEUP>), bytes);
   if (err != cudaSuccess) return -(int)err;
   decode_kernel<GATEUP><<<num_sms * kCtasPerSm, kThreads, bytes, s>>>(p);
   err = cudaGetLastError();

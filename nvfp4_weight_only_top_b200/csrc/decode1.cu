@@ -523,7 +523,7 @@ int launch_d1(const D1Params& p, int num_sms, cudaStream_t s) {
       kRing * kStage + H * 2 + 2 * I * 4 + (2 * kRing + 1) * 8 + kMaxRankE * 8 + 5 * kMaxK * 4 + 4 + 4 * kMaxLast +
       4 * 32;
   auto kern = decode1_kernel<UG, UD>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (err != cudaSuccess) return -(int)err;
   // Cooperative launch: all CTAs are resident at once, which the grid barriers need.
   cudaLaunchConfig_t cfg = {};

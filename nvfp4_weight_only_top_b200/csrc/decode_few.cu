@@ -507,7 +507,7 @@ int launch_dn(const DNParams& p, int num_sms, cudaStream_t s) {
   const int smem =
       kRing * kStage + 2 * H * 2 + 2 * I * 4 + (2 * kRing + 1) * 8 + 5 * kMaxSlots * 4 + 4 + 4 * kMaxLast + 4 * 48;
   auto kern = decode_few_kernel<UG, UD>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (err != cudaSuccess) return -(int)err;
   // Cooperative launch: all CTAs are resident at once, which the grid barriers need.
   cudaLaunchConfig_t cfg = {};

@@ -63,36 +63,6 @@ __global__ void __launch_bounds__(kEncThreads) enc_amax_kernel(const uint16_t* w
   }
 }
 
-// E4M3 byte of a non-negative f32, nearest even, saturating at 448.
-__device__ __forceinline__ uint32_t f32_to_e4m3_byte(float v) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
-  return r & 0xFFu;
-}
-
-// Value of an E4M3 byte (exact: every E4M3 value is an f16 value).
-__device__ __forceinline__ float e4m3_byte_to_f32(uint32_t b) {
-  const uint32_t h2 = e4m3x2_to_f16x2((uint16_t)b);
-  float f;
-  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.f32.f16 %0, lo;\n\t}" : "=f"(f) : "r"(h2));
-  return f;
-}
-
-// Eight E2M1 magnitude codes (element i in bits 4i .. 4i+3, bit 4i+3 clear) of non-negative f32
-// values, nearest magnitude, ties to even, saturating at 6.
-__device__ __forceinline__ uint32_t e2m1x8_mag(const float (&a)[8]) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
-      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
-      : "=r"(r)
-      : "f"(a[0]), "f"(a[1]), "f"(a[2]), "f"(a[3]), "f"(a[4]), "f"(a[5]), "f"(a[6]), "f"(a[7]));
-  return r & 0x77777777u;
-}
-
 // Sign bits of eight BF16 values (four packed pairs) at the code positions 4i + 3.
 __device__ __forceinline__ uint32_t e2m1x8_signs(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t p3) {
   const uint32_t p[4] = {p0, p1, p2, p3};

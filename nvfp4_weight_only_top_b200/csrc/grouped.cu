@@ -63,10 +63,17 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_kernel(const GParams p) 
   constexpr int U = GATEUP ? UG : UD;                      // 128-input units per warp and stage
   constexpr int kRowsSt = GATEUP ? 8 : 32;                 // rows per stage (per matrix)
   constexpr int kCodesM = kRowsSt * K / 2, kScalesM = kRowsSt * K / 16;
-  constexpr int kStage = GATEUP ? 2 * (kCodesM + kScalesM) : kCodesM + kScalesM;
+  // A ring slot holds the stage's code rows back to back (each matrix one contiguous copy), then
+  // the scale rows.  (One copy per row with a padded pitch would avoid the 2-way bank conflicts of
+  // the 8 rows a warp reads at once, but 16-32 small copies per stage streamed far slower.)
+  constexpr int kPitch = K / 2;
+  constexpr int kMats = GATEUP ? 2 : 1;
+  constexpr int kScBase = kMats * kCodesM;                 // scales follow the code rows
+  constexpr int kStage = kScBase + kMats * kScalesM;       // bytes of a ring slot
+  constexpr int kTx = kStage;                              // bytes the copies of a stage deliver
   constexpr int kSpg = NOUT / kRowsSt;                     // stages per group
   constexpr int kUStep = GATEUP ? kGW : 4;                 // unit stride between a warp's units
-  static_assert(kStage % 128 == 0, "stage alignment");
+  static_assert(kStage % 128 == 0 && kPitch % 16 == 0, "stage alignment");
 
   extern __shared__ __align__(128) uint8_t smem[];
   float4* red = reinterpret_cast<float4*>(smem + kGRing * kStage);      // [2][kGW][32] partial sums
@@ -89,14 +96,11 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_kernel(const GParams p) 
     const uint8_t* rec = p.bank + (uint64_t)__ldg(&p.groups[g].x) * p.stride;
     const uint64_t r0 = (uint64_t)st * kRowsSt;
     uint8_t* dst = smem + s * kStage;
-    mbar_arrive_expect_tx(&full[s], kStage);
-    bulk_g2s(dst, rec + p.codes_off[0] + r0 * (K / 2), kCodesM, &full[s], pol);
-    if (GATEUP) {
-      bulk_g2s(dst + kCodesM, rec + p.codes_off[1] + r0 * (K / 2), kCodesM, &full[s], pol);
-      bulk_g2s(dst + 2 * kCodesM, rec + p.scales_off[0] + r0 * (K / 16), kScalesM, &full[s], pol);
-      bulk_g2s(dst + 2 * kCodesM + kScalesM, rec + p.scales_off[1] + r0 * (K / 16), kScalesM, &full[s], pol);
-    } else {
-      bulk_g2s(dst + kCodesM, rec + p.scales_off[0] + r0 * (K / 16), kScalesM, &full[s], pol);
+    mbar_arrive_expect_tx(&full[s], kTx);
+#pragma unroll
+    for (int m = 0; m < kMats; ++m) {
+      bulk_g2s(dst + m * kCodesM, rec + p.codes_off[m] + r0 * (K / 2), kCodesM, &full[s], pol);
+      bulk_g2s(dst + kScBase + m * kScalesM, rec + p.scales_off[m] + r0 * (K / 16), kScalesM, &full[s], pol);
     }
   };
   if (threadIdx.x == 0) {
@@ -114,8 +118,7 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_kernel(const GParams p) 
   // 16 tile + gid and 16 tile + gid + 8.
   // (the second row is a fixed distance further: the up matrix, or 8 rows down)
   const int row_a = GATEUP ? gid : 16 * tile + gid;
-  constexpr uint32_t kCodeB = GATEUP ? kCodesM : 8 * (K / 2), kScB = GATEUP ? kScalesM : 8 * (K / 16);
-  constexpr uint32_t kScBase = GATEUP ? 2 * kCodesM : kCodesM;
+  constexpr uint32_t kCodeB = 8 * kPitch, kScB = GATEUP ? kScalesM : 8 * (K / 16);
   uint32_t xr[U][16];                                      // B: row gid's f16 at this thread's K
   int cur_g = -1, q0 = 0, nrows = 0, issued = cnt < kGRing ? cnt : kGRing;
   float gm0 = 0.0f, gm1 = 0.0f;
@@ -207,9 +210,11 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_kernel(const GParams p) 
     // ---- the stage: partial sums over this warp's units
     const int s = q % kGRing;
     if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (q / kGRing) & 1))) ok = false;
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    // four independent accumulators (one per code word of a unit), so that consecutive MMAs do not
+    // wait for each other's results; added at the end
+    float acc[4][4] = {};
     if (ok) {
-      const uint32_t cbase = sbase + s * kStage + row_a * (K / 2) + u0 * 64 + tid4 * 16;
+      const uint32_t cbase = sbase + s * kStage + row_a * kPitch + u0 * 64 + tid4 * 16;
       const uint32_t sbase2 = sbase + s * kStage + kScBase + row_a * (K / 16) + u0 * 8 + tid4 * 2;
 #pragma unroll
       for (int j = 0; j < U; ++j) {
@@ -226,16 +231,18 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_kernel(const GParams p) 
           e2m1x8_to_f16x8(ca[w4], fa);
           e2m1x8_to_f16x8(cb[w4], fb);
           const uint32_t a0[4] = {hmul2(fa[0], sA), hmul2(fb[0], sB), hmul2(fa[1], sA), hmul2(fb[1], sB)};
-          mma_16816(acc, a0, xr[j][4 * w4], xr[j][4 * w4 + 1]);
+          mma_16816(acc[w4], a0, xr[j][4 * w4], xr[j][4 * w4 + 1]);
           const uint32_t a1[4] = {hmul2(fa[2], sA), hmul2(fb[2], sB), hmul2(fa[3], sA), hmul2(fb[3], sB)};
-          mma_16816(acc, a1, xr[j][4 * w4 + 2], xr[j][4 * w4 + 3]);
+          mma_16816(acc[w4], a1, xr[j][4 * w4 + 2], xr[j][4 * w4 + 3]);
         }
       }
       fence_proxy_async_smem();            // the reads above come before the slot's next TMA
     }
     // ---- fixed-order sum of the warps' partials, then the epilogue
     const int buf = q & 1;
-    red[(buf * kGW + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    red[(buf * kGW + warp) * 32 + lane] =
+        make_float4((acc[0][0] + acc[1][0]) + (acc[2][0] + acc[3][0]), (acc[0][1] + acc[1][1]) + (acc[2][1] + acc[3][1]),
+                    (acc[0][2] + acc[1][2]) + (acc[2][2] + acc[3][2]), (acc[0][3] + acc[1][3]) + (acc[2][3] + acc[3][3]));
     if (!ok) *s_abort = 1;
     named_bar_sync(1, 32 * kGW);
     if (*s_abort) break;                                    // every warp leaves together
@@ -297,7 +304,7 @@ int launch_g(const GParams& p, int num_sms, cudaStream_t s) {
   constexpr int kStage = (GATEUP ? 2 : 1) * (kRowsSt * K / 2 + kRowsSt * K / 16);
   const int smem = kGRing * kStage + 2 * kGW * 32 * 16 + kGRing * 8 + kGW * kGRows * 4 + 16;
   auto kern = grouped_kernel<UG, UD, GATEUP>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (err != cudaSuccess) return -(int)err;
   kern<<<num_sms, kGThreads, smem, s>>>(p);
   err = cudaGetLastError();

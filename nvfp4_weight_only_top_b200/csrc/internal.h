@@ -1,6 +1,7 @@
 // Internal launch interface between the C ABI (moe_nvfp4.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -100,19 +101,54 @@ constexpr int kPrefillRows = 256;
 bool prefill_supported(int H, int I);
 // xp [R, H] bf16 = x[perm[r] / k] for every routed row r (expert order).
 int launch_gather(const uint16_t* x, const int32_t* perm, int k, int64_t R, int H, void* xp, cudaStream_t s);
-// hb [R, I] bf16 = silu(xp Wg^T gg) * (xp Wu^T gu).
+// xp [R, H] f16 = x[perm[r] / k] 2^s_r (s_r the row's prescale), colscale[r] = 2^-s_r.
+int launch_gather_f16(const uint16_t* x, const int32_t* perm, int k, int64_t R, int H, void* xp, float* colscale,
+                      cudaStream_t s);
+// hb [R, I] bf16 = silu(xp Wg^T gg) * (xp Wu^T gu); with colscale, xp holds prescaled f16 rows
+// (F16 MMA operands) whose results are multiplied by colscale[r], else bf16 rows.
 // tile_ctr: a counter zeroed before the launch (tiles are handed out dynamically).
-int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const RouteBufs& rb, void* hb,
-                          unsigned* tile_ctr, int num_sms, cudaStream_t s);
+int launch_prefill_gateup(const BankView& bank, const void* xp, const float* colscale, int64_t R, const RouteBufs& rb,
+                          void* hb, unsigned* tile_ctr, int num_sms, cudaStream_t s);
 // y [R, H] f32 = hb Wd^T gd.
 int launch_prefill_down(const BankView& bank, const void* hb, int64_t R, const RouteBufs& rb, float* y,
                         unsigned* tile_ctr, int num_sms, cudaStream_t s);
+
+// W4A4 path (NVFP4 activations on tcgen05 kind::mxf4nvf4), groups of up to kW4A4Rows rows.
+constexpr int kW4A4Rows = 128;
+bool w4a4_supported(int H, int I);
+// Optional outputs of the gate/up kernel in slot order (row perm[r]); NULL members are skipped.
+struct W4A4Taps {
+  float* h;                // [R][I] f32, h before quantization
+  uint8_t* h_codes;        // [R][I/2]
+  uint8_t* h_scales;       // [R][I/16]
+};
+// x[perm[r] / k] quantized with act_scales[2 e] (e the row's expert): codes [R][H/2], scales
+// [R][H/16] in expert order, and in slot order too when tap_codes is not NULL.
+int launch_w4a4_quant_x(const uint16_t* x, const RouteBufs& rb, int k, int64_t R, int H, const float* act_scales,
+                        uint8_t* codes, uint8_t* scales, uint8_t* tap_codes, uint8_t* tap_scales, cudaStream_t s);
+// h = silu(xq Wg^T gg sx) * (xq Wu^T gu sx), quantized with act_scales[2 e + 1] into h_codes [R][I/2]
+// and h_scales [R][I/16] (expert order).  tile_ctr: a counter zeroed before the launch.
+int launch_w4a4_gateup(const BankView& bank, const float* act_scales, const uint8_t* x_codes, const uint8_t* x_scales,
+                       int64_t R, const RouteBufs& rb, uint8_t* h_codes, uint8_t* h_scales, const W4A4Taps& taps,
+                       unsigned* tile_ctr, int num_sms, cudaStream_t s);
+// y [R][H] f32 = hq Wd^T gd sh.
+int launch_w4a4_down(const BankView& bank, const float* act_scales, const uint8_t* h_codes, const uint8_t* h_scales,
+                     int64_t R, const RouteBufs& rb, float* y, unsigned* tile_ctr, int num_sms, cudaStream_t s);
+
+// Tiled tensor map over a byte tensor of the given rank (dims innermost first, strides in bytes
+// of dims 1.., box sizes); 0 or a negative cudaError_t.
+int make_tensor_map(CUtensorMap* map, int rank, const void* base, const uint64_t* dims, const uint64_t* strides,
+                    const uint32_t* box, CUtensorMapSwizzle swizzle);
 
 // NVFP4 encoder: n projections [n, out_f, in_f] of BF16 weights -> codes, block scales and the
 // stored global of projection i at dst + i * stride + {codes_off, scales_off, global_off}.
 // Returns the number of kernels launched or a negative cudaError_t.
 int launch_encode(const uint16_t* w, int64_t n, int out_f, int in_f, int global_mode, uint8_t* dst, uint64_t stride,
                   uint64_t codes_off, uint64_t scales_off, uint64_t global_off, int num_sms, cudaStream_t s);
+
+// Sets a kernel's dynamic shared-memory limit on the current device, once per (kernel, device,
+// size): the attribute call costs host time on every launch otherwise.
+cudaError_t set_smem_limit(const void* kernel, int bytes);
 
 // C-ABI bridge (moe_nvfp4.cu): status and message of the calling host thread, the current
 // device (sm_100 check, SM count).

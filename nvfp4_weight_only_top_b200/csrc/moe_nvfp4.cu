@@ -52,11 +52,13 @@ struct Workspace {
 };
 std::vector<Workspace> g_ws;
 
+// Staging of moe_nvfp4_forward_host: x and the logits go to the device in one copy, through a
+// pinned host buffer (in) into one device buffer (x at 0, logits at the next 256-byte boundary).
 struct HostStage {
-  void* x = nullptr;
-  void* logits = nullptr;
+  void* in_dev = nullptr;      // x | logits
+  void* in_host = nullptr;     // pinned x | logits
   void* out = nullptr;
-  size_t x_bytes = 0, logits_bytes = 0, out_bytes = 0;
+  size_t in_bytes = 0, out_bytes = 0;
 };
 // One record per device, held by pointer so that growing the vector for another device never
 // moves a record a caller is using.
@@ -163,8 +165,9 @@ moe::BankView view_of(const moe_nvfp4_bank* b) {
 
 // Decode kernels for more than one token, for comparisons: MOE_NVFP4_DECODE=grouped takes the
 // grouped kernels for every T > 1 that their shapes allow, =rows the older row and mma.sync group
-// kernels; unset, 2..16 tokens take the few-token kernel and larger batches the grouped kernels.
+// kernels; unset, 2 .. 11 tokens take the few-token kernel and larger batches the grouped kernels.
 enum { kDecodeDefault = 0, kDecodeGrouped = 1, kDecodeRows = 2 };
+constexpr int64_t kGroupedMinT = 12;     // fewest tokens the grouped kernels take by default
 int decode_kernel_choice() {
   static const int v = [] {
     const char* s = getenv("MOE_NVFP4_DECODE");
@@ -325,13 +328,16 @@ int prefill_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
   int launches = 0;
   prof_before(MOE_NVFP4_KERNEL_ROUTE, s);
   if ((rc = after_launch(moe::launch_route(logits, T, E, k, rb, s), s, "route", &launches))) return rc;
+  // Gate/up runs on F16 operands: the gathered rows are prescaled into f16 and the per-row factors
+  // that undo it sit in the unused second half of the h region (h is bf16 [R, I] there).
+  float* colscale = reinterpret_cast<float*>(w8 + L.h + up256((size_t)R * I * 2));
   prof_before(MOE_NVFP4_KERNEL_PREFILL_GATHER, s);
-  if ((rc = after_launch(moe::launch_gather(static_cast<const uint16_t*>(x), rb.perm, k, R, H, xp, s), s, "gather",
-                         &launches)))
+  if ((rc = after_launch(moe::launch_gather_f16(static_cast<const uint16_t*>(x), rb.perm, k, R, H, xp, colscale, s), s,
+                         "gather", &launches)))
     return rc;
   prof_before(MOE_NVFP4_KERNEL_PREFILL_GATEUP, s);
-  if ((rc = after_launch(moe::launch_prefill_gateup(bv, xp, R, rb, hb, tile_ctr, info.sms, s), s, "prefill gate/up",
-                         &launches)))
+  if ((rc = after_launch(moe::launch_prefill_gateup(bv, xp, colscale, R, rb, hb, tile_ctr, info.sms, s), s,
+                         "prefill gate/up", &launches)))
     return rc;
   prof_before(MOE_NVFP4_KERNEL_PREFILL_DOWN, s);
   if ((rc = after_launch(moe::launch_prefill_down(bv, hb, R, rb, y, tile_ctr + 1, info.sms, s), s, "prefill down", &launches)))
@@ -400,7 +406,11 @@ int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
     t_last_launches = launches;
     return MOE_NVFP4_OK;
   }
-  if (moe::decode_few_supported(H, I, k, (int)T, info.sms) && decode_kernel_choice() == kDecodeDefault) {
+  // 2 .. 11 tokens: the few-token kernel (one launch after the router, combine inside); from 12
+  // tokens on the grouped kernels read each expert once per group of 8 rows instead of once per
+  // routed row and are faster (measured: 16 tokens 529 -> 480 us, equal at 12).
+  if (moe::decode_few_supported(H, I, k, (int)T, info.sms) && T < kGroupedMinT &&
+      decode_kernel_choice() == kDecodeDefault) {
     // A few tokens: the router, then one persistent kernel over one slot per routed row in the
     // router's permutation order (expert order).
     prof_before(MOE_NVFP4_KERNEL_ROUTE, s);
@@ -504,11 +514,112 @@ int noalloc_scratch(int dev, void** out) {
   return MOE_NVFP4_OK;
 }
 
+// W4A4 path: route (groups of up to 128 rows) -> quantize x -> tcgen05 kind::mxf4nvf4 gate/up (h
+// quantized in its epilogue) -> down -> combine.  The x codes and scales live in the y region
+// (dead once gate/up has run), the h codes and scales in the h region: the prefill path's
+// workspace.
+int w4a4_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_bank* bank, const float* act_scales,
+              int32_t k, void* out, void* x_next, void* workspace, size_t workspace_bytes,
+              const moe_nvfp4_w4a4_taps* taps, void* stream) {
+  t_last_launches = 0;
+  int rc = check_bank(bank);
+  if (rc) return rc;
+  const int E = bank->num_experts, H = bank->hidden, I = bank->intermediate;
+  if ((rc = check_k_T(T, E, k))) return rc;
+  if (!moe::w4a4_supported(H, I))
+    return fail(MOE_NVFP4_ERR_UNSUPPORTED, "W4A4 path needs H %% 256 == 0 and I %% 256 == 0 (H=%d, I=%d)", H, I);
+  int dev;
+  DeviceInfo info;
+  if ((rc = current_device(&dev, &info))) return rc;
+  if (T == 0) return MOE_NVFP4_OK;
+  if (!x || !logits || !out || !act_scales)
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "x, logits, act_scales and out must not be NULL");
+  if (!aligned(x, 16) || !aligned(logits, 16) || !aligned(out, 16) || !aligned(act_scales, 16) ||
+      (x_next && !aligned(x_next, 16)))
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "x, logits, act_scales, out and x_next must be 16-byte aligned");
+  moe_nvfp4_w4a4_taps tp{};
+  if (taps) tp = *taps;
+  if (!tp.x_codes_dev != !tp.x_scales_dev || !tp.h_codes_dev != !tp.h_scales_dev)
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "taps: codes and scales come in pairs (both set or both NULL)");
+  const void* tps[5] = {tp.x_codes_dev, tp.x_scales_dev, tp.h_dev, tp.h_codes_dev, tp.h_scales_dev};
+  for (const void* q : tps)
+    if (q && !aligned(q, 16)) return fail(MOE_NVFP4_ERR_INVALID_ARG, "taps must be 16-byte aligned");
+  const WsLayout L = ws_layout(T, E, k, H, I, MOE_NVFP4_PATH_PREFILL);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  if (ws) {
+    if (workspace_bytes < L.total)
+      return fail(MOE_NVFP4_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes,
+                  L.total);
+    if (!aligned(ws, 256)) return fail(MOE_NVFP4_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  } else if ((rc = ensure_workspace(dev, L.total, s, &ws))) {
+    return rc;
+  }
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  moe::RouteBufs rb = route_bufs(w8, L);
+  rb.group_rows = moe::kW4A4Rows;
+  rb.split_singles = 0;
+  const moe::BankView bv = view_of(bank);
+  const int64_t R = T * k;
+  uint8_t* xc = w8 + L.y;
+  uint8_t* xs = xc + up256((size_t)R * H / 2);
+  uint8_t* hc = w8 + L.h;
+  uint8_t* hs = hc + up256((size_t)R * I / 2);
+  float* y = reinterpret_cast<float*>(w8 + L.y);
+  unsigned* tile_ctr = reinterpret_cast<unsigned*>(w8 + L.bar);
+  {
+    const cudaError_t e = cudaMemsetAsync(tile_ctr, 0, 2 * sizeof(unsigned), s);
+    if (e != cudaSuccess) return cuda_fail(e, "clear tile counters");
+  }
+  int launches = 0;
+  prof_before(MOE_NVFP4_KERNEL_ROUTE, s);
+  if ((rc = after_launch(moe::launch_route(logits, T, E, k, rb, s), s, "route", &launches))) return rc;
+  prof_before(MOE_NVFP4_KERNEL_W4A4_QUANT, s);
+  if ((rc = after_launch(moe::launch_w4a4_quant_x(static_cast<const uint16_t*>(x), rb, k, R, H, act_scales, xc, xs,
+                                                  tp.x_codes_dev, tp.x_scales_dev, s),
+                         s, "W4A4 quantize x", &launches)))
+    return rc;
+  const moe::W4A4Taps wt{tp.h_dev, tp.h_codes_dev, tp.h_scales_dev};
+  prof_before(MOE_NVFP4_KERNEL_W4A4_GATEUP, s);
+  if ((rc = after_launch(moe::launch_w4a4_gateup(bv, act_scales, xc, xs, R, rb, hc, hs, wt, tile_ctr, info.sms, s), s,
+                         "W4A4 gate/up", &launches)))
+    return rc;
+  prof_before(MOE_NVFP4_KERNEL_W4A4_DOWN, s);
+  if ((rc = after_launch(moe::launch_w4a4_down(bv, act_scales, hc, hs, R, rb, y, tile_ctr + 1, info.sms, s), s,
+                         "W4A4 down", &launches)))
+    return rc;
+  prof_before(MOE_NVFP4_KERNEL_COMBINE, s);
+  if ((rc = after_launch(moe::launch_combine(y, rb.w, rb.inv, T, k, H, static_cast<const uint16_t*>(x),
+                                             static_cast<uint16_t*>(out), static_cast<uint16_t*>(x_next), s),
+                         s, "combine", &launches)))
+    return rc;
+  t_last_launches = launches;
+  return MOE_NVFP4_OK;
+}
+
 }  // namespace
 
 // Bridge for the other translation units of the C ABI (pack.cu): error reporting and the
 // current device's checks, with the same semantics as the entry points here.
 namespace moe {
+
+cudaError_t set_smem_limit(const void* kernel, int bytes) {
+  struct Key {
+    const void* k;
+    int dev, bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Key> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  for (const Key& d : done)
+    if (d.k == kernel && d.dev == dev && d.bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.push_back(Key{kernel, dev, bytes});
+  return e;
+}
 
 int api_fail(int code, const char* msg) { return fail(code, "%s", msg); }
 
@@ -523,6 +634,18 @@ int api_device(int* dev, int* sms) {
 
 }  // namespace moe
 
+// Host inputs of at least this many bytes in page-locked memory are copied to the device directly.
+static constexpr size_t kDirectCopyBytes = (size_t)1 << 20;
+
+static bool is_pinned(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();                       // pageable memory of old runtimes reports an error
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost;
+}
+
 extern "C" {
 
 int moe_nvfp4_forward(const void* x_dev, const float* logits_dev, int64_t T, const moe_nvfp4_bank* bank, int32_t k,
@@ -535,6 +658,14 @@ int moe_nvfp4_forward_ex(const void* x_dev, const float* logits_dev, int64_t T, 
                          int32_t path, void* stream) {
   return forward_impl(x_dev, logits_dev, T, bank, k, out_dev, x_next_dev, workspace_dev, workspace_bytes, path,
                       stream);
+}
+
+int moe_nvfp4_forward_w4a4(const void* x_dev, const float* logits_dev, int64_t T, const moe_nvfp4_bank* bank,
+                           const float* act_scales_dev, int32_t k, void* out_dev, void* x_next_dev,
+                           void* workspace_dev, size_t workspace_bytes, const moe_nvfp4_w4a4_taps* taps,
+                           void* stream) {
+  return w4a4_impl(x_dev, logits_dev, T, bank, act_scales_dev, k, out_dev, x_next_dev, workspace_dev, workspace_bytes,
+                   taps, stream);
 }
 
 int moe_nvfp4_forward_host(const void* x_host, const float* logits_host, int64_t T, const moe_nvfp4_bank* bank,
@@ -555,22 +686,55 @@ int moe_nvfp4_forward_host(const void* x_host, const float* logits_host, int64_t
     st = g_stage[dev].get();
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (xb > st->x_bytes || lb > st->logits_bytes || xb > st->out_bytes) {
+  const size_t lo = up256(xb), ib = lo + lb;          // logits after x, 256-byte aligned
+  if (ib > st->in_bytes || xb > st->out_bytes) {
     cudaError_t e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "synchronise before staging growth");
-    if ((rc = ensure_stage(&st->x, &st->x_bytes, xb))) return rc;
-    if ((rc = ensure_stage(&st->logits, &st->logits_bytes, lb))) return rc;
+    if (ib > st->in_bytes) {
+      if (st->in_host) cudaFreeHost(st->in_host);
+      st->in_host = nullptr;
+      size_t have = st->in_bytes;
+      if ((rc = ensure_stage(&st->in_dev, &have, ib))) return rc;
+      e = cudaHostAlloc(&st->in_host, ib, cudaHostAllocDefault);
+      if (e != cudaSuccess) {
+        st->in_bytes = 0;
+        return cuda_fail(e, "pinned staging allocation");
+      }
+      st->in_bytes = ib;
+    }
     if ((rc = ensure_stage(&st->out, &st->out_bytes, xb))) return rc;
   }
-  cudaError_t e = cudaMemcpyAsync(st->x, x_host, xb, cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return cuda_fail(e, "copy x to device");
-  e = cudaMemcpyAsync(st->logits, logits_host, lb, cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return cuda_fail(e, "copy logits to device");
-  rc = forward_impl(st->x, static_cast<const float*>(st->logits), T, bank, k, st->out, nullptr, nullptr, 0,
+  cudaError_t e;
+  if (ib >= kDirectCopyBytes && is_pinned(x_host) && is_pinned(logits_host)) {
+    // Large inputs already in page-locked memory: two direct copies (a host memcpy into the
+    // staging buffer would cost more than the second copy's launch).
+    e = cudaMemcpyAsync(st->in_dev, x_host, xb, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(static_cast<uint8_t*>(st->in_dev) + lo, logits_host, lb, cudaMemcpyHostToDevice, s);
+  } else {
+    // Small or pageable inputs: one host copy into the pinned staging buffer (free again here:
+    // every call ends with a stream synchronisation), then one copy to the device.
+    memcpy(st->in_host, x_host, xb);
+    memcpy(static_cast<uint8_t*>(st->in_host) + lo, logits_host, lb);
+    e = cudaMemcpyAsync(st->in_dev, st->in_host, ib, cudaMemcpyHostToDevice, s);
+  }
+  if (e != cudaSuccess) {
+    cudaStreamSynchronize(s);
+    return cuda_fail(e, "copy x and logits to device");
+  }
+  const void* xd = st->in_dev;
+  const float* ld = reinterpret_cast<const float*>(static_cast<uint8_t*>(st->in_dev) + lo);
+  rc = forward_impl(xd, ld, T, bank, k, st->out, nullptr, nullptr, 0,
                     MOE_NVFP4_PATH_AUTO, stream);
-  if (rc) return rc;
+  if (rc) {
+    cudaStreamSynchronize(s);                 // the copy from the pinned buffer may still run
+    return rc;
+  }
   e = cudaMemcpyAsync(out_host, st->out, xb, cudaMemcpyDeviceToHost, s);
-  if (e != cudaSuccess) return cuda_fail(e, "copy out to host");
+  if (e != cudaSuccess) {
+    cudaStreamSynchronize(s);
+    return cuda_fail(e, "copy out to host");
+  }
   e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "synchronise");
   return MOE_NVFP4_OK;

@@ -63,6 +63,8 @@ static_assert(kSmemBytes <= 232448, "shared memory per block");
 
 struct PrefillParams {
   const uint8_t* bank;
+  int f16;                 // 1: F16 operands (gate/up: activations prescaled per row, colscale undoes it)
+  const float* colscale;   // f16: per activation row the factor 2^-s of its prescale
   uint64_t stride;
   uint64_t global_off[2];  // global scale of the matrix of M-tile 0 / M-tile 1
   int global_mode;
@@ -211,11 +213,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 bcast_half(h23, true)};
         const uint32_t w[8] = {f.c[mt][0].x, f.c[mt][0].y, f.c[mt][0].z, f.c[mt][0].w,
                                f.c[mt][1].x, f.c[mt][1].y, f.c[mt][1].z, f.c[mt][1].w};
+        if (p.f16) {
+          // F16 operand: E2M1 -> f16 (cvt) times the block scale in f16 -- two instructions per pair
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {                  // word j = K 8j .. 8j+7 = 16-byte chunk j
-          uint32_t e[4];
-          e2m1x8_scaled_to_bf16x8(w[j], sc[j >> 1], e);
-          st_shared_v4(base + ((j ^ (t & 7)) << 4), e[0], e[1], e[2], e[3]);
+          for (int j = 0; j < 8; ++j) {
+            uint32_t e[4];
+            e2m1x8_to_f16x8(w[j], e);
+            st_shared_v4(base + ((j ^ (t & 7)) << 4), hmul2(e[0], sc[j >> 1]), hmul2(e[1], sc[j >> 1]),
+                         hmul2(e[2], sc[j >> 1]), hmul2(e[3], sc[j >> 1]));
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {                // word j = K 8j .. 8j+7 = 16-byte chunk j
+            uint32_t e[4];
+            e2m1x8_scaled_to_bf16x8(w[j], sc[j >> 1], e);
+            st_shared_v4(base + ((j ^ (t & 7)) << 4), e[0], e[1], e[2], e[3]);
+          }
         }
       }
     };
@@ -237,11 +250,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nn = min(32, grp.z - n0);
         if (p.gateup) {
           uint16_t* o = static_cast<uint16_t*>(p.out) + (size_t)(grp.y + n0) * p.out_stride + m * kBM + t;
+          const float* cs = p.colscale + grp.y + n0;     // (f16 operands: undo each row's prescale)
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (j < nn)
+            if (j < nn) {
+              const float c = p.f16 ? __ldg(cs + j) : 1.0f;
               o[(size_t)j * p.out_stride] = (uint16_t)f32_to_bf16_bits(
-                  silu_mul_fast(__uint_as_float(d0[j]) * gm0, __uint_as_float(d1[j]) * gm1));
+                  silu_mul_fast(__uint_as_float(d0[j]) * c * gm0, __uint_as_float(d1[j]) * c * gm1));
+            }
         } else {
           float* o = static_cast<float*>(p.out) + (size_t)(grp.y + n0) * p.out_stride + m * 2 * kBM + t;
 #pragma unroll
@@ -388,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tt < 0) break;
         const int4 grp = __ldg(&p.groups[tt / p.tiles_per_group]);
         const int N = (grp.z + 15) & ~15;
-        const uint32_t idesc = idesc_bf16(kBM, N);
+        const uint32_t idesc = p.f16 ? idesc_f16(kBM, N) : idesc_bf16(kBM, N);
         if (i > 0 && !mbar_wait(d_empty, (i - 1) & 1)) break;
         tc_fence_after();
         for (int c = 0; c < nst; ++c, ++q) {
@@ -424,6 +440,53 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Gathers the routed rows of x (bf16 [T, H]) in expert order into xp as f16 [R, H], each row
+// times the exact power of two 2^s that puts its largest magnitude in [2^9, 2^10) (the decode
+// kernels' prescale; every BF16 value down to 2^-23 of the row's maximum is exact in f16), and
+// writes colscale[r] = 2^-s.  One CTA of 128 threads per routed row: the maximum first, then the
+// conversion.
+constexpr int kGatherThreads = 128;
+constexpr int kGatherPer = 8;          // 16-byte chunks per thread (H <= 8192)
+__global__ void __launch_bounds__(kGatherThreads) gather_f16_kernel(const uint16_t* __restrict__ x,
+                                                                   const int32_t* __restrict__ perm, int k, int H,
+                                                                   uint16_t* __restrict__ xp,
+                                                                   float* __restrict__ colscale) {
+  const int64_t r = blockIdx.x;
+  const int t = perm[r] / k;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+  const int n8 = H / 8;
+  uint4 v[kGatherPer];
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < kGatherPer; ++i) {
+    const int c = (int)threadIdx.x + i * kGatherThreads;
+    if (c < n8) {
+      v[i] = __ldg(src + c);
+      m = max(m, bf16x8_abs_max_bits(v[i]));
+    }
+  }
+  __shared__ uint32_t s_m[kGatherThreads / 32];
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  if ((threadIdx.x & 31) == 0) s_m[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = max(max(s_m[0], s_m[1]), max(s_m[2], s_m[3]));
+  const int sh = prescale_shift_bf16(m);
+  const float f = exp2_int(sh);
+  uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * H);
+#pragma unroll
+  for (int i = 0; i < kGatherPer; ++i) {
+    const int c = (int)threadIdx.x + i * kGatherThreads;
+    if (c < n8) {
+      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) o[j] = pack_f16x2(bf16_bits_to_f32(w[j] & 0xFFFFu) * f, bf16_bits_to_f32(w[j] >> 16) * f);
+      dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+  if (threadIdx.x == 0) colscale[r] = exp2_int(-sh);
+}
+
 // Gathers the routed rows of x (bf16 [T, H]) in expert order into xp (bf16 [R, H]).
 __global__ void gather_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int k, int64_t R,
                               int H, uint16_t* __restrict__ xp) {
@@ -452,7 +515,8 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Tensor map over a row-major bf16 matrix [rows, cols]: boxes of 64 columns x 64 rows, 128B swizzle.
+// Tensor map over a row-major 16-bit matrix [rows, cols]: boxes of 64 columns x 64 rows, 128B
+// swizzle (the copy moves bytes; bf16 and f16 rows use the same map).
 int make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int cols) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return -(int)cudaErrorNotSupported;
@@ -482,7 +546,7 @@ int make_bank_map(CUtensorMap* map, const BankView& bank, uint64_t off, int rows
 }
 
 int launch_prefill(const PrefillParams& p, const Maps& maps, int num_sms, cudaStream_t s) {
-  cudaError_t err = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(prefill_kernel), kSmemBytes);
   if (err != cudaSuccess) return -(int)err;
   prefill_kernel<<<num_sms, kThreads, kSmemBytes, s>>>(maps, p);
   err = cudaGetLastError();
@@ -503,7 +567,34 @@ int make_weight_maps(Maps* maps, const BankView& bank, int proj0, int proj1, int
 
 }  // namespace
 
+int make_tensor_map(CUtensorMap* map, int rank, const void* base, const uint64_t* dims, const uint64_t* strides,
+                    const uint32_t* box, CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return -(int)cudaErrorNotSupported;
+  if (rank < 1 || rank > 5) return -(int)cudaErrorInvalidValue;
+  cuuint64_t d[5], st[4];
+  cuuint32_t b[5], e[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    e[i] = 1;
+    if (i + 1 < rank) st[i] = strides[i];
+  }
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void*>(base), d, st, b, e,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -(int)cudaErrorInvalidValue;
+}
+
 bool prefill_supported(int H, int I) { return H % 256 == 0 && I % 256 == 0; }
+
+int launch_gather_f16(const uint16_t* x, const int32_t* perm, int k, int64_t R, int H, void* xp, float* colscale,
+                      cudaStream_t s) {
+  if (H / 8 > kGatherPer * kGatherThreads) return -(int)cudaErrorInvalidValue;
+  gather_f16_kernel<<<(unsigned)R, kGatherThreads, 0, s>>>(x, perm, k, H, static_cast<uint16_t*>(xp), colscale);
+  const cudaError_t err = cudaGetLastError();
+  return err == cudaSuccess ? 1 : -(int)err;
+}
 
 int launch_gather(const uint16_t* x, const int32_t* perm, int k, int64_t R, int H, void* xp, cudaStream_t s) {
   const int64_t n = R * (H / 8);
@@ -512,8 +603,8 @@ int launch_gather(const uint16_t* x, const int32_t* perm, int k, int64_t R, int 
   return err == cudaSuccess ? 1 : -(int)err;
 }
 
-int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const RouteBufs& rb, void* hb,
-                          unsigned* tile_ctr, int num_sms, cudaStream_t s) {
+int launch_prefill_gateup(const BankView& bank, const void* xp, const float* colscale, int64_t R, const RouteBufs& rb,
+                          void* hb, unsigned* tile_ctr, int num_sms, cudaStream_t s) {
   Maps maps;
   int rc = make_rows_map(&maps.x, xp, R, bank.H);
   if (!rc) rc = make_weight_maps(&maps, bank, 0, 1, bank.I, bank.H);
@@ -527,6 +618,8 @@ int launch_prefill_gateup(const BankView& bank, const void* xp, int64_t R, const
   p.K = bank.H;
   p.tiles_per_group = bank.I / kBM;
   p.gateup = 1;
+  p.f16 = colscale != nullptr;
+  p.colscale = colscale;
   p.groups = rb.groups;
   p.ngroups = rb.ngroups;
   p.tile_ctr = tile_ctr;

@@ -288,8 +288,7 @@ int units_per_lane(int K) { return (K % 512 == 0 && K / 512 <= 10) ? K / 512 : 0
 template <int UPL, int NX, int DEPTH, int WARPS, bool GATEUP>
 cudaError_t launch_one(const RowParams& p, int num_sms, cudaStream_t s) {
   const int smem = WARPS * NX * 4 * 32 * 16;
-  cudaError_t err = cudaFuncSetAttribute(rows_kernel<UPL, NX, DEPTH, WARPS, GATEUP>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(rows_kernel<UPL, NX, DEPTH, WARPS, GATEUP>), smem);
   if (err != cudaSuccess) return err;
   rows_kernel<UPL, NX, DEPTH, WARPS, GATEUP><<<num_sms, 32 * WARPS, smem, s>>>(p);
   return cudaGetLastError();

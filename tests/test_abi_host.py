@@ -227,3 +227,31 @@ def test_encode_rejects_bad_arguments_on_the_host(kw):
 def test_encode_without_a_device_is_unsupported():
     assert _enc() == _abi.ERR_UNSUPPORTED
     assert moe.moe_nvfp4_last_launch_count() == 0
+
+
+def _fwd_w4a4(bank, T=4, k=2, taps=None):
+    lib = moe.lib()
+    return lib.moe_nvfp4_forward_w4a4(ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000), T, ctypes.byref(bank),
+                                      ctypes.c_void_p(0x50000), k, ctypes.c_void_p(0x40000), None, None, 0, taps, None)
+
+
+def test_w4a4_host_validation_runs_before_the_device():
+    lib = moe.lib()
+    assert _fwd_w4a4(_bank(), k=0) == _abi.ERR_INVALID_ARG
+    assert _fwd_w4a4(_bank(), T=-1) == _abi.ERR_INVALID_ARG
+    for H, I in ((384, 256), (256, 128)):
+        lay = moe_inputs.record_layout(16, H, I)
+        b = _bank(hidden=H, intermediate=I, record_stride=lay.record_stride, codes_off=lay.codes_off,
+                  scales_off=lay.scales_off, global_off=lay.global_off)
+        assert _fwd_w4a4(b) == _abi.ERR_UNSUPPORTED
+        assert "W4A4 path needs H % 256 == 0 and I % 256 == 0" in lib.moe_nvfp4_last_error().decode()
+
+
+def test_w4a4_binding_checks_scales_and_taps():
+    import torch
+    bank = _bank()
+    x, lg, out = _cpu((4, 256), torch.bfloat16), _cpu((4, 16), torch.float32), _cpu((4, 256), torch.bfloat16)
+    with pytest.raises(ValueError, match="act_scales has shape"):
+        moe.moe_nvfp4_forward_w4a4(x, lg, bank, _cpu((16,), torch.float32), 2, out=out)
+    with pytest.raises(ValueError, match="act_scales has dtype"):
+        moe.moe_nvfp4_forward_w4a4(x, lg, bank, _cpu((16, 2), torch.float16), 2, out=out)
