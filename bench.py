@@ -387,6 +387,33 @@ def measure(cfg, args, ws, rank, local, steps, warm):
         g1.record(s)
         torch.cuda.synchronize()
         py_ms = max_over_ranks(ws, g0.elapsed_time(g1))
+        # Where the host call's time goes: the same three steps issued one by one on device buffers
+        # (copy in, one layer call, copy out), each bracketed by events, and the host's wall time
+        # for the whole sequence including the synchronisation.
+        import time
+        xd, ld, od = torch.empty_like(x), torch.empty_like(logits[0]), torch.empty_like(out)
+        bev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        parts = {"h2d_us": [], "layer_us": [], "d2h_us": [], "wall_us": []}
+        for i in range(min(n_e2e, 200)):
+            w0 = time.perf_counter()
+            bev[0].record(s)
+            xd.copy_(xh.view(torch.bfloat16), non_blocking=True)
+            ld.copy_(lgh[i % nsets], non_blocking=True)
+            bev[1].record(s)
+            moe.moe_nvfp4_forward_ex(xd, ld, banks[0], cfg.k, out=od, workspace=wsbuf, stream=s)
+            bev[2].record(s)
+            oh.view(torch.bfloat16).copy_(od, non_blocking=True)
+            bev[3].record(s)
+            s.synchronize()
+            parts["wall_us"].append((time.perf_counter() - w0) * 1e6)
+            parts["h2d_us"].append(bev[0].elapsed_time(bev[1]) * 1e3)
+            parts["layer_us"].append(bev[1].elapsed_time(bev[2]) * 1e3)
+            parts["d2h_us"].append(bev[2].elapsed_time(bev[3]) * 1e3)
+        breakdown = {k_: float(np.median(v)) for k_, v in parts.items()}
+        breakdown["note"] = ("medians of the copy in, one layer call and the copy out issued one by one on device "
+                             "buffers (event-timed), and the host wall time of the sequence with its "
+                             "synchronisation; the graph-timed step is the device time per layer when calls run "
+                             "back to back")
         api = ("moe_nvfp4_forward_host, the C entry point (pinned host x/logits/out; one staging copy in, the "
                "layer, the copy out and the synchronisation inside)")
         h2d = cfg.T * cfg.H * 2 + cfg.T * cfg.E * 4
@@ -427,6 +454,7 @@ def measure(cfg, args, ws, rank, local, steps, warm):
     if cfg.layers == 1:
         e2e["python_binding"] = {"value": cfg.T * n_e2e * ws / (py_ms / 1000.0), "unit": "tok/s",
                                  "ms_per_step": py_ms / n_e2e}
+        e2e["breakdown"] = breakdown
 
     if rank != 0:
         return None

@@ -405,6 +405,14 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int x, i
       : "memory");
 }
 
+// Prefetch of box (x, y, z) of a 3-D tensor map into L2 (no shared memory, no completion): issued
+// a few stages ahead of the load of the same box, so that the load finds its bytes in L2.
+__device__ __forceinline__ void tma_prefetch_3d(const void* map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map), "r"(x), "r"(y),
+               "r"(z)
+               : "memory");
+}
+
 // Shared-memory matrix descriptor (sm_100) for a K-major operand stored in 128-byte swizzle
 // atoms (8 rows x 128 B, 1024 B apart): start address, leading offset 1 (unused when
 // swizzled), stride offset 1024 B, descriptor version 1, layout SWIZZLE_128B.

@@ -113,6 +113,15 @@ int launch_prefill_gateup(const BankView& bank, const void* xp, const float* col
 int launch_prefill_down(const BankView& bank, const void* hb, int64_t R, const RouteBufs& rb, float* y,
                         unsigned* tile_ctr, int num_sms, cudaStream_t s);
 
+// Prefill path on CTA pairs (tcgen05 cta_group::2, M = 256): the same outputs as
+// launch_prefill_gateup / launch_prefill_down.  prefill2_pairs: pairs resident at once (0: not
+// available on this device).
+int prefill2_pairs(int num_sms);
+int launch_prefill2_gateup(const BankView& bank, const void* xp, const float* colscale, int64_t R,
+                           const RouteBufs& rb, void* hb, int pairs, cudaStream_t s);
+int launch_prefill2_down(const BankView& bank, const void* hb, int64_t R, const RouteBufs& rb, float* y, int pairs,
+                         cudaStream_t s);
+
 // W4A4 path (NVFP4 activations on tcgen05 kind::mxf4nvf4), groups of up to kW4A4Rows rows.
 constexpr int kW4A4Rows = 128;
 bool w4a4_supported(int H, int I);

@@ -54,11 +54,30 @@ std::vector<Workspace> g_ws;
 
 // Staging of moe_nvfp4_forward_host: x and the logits go to the device in one copy, through a
 // pinned host buffer (in) into one device buffer (x at 0, logits at the next 256-byte boundary).
+// A captured small host call (copy in, layer, copy out) for one (T, k, bank) and the staging and
+// workspace buffers it was captured with; replayed with one graph launch.
+struct HostGraph {
+  int64_t T = 0;
+  int k = 0;
+  moe_nvfp4_bank bank{};
+  const void* in_dev = nullptr;
+  const void* in_host = nullptr;
+  const void* out = nullptr;
+  const void* out_host = nullptr;
+  const void* ws = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  int launches = 0;
+  uint64_t used = 0;
+};
 struct HostStage {
   void* in_dev = nullptr;      // x | logits
   void* in_host = nullptr;     // pinned x | logits
   void* out = nullptr;
-  size_t in_bytes = 0, out_bytes = 0;
+  void* out_host = nullptr;    // pinned out (graph replays)
+  size_t in_bytes = 0, out_bytes = 0, out_host_bytes = 0;
+  cudaStream_t capture = nullptr;
+  std::vector<HostGraph> graphs;
+  uint64_t tick = 0;
 };
 // One record per device, held by pointer so that growing the vector for another device never
 // moves a record a caller is using.
@@ -174,6 +193,16 @@ int decode_kernel_choice() {
     if (s && strcmp(s, "grouped") == 0) return (int)kDecodeGrouped;
     if (s && strcmp(s, "rows") == 0) return (int)kDecodeRows;
     return (int)kDecodeDefault;
+  }();
+  return v;
+}
+
+// Prefill kernel: the single-CTA kernel; MOE_NVFP4_PREFILL=pair selects the CTA-pair kernel
+// (cta_group::2), which computes the same result (see prefill2.cu).
+bool prefill_pair_kernel() {
+  static const bool v = [] {
+    const char* s = getenv("MOE_NVFP4_PREFILL");
+    return s && strcmp(s, "pair") == 0;
   }();
   return v;
 }
@@ -335,13 +364,15 @@ int prefill_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
   if ((rc = after_launch(moe::launch_gather_f16(static_cast<const uint16_t*>(x), rb.perm, k, R, H, xp, colscale, s), s,
                          "gather", &launches)))
     return rc;
+  const int pairs = prefill_pair_kernel() ? moe::prefill2_pairs(info.sms) : 0;
   prof_before(MOE_NVFP4_KERNEL_PREFILL_GATEUP, s);
-  if ((rc = after_launch(moe::launch_prefill_gateup(bv, xp, colscale, R, rb, hb, tile_ctr, info.sms, s), s,
-                         "prefill gate/up", &launches)))
-    return rc;
+  rc = pairs > 0 ? moe::launch_prefill2_gateup(bv, xp, colscale, R, rb, hb, pairs, s)
+                 : moe::launch_prefill_gateup(bv, xp, colscale, R, rb, hb, tile_ctr, info.sms, s);
+  if ((rc = after_launch(rc, s, "prefill gate/up", &launches))) return rc;
   prof_before(MOE_NVFP4_KERNEL_PREFILL_DOWN, s);
-  if ((rc = after_launch(moe::launch_prefill_down(bv, hb, R, rb, y, tile_ctr + 1, info.sms, s), s, "prefill down", &launches)))
-    return rc;
+  rc = pairs > 0 ? moe::launch_prefill2_down(bv, hb, R, rb, y, pairs, s)
+                 : moe::launch_prefill_down(bv, hb, R, rb, y, tile_ctr + 1, info.sms, s);
+  if ((rc = after_launch(rc, s, "prefill down", &launches))) return rc;
   prof_before(MOE_NVFP4_KERNEL_COMBINE, s);
   if ((rc = after_launch(moe::launch_combine(y, rb.w, rb.inv, T, k, H, static_cast<const uint16_t*>(x),
                                              static_cast<uint16_t*>(out), static_cast<uint16_t*>(x_next), s),
@@ -668,6 +699,81 @@ int moe_nvfp4_forward_w4a4(const void* x_dev, const float* logits_dev, int64_t T
                    taps, stream);
 }
 
+// Host calls whose inputs fit in this many bytes replay a captured graph.
+static constexpr size_t kGraphMaxBytes = (size_t)64 << 10;
+static constexpr size_t kMaxHostGraphs = 8;
+
+// The graph of a small host call: H2D copy of the staged x | logits, the layer on the internal
+// workspace, D2H copy into the pinned out staging buffer.  Captured on a library stream (the
+// caller's may be the legacy stream, which cannot capture), launched on the caller's.
+// With build false, only looks the graph up (*out_g = NULL when there is none).
+static int host_graph(HostStage* st, int dev, int64_t T, const moe_nvfp4_bank* bank, int32_t k, size_t ib,
+                      size_t lo, size_t xb, bool build, HostGraph** out_g) {
+  const int E = bank->num_experts, H = bank->hidden, I = bank->intermediate;
+  void* ws = nullptr;
+  int rc;
+  const size_t need = ws_layout(T, E, k, H, I, resolve_path(MOE_NVFP4_PATH_AUTO, T, k, E, H, I)).total;
+  if (!st->capture) {
+    const cudaError_t e = cudaStreamCreateWithFlags(&st->capture, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return cuda_fail(e, "capture stream");
+  }
+  if ((rc = ensure_workspace(dev, need, st->capture, &ws))) return rc;
+  for (HostGraph& g : st->graphs)
+    if (g.T == T && g.k == k && !memcmp(&g.bank, bank, sizeof(*bank)) && g.in_dev == st->in_dev && g.in_host == st->in_host &&
+        g.out == st->out && g.out_host == st->out_host && g.ws == ws) {
+      g.used = ++st->tick;
+      *out_g = &g;
+      return MOE_NVFP4_OK;
+    }
+  *out_g = nullptr;
+  if (!build) return MOE_NVFP4_OK;
+  cudaStream_t c = st->capture;
+  cudaError_t e = cudaStreamBeginCapture(c, cudaStreamCaptureModeThreadLocal);
+  if (e != cudaSuccess) return cuda_fail(e, "begin capture");
+  e = cudaMemcpyAsync(st->in_dev, st->in_host, ib, cudaMemcpyHostToDevice, c);
+  rc = e != cudaSuccess ? cuda_fail(e, "capture copy in") : MOE_NVFP4_OK;
+  if (!rc)
+    rc = forward_impl(st->in_dev, reinterpret_cast<const float*>(static_cast<uint8_t*>(st->in_dev) + lo), T, bank, k,
+                      st->out, nullptr, nullptr, 0, MOE_NVFP4_PATH_AUTO, c);
+  const int launches = t_last_launches;
+  if (!rc) {
+    e = cudaMemcpyAsync(st->out_host, st->out, xb, cudaMemcpyDeviceToHost, c);
+    if (e != cudaSuccess) rc = cuda_fail(e, "capture copy out");
+  }
+  cudaGraph_t graph = nullptr;
+  e = cudaStreamEndCapture(c, &graph);
+  if (!rc && e != cudaSuccess) rc = cuda_fail(e, "end capture");
+  cudaGraphExec_t exec = nullptr;
+  if (!rc) {
+    e = cudaGraphInstantiate(&exec, graph, 0);
+    if (e != cudaSuccess) rc = cuda_fail(e, "instantiate");
+  }
+  if (graph) cudaGraphDestroy(graph);
+  if (rc) return rc;
+  if (st->graphs.size() >= kMaxHostGraphs) {
+    size_t lru = 0;
+    for (size_t i = 1; i < st->graphs.size(); ++i)
+      if (st->graphs[i].used < st->graphs[lru].used) lru = i;
+    cudaGraphExecDestroy(st->graphs[lru].exec);
+    st->graphs.erase(st->graphs.begin() + lru);
+  }
+  HostGraph g;
+  g.T = T;
+  g.k = k;
+  g.bank = *bank;
+  g.in_dev = st->in_dev;
+  g.in_host = st->in_host;
+  g.out = st->out;
+  g.out_host = st->out_host;
+  g.ws = ws;
+  g.exec = exec;
+  g.launches = launches;
+  g.used = ++st->tick;
+  st->graphs.push_back(g);
+  *out_g = &st->graphs.back();
+  return MOE_NVFP4_OK;
+}
+
 int moe_nvfp4_forward_host(const void* x_host, const float* logits_host, int64_t T, const moe_nvfp4_bank* bank,
                            int32_t k, void* out_host, void* stream) {
   int rc = check_bank(bank);
@@ -703,6 +809,49 @@ int moe_nvfp4_forward_host(const void* x_host, const float* logits_host, int64_t
       st->in_bytes = ib;
     }
     if ((rc = ensure_stage(&st->out, &st->out_bytes, xb))) return rc;
+  }
+  if (ib <= kGraphMaxBytes && !t_prof_on && !sync_each_kernel()) {
+    // Small call: stage x and the logits, replay (or capture once) copy in + layer + copy out.
+    if (xb > st->out_host_bytes) {
+      cudaError_t e = cudaStreamSynchronize(s);
+      if (e != cudaSuccess) return cuda_fail(e, "synchronise before staging growth");
+      if (st->out_host) cudaFreeHost(st->out_host);
+      st->out_host = nullptr;
+      st->out_host_bytes = 0;
+      e = cudaHostAlloc(&st->out_host, kGraphMaxBytes, cudaHostAllocDefault);
+      if (e != cudaSuccess) return cuda_fail(e, "pinned staging allocation");
+      st->out_host_bytes = kGraphMaxBytes;
+    }
+    HostGraph* g = nullptr;
+    if ((rc = host_graph(st, dev, T, bank, k, ib, lo, xb, false, &g))) return rc;
+    memcpy(st->in_host, x_host, xb);
+    memcpy(static_cast<uint8_t*>(st->in_host) + lo, logits_host, lb);
+    cudaError_t e;
+    int launches;
+    if (g) {
+      e = cudaGraphLaunch(g->exec, s);
+      launches = g->launches;
+    } else {
+      // First call of this kind: run it eagerly (every kernel attribute is then set outside any
+      // capture), and capture the graph for the next calls once it has completed.
+      e = cudaMemcpyAsync(st->in_dev, st->in_host, ib, cudaMemcpyHostToDevice, s);
+      if (e == cudaSuccess) {
+        rc = forward_impl(st->in_dev, reinterpret_cast<const float*>(static_cast<uint8_t*>(st->in_dev) + lo), T,
+                          bank, k, st->out, nullptr, nullptr, 0, MOE_NVFP4_PATH_AUTO, stream);
+        if (rc) {
+          cudaStreamSynchronize(s);
+          return rc;
+        }
+        e = cudaMemcpyAsync(st->out_host, st->out, xb, cudaMemcpyDeviceToHost, s);
+      }
+      launches = t_last_launches;
+    }
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "host call");
+    memcpy(out_host, st->out_host, xb);
+    if (!g && (rc = host_graph(st, dev, T, bank, k, ib, lo, xb, true, &g))) return rc;
+    t_last_launches = launches;
+    return MOE_NVFP4_OK;
   }
   cudaError_t e;
   if (ib >= kDirectCopyBytes && is_pinned(x_host) && is_pinned(logits_host)) {

@@ -44,6 +44,7 @@ constexpr int kKC = 64;                        // K per stage: one 128-byte swiz
 constexpr int kStages = 3;                     // operand stages (A and B, bf16)
 constexpr int kWStages = 3;                    // raw code stages
 constexpr int kSStages = 2;                    // raw scale stages (4 operand stages each)
+constexpr int kPrefetch = 8;                   // stages of raw codes prefetched into L2 ahead of their load
 constexpr int kMaxN = 256;
 constexpr int kBoxRows = 64;                   // activation rows per TMA box
 constexpr int kThreads = 32 * 7;
@@ -361,6 +362,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         int g, m;
         cur.at(tt, g, m);
         const int e = __ldg(&p.groups[g].x);
+        auto prefetch_stage = [&](int m_, int e_, int cs) {
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            tma_prefetch_3d(&maps.codes[mt], cs * (kKC / 2), row0_of(p, m_, mt), e_);
+            if ((cs & 3) == 0) tma_prefetch_3d(&maps.scales[mt], (cs >> 2) * 16, row0_of(p, m_, mt), e_);
+          }
+        };
         for (int c = 0; c < nst && ok; ++c, ++q) {
           if ((c & 3) == 0) {                       // scales of stages c .. c+3
             const int ss = qs % kSStages;
@@ -375,6 +383,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                           &s_full[ss]);
             ++qs;
           }
+          // The raw codes come from HBM in 32-byte rows: prefetch them into L2 kPrefetch stages
+          // ahead of their load (the ring is only kWStages deep).
+          if (c == 0)
+            for (int cp = 1; cp < kPrefetch && cp < nst; ++cp) prefetch_stage(m, e, cp);
+          if (c + kPrefetch < nst) prefetch_stage(m, e, c + kPrefetch);
           const int ws = q % kWStages;
           if (!mbar_wait(&w_empty[ws], ((q / kWStages) & 1) ^ 1)) {
             ok = false;

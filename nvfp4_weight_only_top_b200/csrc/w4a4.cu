@@ -14,21 +14,25 @@
 // Kernels:
 //   w4a4_quant_x_kernel -- one warp per routed row (expert order): 16 BF16 inputs per lane and
 //       step -> 8 code bytes and one scale byte;
-//   w4a4_gemm_kernel<gate/up | down> -- one persistent CTA per SM, tiles handed out from a global
-//       counter.  Tile = one group of up to 128 routed rows of one expert (MMA M = 128) x 256
-//       weight rows (MMA N = 256; gate/up: 128 gate rows and the same 128 up rows).  Per K stage of
-//       256 inputs (one 128-byte swizzle row of codes):
+//   w4a4_gemm_kernel<stages, gate/up | down> -- one persistent CTA per SM, tiles handed out from a
+//       global counter.  Tile = one group of up to 128 routed rows of one expert (MMA M = 128) x
+//       256 weight rows (MMA N = 256; gate/up: 128 gate rows and the same 128 up rows).  Per K
+//       stage of 256 inputs (one 128-byte swizzle row of codes; 54 KB; four stages in flight for
+//       gate/up, three for down, whose epilogue staging takes the room of the fourth):
 //         warp 8 (one thread)  TMA: activation codes 128 x 128 B, weight codes 2 x 128 x 128 B (both
 //                              128B-swizzled, K-major), scale bytes 128 x 16 B and 2 x 128 x 16 B;
-//         warp 9               rearranges the scale bytes into the layout the tensor core reads them
-//                              in: per MMA (64 inputs) and 128 rows, 512 bytes with row 32j + i at
-//                              byte 16 i + 4 j (its four block scales in one 32-bit word);
+//         warp 9               rearranges the scale bytes in place into the layout the tensor core
+//                              reads them in: per MMA (64 inputs) and 128 rows, 512 bytes with row
+//                              32j + i at byte 16 i + 4 j (its four block scales in one 32-bit word);
 //         warp 10 (one thread) tcgen05.cp of those 512-byte chunks into tensor memory (32 lanes x
 //                              128 bits, broadcast to the four lane quarters), then four MMAs of
 //                              K = 64; tcgen05.commit frees the stage;
-//         warps 0-7            epilogue: each thread owns one routed row (a TMEM lane); gate/up
-//                              forms h from gate and up columns, quantizes it per block of 16 in
-//                              registers and stores codes and scales; down stores y in f32.
+//         warps 0-7            epilogue: each thread owns one routed row (a TMEM lane) and copies
+//                              its accumulator columns to registers first, handing the accumulator
+//                              back to the next tile's MMAs; gate/up then forms h from gate and up
+//                              columns and quantizes it per block of 16 in registers, storing codes
+//                              and scales; down stores y in f32 through a per-warp shared tile, a
+//                              row's 32 columns per warp store.
 // Tensor memory: accumulator columns 0..255, then two sets of 48 scale-factor columns (one per
 // stage parity: 4 MMAs x (4 columns for the activations + 8 for the weights)).
 #include <cuda.h>
@@ -43,21 +47,29 @@ namespace {
 constexpr int kM = 128;                   // routed rows per tile (MMA M)
 constexpr int kN = 256;                   // weight rows per tile (MMA N)
 constexpr int kKS = 256;                  // inputs per stage
-constexpr int kSt = 3;                    // pipeline stages
 constexpr int kACodes = kM * kKS / 2;     // 16 KB
 constexpr int kBCodes = kN * kKS / 2;     // 32 KB
 constexpr int kARaw = kM * 16;            // 2 KB: 16 scale bytes per row and stage
 constexpr int kBRaw = kN * 16;            // 4 KB
-constexpr int kAAtoms = 4 * 512;          // per stage: 4 MMAs x 128 rows x 4 scale bytes
-constexpr int kBAtoms = 4 * 1024;         // per stage: 4 MMAs x 256 rows x 4 scale bytes
-constexpr int kOffBc = kSt * kACodes;
-constexpr int kOffAr = kOffBc + kSt * kBCodes;
-constexpr int kOffBr = kOffAr + kSt * kARaw;
-constexpr int kOffAa = kOffBr + kSt * kBRaw;
-constexpr int kOffBa = kOffAa + kSt * kAAtoms;
-constexpr int kOffBars = kOffBa + kSt * kBAtoms;
-constexpr int kSmem = kOffBars + 512 /*barriers, tile queue*/ + 1024 /*alignment*/;
-static_assert(kSmem <= 232448, "shared memory per block");
+constexpr int kEpiPitch = 36;             // floats per staged row (16-byte aligned, 4 wavefronts per v4 store)
+constexpr int kEpiBytes = 8 * 32 * kEpiPitch * 4;   // per epilogue warp: 32 rows x 32 floats
+
+// Shared-memory layout with ST stages: activation codes | weight codes | activation scale bytes |
+// weight scale bytes (both rearranged in place into the tensor core's layout) | barriers | (down
+// only) the epilogue's staging of y.  Gate/up keeps four stages in flight, down three (its
+// epilogue staging takes the room of the fourth).
+template <int ST, bool GATEUP>
+struct Layout {
+  static constexpr int kOffBc = ST * kACodes;
+  static constexpr int kOffAr = kOffBc + ST * kBCodes;
+  static constexpr int kOffBr = kOffAr + ST * kARaw;
+  static constexpr int kOffBars = kOffBr + ST * kBRaw;
+  static constexpr int kOffEpi = kOffBars + 512;  // barriers, tile queue
+  static constexpr int kSmem = kOffEpi + (GATEUP ? 0 : kEpiBytes) + 1024 /*alignment*/;
+  static_assert(kSmem <= 232448, "shared memory per block");
+};
+constexpr int kStGateUp = 4, kStDown = 3;
+constexpr int kPrefetch = 6;              // stages of weights prefetched into L2 ahead of their load
 constexpr int kEpiWarps = 8;
 constexpr int kWarpTma = kEpiWarps, kWarpSf = kEpiWarps + 1, kWarpMma = kEpiWarps + 2;
 constexpr int kThreads = 32 * (kEpiWarps + 3);
@@ -98,6 +110,9 @@ struct GemmMaps {
 __device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
+__device__ __forceinline__ void st_shared_v4f(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
 __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
@@ -132,17 +147,17 @@ __host__ __device__ __forceinline__ uint32_t idesc_nvf4(int M, int N) {
   return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+template <int kSt, bool GATEUP>
 __global__ void __launch_bounds__(kThreads, 1) w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps,
                                                                 const GemmParams p) {
+  using L = Layout<kSt, GATEUP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* sAc = smem;
-  uint8_t* sBc = smem + kOffBc;
-  uint8_t* sAr = smem + kOffAr;
-  uint8_t* sBr = smem + kOffBr;
-  uint8_t* sAa = smem + kOffAa;
-  uint8_t* sBa = smem + kOffBa;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBars);
+  uint8_t* sBc = smem + L::kOffBc;
+  uint8_t* sAr = smem + L::kOffAr;                     // scale bytes: raw, then the tensor core's layout
+  uint8_t* sBr = smem + L::kOffBr;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBars);
   uint64_t* full = bars;                   // [kSt] TMA -> scale warp, MMA
   uint64_t* sf_full = full + kSt;          // [kSt] scale warp -> MMA
   uint64_t* empty = sf_full + kSt;         // [kSt] MMA commit -> TMA
@@ -206,18 +221,27 @@ __global__ void __launch_bounds__(kThreads, 1) w4a4_gemm_kernel(const __grid_con
       tc_fence_after();
       const bool valid = r < grp.z;
       const int64_t row = (int64_t)grp.y + r;
-      if (p.gateup) {
+      // All of this warp's accumulator columns go to registers first (128 per thread), and the
+      // accumulator is handed back before any arithmetic, so the next tile's MMAs overlap the
+      // rest of this epilogue.
+      uint32_t d[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(lane_base + (GATEUP ? (c & 1) * 128 + 64 * hf + 32 * (c >> 1) : 128 * hf + 32 * c), d[c]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(d_empty);
+      if (GATEUP) {
+        // d[2c] = gate, d[2c + 1] = up columns of h columns 64 hf + 32 c .. +31
         const float cg = gm0 * sx, cu = gm1 * sx;
-#pragma unroll 1
+#pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int col = 64 * hf + 32 * c;          // h column within the tile
-          uint32_t dg[32], du[32];
-          tmem_ld32(lane_base + col, dg);
-          tmem_ld32(lane_base + 128 + col, du);
-          tmem_wait_ld();
           float hv[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) hv[j] = silu_mul(__uint_as_float(dg[j]) * cg, __uint_as_float(du[j]) * cu);
+          for (int j = 0; j < 32; ++j)
+            hv[j] = silu_mul(__uint_as_float(d[2 * c][j]) * cg, __uint_as_float(d[2 * c + 1][j]) * cu);
           uint32_t cw[4], sc[2];
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
@@ -247,25 +271,24 @@ __global__ void __launch_bounds__(kThreads, 1) w4a4_gemm_kernel(const __grid_con
           }
         }
       } else {
+        // y through a per-warp shared-memory tile: a thread holds 32 columns of one row, a warp
+        // store writes 32 columns of one row (128 contiguous bytes) -- row by row.
         const float cy = gm0 * sh;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          const int col = 128 * hf + 32 * c;
-          uint32_t d[32];
-          tmem_ld32(lane_base + col, d);
-          tmem_wait_ld();
-          if (valid) {
-            float4* o = reinterpret_cast<float4*>(p.y + row * p.H + m * kN + col);
+        float* stg = reinterpret_cast<float*>(smem + L::kOffEpi) + warp * 32 * kEpiPitch;
+        const uint32_t my = smem_addr(stg + lane * kEpiPitch);
+        const int nrows = min(32, grp.z - 32 * q4);    // valid rows of this lane quarter
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              o[j] = make_float4(__uint_as_float(d[4 * j]) * cy, __uint_as_float(d[4 * j + 1]) * cy,
-                                 __uint_as_float(d[4 * j + 2]) * cy, __uint_as_float(d[4 * j + 3]) * cy);
-          }
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4f(my + 16 * j, __uint_as_float(d[c][4 * j]) * cy, __uint_as_float(d[c][4 * j + 1]) * cy,
+                          __uint_as_float(d[c][4 * j + 2]) * cy, __uint_as_float(d[c][4 * j + 3]) * cy);
+          __syncwarp();
+          float* o = p.y + ((int64_t)grp.y + 32 * q4) * p.H + m * kN + 128 * hf + 32 * c + lane;
+          for (int rr = 0; rr < nrows; ++rr) o[(int64_t)rr * p.H] = stg[rr * kEpiPitch + lane];
+          __syncwarp();
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(d_empty);
     }
   } else if (warp == kWarpTma) {
     // ------------------------------------------------------------ tile scheduler + TMA
@@ -282,8 +305,17 @@ __global__ void __launch_bounds__(kThreads, 1) w4a4_gemm_kernel(const __grid_con
         if (tt < 0) break;
         const int g = tt / p.tiles_per_group, m = tt - g * p.tiles_per_group;
         const int4 grp = __ldg(&p.groups[g]);
-        const int row0 = p.gateup ? m * 128 : m * kN, row1 = p.gateup ? m * 128 : m * kN + 128;
+        const int row0 = GATEUP ? m * 128 : m * kN, row1 = GATEUP ? m * 128 : m * kN + 128;
+        // Weight boxes come from HBM: prefetch them into L2 kPrefetch stages ahead of their load.
+        auto prefetch_stage = [&](int cs) {
+          tma_prefetch_3d(&maps.b_codes[0], cs * (kKS / 2), row0, grp.x);
+          tma_prefetch_3d(&maps.b_codes[1], cs * (kKS / 2), row1, grp.x);
+          tma_prefetch_3d(&maps.b_scales[0], cs * 16, row0, grp.x);
+          tma_prefetch_3d(&maps.b_scales[1], cs * 16, row1, grp.x);
+        };
+        for (int cp = 1; cp < kPrefetch && cp < nst; ++cp) prefetch_stage(cp);
         for (int c = 0; c < nst; ++c, ++q) {
+          if (c + kPrefetch < nst) prefetch_stage(c + kPrefetch);
           const int s = q % kSt;
           if (!mbar_wait(&empty[s], ((q / kSt) & 1) ^ 1)) {
             ok = false;
@@ -322,30 +354,30 @@ __global__ void __launch_bounds__(kThreads, 1) w4a4_gemm_kernel(const __grid_con
           ok = false;
           break;
         }
-        const uint32_t ar = smem_addr(sAr + s * kARaw), aa = smem_addr(sAa + s * kAAtoms);
-        const uint32_t br = smem_addr(sBr + s * kBRaw), ba = smem_addr(sBa + s * kBAtoms);
+        // In place: every lane loads its 12 rows before any lane stores.
+        const uint32_t ar = smem_addr(sAr + s * kARaw), br = smem_addr(sBr + s * kBRaw);
+        uint4 va[4], vb[8];
+#pragma unroll
+        for (int it = 0; it < 4; ++it) va[it] = lds_v4(ar + 16 * (32 * j4 + 8 * it + i8));
+#pragma unroll
+        for (int it = 0; it < 8; ++it) vb[it] = lds_v4(br + 16 * (128 * (it >> 2) + 32 * j4 + 8 * (it & 3) + i8));
+        __syncwarp();
 #pragma unroll
         for (int it = 0; it < 4; ++it) {
-          const int ii = 8 * it + i8, rr = 32 * j4 + ii;
-          const uint4 v = lds_v4(ar + 16 * rr);
-          const uint32_t dst = aa + 16 * ii + 4 * j4;
-          st_shared_u32(dst, v.x);
-          st_shared_u32(dst + 512, v.y);
-          st_shared_u32(dst + 1024, v.z);
-          st_shared_u32(dst + 1536, v.w);
+          const uint32_t dst = ar + 16 * (8 * it + i8) + 4 * j4;
+          st_shared_u32(dst, va[it].x);
+          st_shared_u32(dst + 512, va[it].y);
+          st_shared_u32(dst + 1024, va[it].z);
+          st_shared_u32(dst + 1536, va[it].w);
         }
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-          for (int it = 0; it < 4; ++it) {
-            const int ii = 8 * it + i8, rr = 128 * cc + 32 * j4 + ii;
-            const uint4 v = lds_v4(br + 16 * rr);
-            const uint32_t dst = ba + 512 * cc + 16 * ii + 4 * j4;
-            st_shared_u32(dst, v.x);
-            st_shared_u32(dst + 1024, v.y);
-            st_shared_u32(dst + 2048, v.z);
-            st_shared_u32(dst + 3072, v.w);
-          }
+        for (int it = 0; it < 8; ++it) {
+          const uint32_t dst = br + 512 * (it >> 2) + 16 * (8 * (it & 3) + i8) + 4 * j4;
+          st_shared_u32(dst, vb[it].x);
+          st_shared_u32(dst + 1024, vb[it].y);
+          st_shared_u32(dst + 2048, vb[it].z);
+          st_shared_u32(dst + 3072, vb[it].w);
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sf_full[s]);
@@ -374,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a4_gemm_kernel(const __grid_con
           }
           tc_fence_after();
           const uint32_t sf = tmem + kSfCol + (uint32_t)((q & 1) * kSfSet);
-          const uint32_t aa = smem_addr(sAa + s * kAAtoms), ba = smem_addr(sBa + s * kBAtoms);
+          const uint32_t aa = smem_addr(sAr + s * kARaw), ba = smem_addr(sBr + s * kBRaw);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             tc_cp_sf(sf + 12 * k, smem_desc_sf(aa + 512 * k));
@@ -467,12 +499,19 @@ int make_weight_maps(GemmMaps* m, const BankView& bank, int proj0, int proj1, in
   return 0;
 }
 
-int launch_gemm(const GemmParams& p, const GemmMaps& maps, int num_sms, cudaStream_t s) {
-  cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(w4a4_gemm_kernel), kSmem);
+template <int ST, bool GATEUP>
+int launch_gemm_t(const GemmParams& p, const GemmMaps& maps, int num_sms, cudaStream_t s) {
+  constexpr int smem = Layout<ST, GATEUP>::kSmem;
+  cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(w4a4_gemm_kernel<ST, GATEUP>), smem);
   if (err != cudaSuccess) return -(int)err;
-  w4a4_gemm_kernel<<<num_sms, kThreads, kSmem, s>>>(maps, p);
+  w4a4_gemm_kernel<ST, GATEUP><<<num_sms, kThreads, smem, s>>>(maps, p);
   err = cudaGetLastError();
   return err == cudaSuccess ? 1 : -(int)err;
+}
+
+int launch_gemm(const GemmParams& p, const GemmMaps& maps, int num_sms, cudaStream_t s) {
+  return p.gateup ? launch_gemm_t<kStGateUp, true>(p, maps, num_sms, s)
+                  : launch_gemm_t<kStDown, false>(p, maps, num_sms, s);
 }
 
 }  // namespace

@@ -154,6 +154,37 @@ def test_forward_host_matches_device_call():
     assert np.array_equal(bits_of(dev), host)
 
 
+def test_forward_host_repeated_calls_replay_correctly():
+    """Small host calls replay a captured graph after their first (eager) call: repeated calls
+    with new inputs, alternating sizes and banks, pinned and pageable buffers, and a growth of
+    the internal workspace in between all equal the device call bit for bit."""
+    import torch
+    import nvfp4_weight_only_top_b200 as moe
+    cfgs = [moe_inputs.LayerConfig("host_a", 16, 4, 1024, 512, 1, seed=3),
+            moe_inputs.LayerConfig("host_b", 16, 4, 1024, 512, 3, seed=4),
+            moe_inputs.LayerConfig("host_c", 32, 8, 512, 256, 2, seed=5)]
+    banks = [device_bank(c) for c in cfgs]
+    for it in range(4):
+        for ci, cfg in enumerate(cfgs):
+            xb = moe_inputs.make_x(cfg, seed=100 + it)
+            lg = moe_inputs.make_logits(cfg, seed=200 + it)
+            if it % 2:
+                xh = torch.from_numpy(xb.view(np.int16)).pin_memory().numpy().view(np.uint16)
+                lh = torch.from_numpy(lg).pin_memory().numpy()
+            else:
+                xh, lh = xb, lg
+            dev = moe.moe_nvfp4_forward(bf16_tensor(xb), torch.from_numpy(lg).cuda(), banks[ci][1], cfg.k)
+            host = moe.moe_nvfp4_forward_host(xh, lh, banks[ci][1], cfg.k)
+            assert np.array_equal(bits_of(dev), host), (it, cfg.name)
+        if it == 1:     # grow the internal workspace (a large call), so cached graphs must be rebuilt
+            big = moe_inputs.LayerConfig("host_big", 16, 4, 1024, 512, 2048, seed=6)
+            bb = device_bank(big)
+            moe.moe_nvfp4_forward(bf16_tensor(moe_inputs.make_x(big)), torch.from_numpy(moe_inputs.make_logits(big)).cuda(),
+                                  bb[1], big.k)
+            torch.cuda.synchronize()
+    assert moe.moe_nvfp4_device_status() == 0
+
+
 def test_workspace_too_small_is_rejected():
     import torch
     import nvfp4_weight_only_top_b200 as moe
