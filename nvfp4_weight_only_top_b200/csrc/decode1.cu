@@ -180,6 +180,9 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
     if (ahead < k) s_ids[ahead] = threadIdx.x;
   }
   __syncthreads();
+  // The producer starts streaming now; the softmax weights are only needed by the combine at the
+  // end (after the consumer warps' later barriers), so warp 0 forms them while the first copies
+  // are in flight.
   if (warp == 0) {                                          // softmax over the k selected
     const int id = lane < k ? s_ids[lane] : 0;
     const float l = lane < k ? __ldg(p.logits + id) : 0.0f;
@@ -197,7 +200,6 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
       }
     }
   }
-  __syncthreads();
 
   if (warp == kNW) {
     // ---------------------------------------------------------------- producer
@@ -502,7 +504,8 @@ __global__ void __launch_bounds__(kThreads1, 1) decode1_kernel(const D1Params p)
         }
       }
     }
-    for (int i = warp; i < *s_ok; i += kNW) {
+    // Warps 1.. combine while warp 0 takes the exit count (and, in the last CTA, clears the set).
+    for (int i = warp - 1; warp > 0 && i < *s_ok; i += kNW - 1) {
       const int c = 32 * s_last[i] + lane;
       float a = 0.0f;
       for (int jj = 0; jj < k; ++jj) a = fmaf(s_w[jj], __ldcg(p.y + (size_t)jj * H + c), a);

@@ -23,6 +23,8 @@ struct RouteBufs {
   int32_t* chunk_counts;  // [nchunks, E] (multi-CTA routing only)
   int group_rows;      // rows per group (decode token tile)
   int split_singles;   // 1: one-row groups go to `singles`; 0: they stay in `groups`
+  int expert_major;    // 1: each expert's groups are listed together (full, then its partial);
+                       // 0: all full groups first, then the partial ones
 };
 
 // Tokens per routing chunk in the multi-CTA router; one CTA routes T <= this on its own.

@@ -303,6 +303,7 @@ moe::RouteBufs route_bufs(uint8_t* ws, const WsLayout& L) {
   b.chunk_counts = reinterpret_cast<int32_t*>(ws + L.chunk_counts);
   b.group_rows = 8;
   b.split_singles = 0;
+  b.expert_major = 0;
   return b;
 }
 
@@ -462,6 +463,7 @@ int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
     // the persistent gate/up and down kernels, then the combine.
     rb.group_rows = 8;
     rb.split_singles = 0;
+    rb.expert_major = 1;           // an expert's groups stream together (repeat reads hit L2)
     float* h = reinterpret_cast<float*>(w8 + L.h);
     float* y = reinterpret_cast<float*>(w8 + L.y);
     prof_before(MOE_NVFP4_KERNEL_ROUTE, s);

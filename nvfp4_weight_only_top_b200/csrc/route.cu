@@ -58,15 +58,19 @@ __device__ int block_scan_excl(int* a, int n, int* warp_tmp) {
 // are cut into groups of group_rows; when split_singles is set, a last group of a single row
 // goes to the one-row list instead.  All full groups (exactly group_rows rows) come first, in
 // expert order, then the partial ones: a kernel that hands out groups in list order starts
-// with the large work items and fills in with the small ones.
+// with the large work items and fills in with the small ones.  With expert_major, each expert's
+// groups are listed together instead (its full groups, then its partial one), so that a kernel
+// streaming the list in order reads an expert's weights for all of its groups at about the same
+// time (the repeats then come from L2).
 __device__ void finish_counts(int* cnt, int* tmp, int* tmp1, int* tmp2, int* warp_tmp, int E, int group_rows,
                               const RouteBufs& b) {
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const int c = cnt[e], full = c / group_rows, r = c - full * group_rows;
     const int single = (b.split_singles && r == 1) ? 1 : 0;
+    const int part = (r > 0 && !single) ? 1 : 0;
     b.counts[e] = c;
-    tmp[e] = full;
-    tmp2[e] = (r > 0 && !single) ? 1 : 0;
+    tmp[e] = b.expert_major ? full + part : full;
+    tmp2[e] = b.expert_major ? 0 : part;
     tmp1[e] = single;
   }
   __syncthreads();
@@ -82,7 +86,8 @@ __device__ void finish_counts(int* cnt, int* tmp, int* tmp1, int* tmp2, int* war
     const int rest = c - full * group_rows - single;        // rows of the partial group
     for (int q = 0; q < full; ++q)
       b.groups[tmp[e] + q] = make_int4(e, cnt[e] + q * group_rows, group_rows, 0);
-    if (rest > 0) b.groups[nf + tmp2[e]] = make_int4(e, cnt[e] + full * group_rows, rest, 0);
+    if (rest > 0)
+      b.groups[b.expert_major ? tmp[e] + full : nf + tmp2[e]] = make_int4(e, cnt[e] + full * group_rows, rest, 0);
     if (single) b.singles[tmp1[e]] = make_int4(e, cnt[e] + c - 1, 1, 0);
   }
   if (threadIdx.x == 0) {
