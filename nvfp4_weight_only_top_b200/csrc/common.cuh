@@ -321,6 +321,50 @@ __device__ __forceinline__ uint32_t nvfp4_encode16(const float (&v)[16], float s
   return scale;
 }
 
+// The same encoding with the 16 code decisions taken from q = f32(|v| x f32(1 / eff)) instead of
+// a division per value, where that gives the same code: q is within about 3 x 2^-24 (relative) of
+// f32(v / eff), so when q (1 - 2^-20) and q (1 + 2^-20) round to the same E2M1 code, no code
+// boundary (nor a tie on one) lies between q and f32(v / eff), and that code is the one the
+// division would give.  Otherwise (rarely) the 8 values of that half are decided by division.
+__device__ __forceinline__ uint32_t nvfp4_encode16_fast(const float (&v)[16], float s2, uint32_t& lo, uint32_t& hi) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t scale = f32_to_e4m3_byte(__fdiv_rn(amax, __fmul_rn(6.0f, s2)));
+  const float eff = __fmul_rn(e4m3_byte_to_f32(scale), s2);
+  lo = 0;
+  hi = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    lo |= (__float_as_uint(v[i]) >> 31) << (4 * i + 3);
+    hi |= (__float_as_uint(v[8 + i]) >> 31) << (4 * i + 3);
+  }
+  if (eff > 0.0f) {
+    const float r = __frcp_rn(eff);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float a[8], b[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float q = __fmul_rn(fabsf(v[8 * h + i]), r);
+        a[i] = __fmul_rn(q, 1.0f - 0x1p-20f);
+        b[i] = __fmul_rn(q, 1.0f + 0x1p-20f);
+      }
+      uint32_t c = e2m1x8_mag(a);
+      if (c != e2m1x8_mag(b)) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = fabsf(__fdiv_rn(v[8 * h + i], eff));
+        c = e2m1x8_mag(a);
+      }
+      if (h)
+        hi |= c;
+      else
+        lo |= c;
+    }
+  }
+  return scale;
+}
+
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
 // SwiGLU with the hardware exponential and fast division (a few ulp; used where the result is

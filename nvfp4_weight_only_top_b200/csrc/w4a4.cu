@@ -241,14 +241,14 @@ __global__ void __launch_bounds__(kThreads, 1) w4a4_gemm_kernel(const __grid_con
           float hv[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            hv[j] = silu_mul(__uint_as_float(d[2 * c][j]) * cg, __uint_as_float(d[2 * c + 1][j]) * cu);
+            hv[j] = silu_mul_fast(__uint_as_float(d[2 * c][j]) * cg, __uint_as_float(d[2 * c + 1][j]) * cu);
           uint32_t cw[4], sc[2];
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
             float blk[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) blk[j] = hv[16 * b + j];
-            sc[b] = nvfp4_encode16(blk, sh, cw[2 * b], cw[2 * b + 1]);
+            sc[b] = nvfp4_encode16_fast(blk, sh, cw[2 * b], cw[2 * b + 1]);
           }
           if (valid) {
             const int hcol = m * kM + col;           // h index
@@ -460,7 +460,7 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
       v[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
     }
     uint32_t lo, hi;
-    const uint32_t sc = nvfp4_encode16(v, s2, lo, hi);
+    const uint32_t sc = nvfp4_encode16_fast(v, s2, lo, hi);
     *reinterpret_cast<uint2*>(codes + r * (H / 2) + 8 * b) = make_uint2(lo, hi);
     scales[r * (H / 16) + b] = (uint8_t)sc;
     if (tap_codes) {

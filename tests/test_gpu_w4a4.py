@@ -136,3 +136,26 @@ def test_w4a4_rejects_unsupported_shapes_and_bad_taps():
     with pytest.raises(moe.MoeError) as ei:      # codes without scales
         moe.moe_nvfp4_forward_w4a4(x, lg, bank, act, cfg.k, taps={"x_codes": codes})
     assert ei.value.code == -1
+
+
+def test_w4a4_code_ties_decided_as_by_division():
+    """Activations exactly on E2M1 rounding ties (and block maxima that make the block scale 1
+    exactly): the GPU decides such codes by division (ties to even); every x code and scale byte
+    equals the oracle's."""
+    cfg = moe_inputs.LayerConfig(name="w4a4_ties", E=8, k=2, H=512, I=256, T=16, seed=2)
+    buf, bank = device_bank(cfg)
+    lg = moe_inputs.make_logits(cfg)
+    s = np.float32(2.0 ** -8)
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    rng = np.random.default_rng(4)
+    x = np.empty((cfg.T, cfg.H), np.float32)
+    for t in range(cfg.T):
+        for b in range(cfg.H // 16):
+            blk = rng.choice(np.concatenate([ties, -ties, ties * 0.5, np.float32([0.5, 1.0, 3.0])]), 16)
+            blk[rng.integers(16)] = 6.0 * (1 if rng.random() < 0.5 else -1)   # block maximum 6 s
+            x[t, 16 * b:16 * b + 16] = blk * s
+    xb = moe_inputs.gen.to_bf16_bits(x)
+    assert np.array_equal(oracle.bf16_bits_to_f64(xb), x.astype(np.float64))   # exact in BF16
+    act = np.tile(np.array([[s, np.float32(4.0 / 2688)]], np.float32), (cfg.E, 1))
+    out, taps = _run(cfg, bank, xb, lg, act)
+    _check_slots(cfg, xb, lg, act, taps, range(cfg.T * cfg.k))
