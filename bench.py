@@ -53,7 +53,7 @@ def parse():
     ap.add_argument("--config", default=None, choices=[c for c in moe_inputs.CONFIGS if c != "tiny"],
                     help="one workload only (default: decode_t1 as the headline, then every other "
                          "full-size workload in the same line)")
-    ap.add_argument("--ncu-case", default=None, choices=["decode_t1_e16", "decode_t16_e16", "decode_t64_e16",
+    ap.add_argument("--ncu-case", default=None, choices=["decode_t1_e16", "decode_t8_e16", "decode_t16_e16", "decode_t64_e16",
                                                         "prefill_t4096_e16", "decode_t64z_e64", "w4a4_t4096_e16"],
                     help="plain layer calls on a small bank for ncu captures (no timing, no graph)")
     ap.add_argument("--calls", type=int, default=4, help="layer calls of --ncu-case")
@@ -718,7 +718,8 @@ def ncu_case(case: str, calls: int) -> None:
 
     Cases (full-size records H=5120, I=2560, 16 experts resident = 354 MB, above the 126 MB L2):
     decode_t1_e16 (T=1, each call routes to 8 experts the previous call did not use),
-    decode_t16_e16 (T=16), decode_t64_e16 (T=64), prefill_t4096_e16 (T=4096, tensor-core path);
+    decode_t8_e16 (T=8, the few-token kernel), decode_t16_e16 and decode_t64_e16 (T=16 and 64, the
+    grouped kernels), prefill_t4096_e16 (T=4096, tensor-core path);
     decode_t64z_e64: T=64 with Zipf routing over 64 resident experts (1.4 GB);
     w4a4_t4096_e16: T=4096 on the W4A4 path (NVFP4 activations).
     """
@@ -749,7 +750,8 @@ def ncu_case(case: str, calls: int) -> None:
     print(f"{case}: {calls} calls ok")
 
 
-NCU_CASES = {"decode_t1_e16": (1, "decode"), "decode_t16_e16": (16, "decode"), "decode_t64_e16": (64, "decode"),
+NCU_CASES = {"decode_t1_e16": (1, "decode"), "decode_t8_e16": (8, "decode"), "decode_t16_e16": (16, "decode"),
+             "decode_t64_e16": (64, "decode"),
              "prefill_t4096_e16": (4096, "prefill"), "decode_t64z_e64": (64, "decode"),
              "w4a4_t4096_e16": (4096, "w4a4")}
 
