@@ -280,3 +280,31 @@ def test_few_tokens_fused_kernel(E, k, H, I, T, mode):
         assert moe.moe_nvfp4_last_launch_count() == (2 if T < 12 else 4)
         assert_layer_close(oracle.bf16_bits_to_f64(out), ref["out"], f"T={T} {E},{k},{H},{I}/{path}")
         assert np.array_equal(xn, oracle.residual_add(xb, out))
+
+
+def test_prefill_pair_kernel_matches_oracle():
+    """The CTA-pair prefill kernel (tcgen05 cta_group::2, selected by MOE_NVFP4_PREFILL=pair when
+    the library loads) on full and partial groups, in a fresh process, against the oracle."""
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import numpy as np, torch, moe_inputs, oracle\n"
+        "import nvfp4_weight_only_top_b200 as moe\n"
+        "from gpu_helpers import device_bank, bf16_tensor, bits_of\n"
+        "from conftest import assert_layer_close\n"
+        "for (E, k, H, I, T) in [(16, 8, 512, 256, 700), (8, 2, 1024, 512, 300)]:\n"
+        "    cfg = moe_inputs.LayerConfig('pair', E, k, H, I, T, 1, 'normal', seed=T)\n"
+        "    buf, bank = device_bank(cfg)\n"
+        "    xb, lg = moe_inputs.make_x(cfg), moe_inputs.make_logits(cfg)\n"
+        "    out = moe.moe_nvfp4_forward_ex(bf16_tensor(xb), torch.from_numpy(lg).cuda(), bank, k, path=moe.PATH_PREFILL)\n"
+        "    torch.cuda.synchronize()\n"
+        "    assert moe.moe_nvfp4_device_status() == 0\n"
+        "    ref = oracle.layer_forward(xb, lg, k, oracle.GeneratedRecords(cfg.seed, 0, E, H, I))\n"
+        "    assert_layer_close(oracle.bf16_bits_to_f64(bits_of(out)), ref['out'], f'pair {E} {k} {H} {I} {T}')\n"
+        "print('pair ok')\n")
+    here = os.path.dirname(os.path.abspath(__file__))
+    env = dict(os.environ, MOE_NVFP4_PREFILL="pair",
+               PYTHONPATH=os.pathsep.join([here, os.path.dirname(here), os.environ.get("PYTHONPATH", "")]))
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and "pair ok" in r.stdout, r.stdout[-2000:] + r.stderr[-2000:]
