@@ -214,6 +214,112 @@ int moe_nvfp4_route(const float* logits_dev, int64_t T, int32_t E, int32_t k, in
                     int32_t* inv_dev, void* stream);
 
 /*
+ * Experts only: y_rows[r] = Wd_e (silu(Wg_e x) * (Wu_e x)) for row r of x_rows with e =
+ * expert_ids[r], in f32, unweighted -- the routed-expert step of the layer without the router
+ * and the combine, for expert parallelism (a rank runs its own experts on the rows other ranks
+ * send it; the layer's method statement is moe_nvfp4_forward's).  x_rows_dev [R, H] BF16,
+ * expert_ids_dev [R] int32 in any order, y_rows_dev [R, H] f32.  An id outside [0, E) marks a
+ * padding row: its y row is zero and it costs no expert work.  The same expert kernels as the
+ * layer (path as in moe_nvfp4_forward_ex with T = R, k = 1): for a row, the result is the one
+ * the layer computes for that row and expert on the same path.  workspace_dev: NULL for the
+ * internal workspace, else at least moe_nvfp4_experts_workspace_bytes(...) bytes, 256-byte
+ * aligned.  R = 0 returns OK.
+ */
+int moe_nvfp4_experts(const void* x_rows_dev, const int32_t* expert_ids_dev, int64_t R,
+                      const moe_nvfp4_bank* bank, float* y_rows_dev, void* workspace_dev,
+                      size_t workspace_bytes, int32_t path, void* stream);
+size_t moe_nvfp4_experts_workspace_bytes(int64_t R, int32_t E, int32_t H, int32_t I,
+                                         int32_t path);
+
+/*
+ * Expert parallelism (EP) over G ranks, one process per GPU.  Source: the pages' servers run the
+ * model with expert parallelism over eight GPUs (page "Running Beam-1.0 (501B) on workstation
+ * GPUs", the serving configurations; page "Beam 1.0 501B-A23B, streaming pack, NVFP4 experts /
+ * MLX 8-bit residents", the eight-GPU server line).  The layer is the one of moe_nvfp4_forward;
+ * EP only changes where each expert runs.  Rank d holds global experts d*El .. d*El+El-1
+ * (El = E / G) as a bank of El records (a moe_nvfp4_bank whose base points at record d*El of the
+ * full bank layout) and routes its own tokens over all E with moe_nvfp4_route (ids, w, counts,
+ * offsets, perm, inv).  counts_all [G][E] int32 is every rank's counts, row s from rank s (an
+ * all-gather the caller performs).  One step, on every rank:
+ *   route -> all-gather counts -> ep_plan -> ep_dispatch -> barrier -> moe_nvfp4_experts on the
+ *   rows received (recv_ids as expert ids) -> barrier -> ep_combine.
+ * The barriers are the caller's (any stream-ordered cross-rank barrier, e.g. an all-reduce of
+ * one element); dispatch ends with a system-scope fence so that a barrier after it publishes its
+ * peer stores.  Receive buffers: rank d's recv_x [Rd, H] BF16 and recv_y [Rd, H] f32, with Rd =
+ * sum over s of counts_all[s][d*El .. d*El+El-1] (the rows the plan sends there), allocated with
+ * moe_nvfp4_ep_buffer_create and opened in every other rank's process with
+ * moe_nvfp4_ep_buffer_open; the caller checks Rd against their capacity before dispatching.
+ */
+#define MOE_NVFP4_EP_EXPERT_MAJOR 0   /* rank d's rows: for e, the rows from rank 0, 1, ...   */
+#define MOE_NVFP4_EP_SOURCE_MAJOR 1   /* rank d's rows: from rank 0 (expert by expert), 1, ... */
+
+/*
+ * From counts_all_dev [G][E]: dst_off_dev [E], the row of the owner's buffer (layout as given)
+ * that receives this rank's first row of global expert g (the others follow in the order of
+ * perm), and recv_ids_dev [recv_rows], the local expert (0 .. El-1) of each row of this rank's
+ * buffer, -1 for rows past the ones the count matrix sends here.  SOURCE_MAJOR is the order an
+ * all-to-all of the rows gathered in perm order delivers (moe_nvfp4_gather_rows, then each
+ * rank's share of them in rank order).  One launch; E % G == 0, G <= 64.
+ */
+int moe_nvfp4_ep_plan(const int32_t* counts_all_dev, int32_t ranks, int32_t num_experts,
+                      int32_t rank, int32_t layout, int32_t* dst_off_dev, int32_t* recv_ids_dev,
+                      int64_t recv_rows, void* stream);
+
+/*
+ * Stores every routed row of this rank (x_dev [T, H] BF16; routed row r = t*k+j) into the
+ * receive buffer of the owner of ids[r], at row dst_off[g] + (inv[r] - offsets[g]) of an
+ * EXPERT_MAJOR plan.  recv_x_ptrs_host: host array of G device pointers valid in this process
+ * (this rank's own buffer, the others opened with moe_nvfp4_ep_buffer_open), each 16-byte
+ * aligned.  ids, perm and offsets are moe_nvfp4_route's for this rank's tokens.
+ * capacity_rows: rows every receive buffer holds; a row whose place falls outside
+ * [0, capacity_rows) is not stored (a plan from counts that do not match the routing).
+ */
+int moe_nvfp4_ep_dispatch(const void* x_dev, int64_t T, int32_t k, int32_t hidden,
+                          int32_t num_experts, const int32_t* ids_dev, const int32_t* perm_dev,
+                          const int32_t* offsets_dev, const int32_t* dst_off_dev, int32_t ranks,
+                          void* const* recv_x_ptrs_host, int64_t capacity_rows, void* stream);
+
+/*
+ * out_dev [T, H] BF16 = bf16(sum_j w[t, j] * y(t, j)), j ascending with f32 fused multiply-adds
+ * (the layer's combine, bit for bit), where y(t, j) is row dst_off[g] + (inv[r] - offsets[g]) of
+ * the recv_y buffer of the owner of g = ids[r], r = t*k+j, read over peer memory.
+ * recv_y_ptrs_host: host array of G device pointers (f32 [capacity_rows, H] each); a row whose
+ * place falls outside [0, capacity_rows) adds nothing.  x_next_dev as in moe_nvfp4_forward_ex
+ * (x_dev is needed only with it).
+ */
+int moe_nvfp4_ep_combine(const void* x_dev, int64_t T, int32_t k, int32_t hidden,
+                         int32_t num_experts, const int32_t* ids_dev, const float* w_dev,
+                         const int32_t* inv_dev, const int32_t* offsets_dev,
+                         const int32_t* dst_off_dev, int32_t ranks,
+                         const float* const* recv_y_ptrs_host, int64_t capacity_rows, void* out_dev,
+                         void* x_next_dev, void* stream);
+
+/*
+ * The two ends of an all-to-all exchange of the rows (for a collective library in place of the
+ * peer-memory kernels): rows_dev [T*k, H] BF16 = x[perm[p] / k] (the routed rows in expert
+ * order), and out = the layer's combine of y_dev [T*k, H] f32 held in that same order (row p is
+ * the result of routed row perm[p]); out[t] = bf16(sum_j w[t, j] * y[inv[t*k+j]]).
+ */
+int moe_nvfp4_gather_rows(const void* x_dev, const int32_t* perm_dev, int64_t T, int32_t k,
+                          int32_t hidden, void* rows_dev, void* stream);
+int moe_nvfp4_combine(const float* y_dev, const float* w_dev, const int32_t* inv_dev, int64_t T,
+                      int32_t k, int32_t hidden, const void* x_dev, void* out_dev,
+                      void* x_next_dev, void* stream);
+
+/*
+ * Peer-visible buffers (CUDA IPC): create allocates `bytes` of device memory on the current
+ * device and writes its 64-byte handle to handle_host; open maps another process's buffer
+ * from its handle into this process (peer access over NVLink) -- a process cannot open its own
+ * handle; close unmaps it, destroy frees a buffer made by create.  The caller exchanges the
+ * handles (e.g. an all-gather of bytes) and keeps each buffer alive until every peer closed it.
+ */
+#define MOE_NVFP4_EP_HANDLE_BYTES 64
+int moe_nvfp4_ep_buffer_create(uint64_t bytes, void** dev_ptr, uint8_t* handle_host);
+int moe_nvfp4_ep_buffer_open(const uint8_t* handle_host, void** peer_ptr);
+int moe_nvfp4_ep_buffer_close(void* peer_ptr);
+int moe_nvfp4_ep_buffer_destroy(void* dev_ptr);
+
+/*
  * NVFP4 encoder: turns BF16 weights into the bank's NVFP4 parts, so that BF16 experts can feed
  * the layer.  w_dev holds n projections [n, out_features, in_features] BF16, row-major (rows =
  * outputs); projection i is written to dst_dev + i * dst_stride: its E2M1 codes at + codes_off

@@ -12,6 +12,7 @@ import numpy as np
 
 from . import _abi
 from ._abi import Bank, MoeError, PackInfo, PATH_AUTO, PATH_DECODE, PATH_PREFILL  # noqa: F401
+from ._abi import EP_EXPERT_MAJOR, EP_SOURCE_MAJOR  # noqa: F401
 
 _LIB = None
 
@@ -203,6 +204,170 @@ def moe_nvfp4_route(logits, k: int, stream=None) -> dict:
     _check(lib().moe_nvfp4_route(_ptr(logits), T, E, k, _ptr(r["ids"]), _ptr(r["w"]), _ptr(r["counts"]),
                                  _ptr(r["offsets"]), _ptr(r["perm"]), _ptr(r["inv"]), _stream(stream)))
     return r
+
+
+def moe_nvfp4_experts(x_rows, expert_ids, bank: Bank, y_rows=None, workspace=None, path: int = PATH_AUTO,
+                      stream=None):
+    """y_rows [R, H] f32 = expert expert_ids[r] applied to x_rows[r] (bf16 [R, H]); ids outside
+    [0, E) are padding rows (zero output)."""
+    import torch
+    if not isinstance(x_rows, torch.Tensor) or x_rows.dim() != 2:
+        raise ValueError("x_rows must be a 2-D torch tensor [R, H]")
+    R = int(x_rows.shape[0])
+    if y_rows is None:
+        y_rows = torch.empty((R, bank.hidden), dtype=torch.float32, device=x_rows.device)
+    need = [("x_rows", x_rows, torch.bfloat16, (R, bank.hidden)), ("expert_ids", expert_ids, torch.int32, (R,)),
+            ("y_rows", y_rows, torch.float32, (R, bank.hidden))]
+    if workspace is not None:
+        need.append(("workspace", workspace, workspace.dtype, tuple(workspace.shape)))
+    for args in need:
+        _need(*args, device=False)
+    for args in need:
+        _need(*args)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().moe_nvfp4_experts(_ptr(x_rows), _ptr(expert_ids), R, ctypes.byref(bank), _ptr(y_rows),
+                                   _ptr(workspace), ws_bytes, path, _stream(stream)))
+    return y_rows
+
+
+def moe_nvfp4_experts_workspace_bytes(R: int, E: int, H: int, I: int, path: int = PATH_AUTO) -> int:
+    return int(lib().moe_nvfp4_experts_workspace_bytes(R, E, H, I, path))
+
+
+def moe_nvfp4_gather_rows(x, perm, k: int, rows=None, stream=None):
+    """rows [T*k, H] bf16 = x[perm[p] // k]: the routed rows in expert order."""
+    import torch
+    if not isinstance(x, torch.Tensor) or x.dim() != 2:
+        raise ValueError("x must be a 2-D torch tensor [T, H]")
+    T, H = (int(v) for v in x.shape)
+    if rows is None:
+        rows = torch.empty((T * k, H), dtype=torch.bfloat16, device=x.device)
+    need = [("x", x, torch.bfloat16, (T, H)), ("perm", perm, torch.int32, (T * k,)),
+            ("rows", rows, torch.bfloat16, (T * k, H))]
+    for args in need:
+        _need(*args, device=False)
+    for args in need:
+        _need(*args)
+    _check(lib().moe_nvfp4_gather_rows(_ptr(x), _ptr(perm), T, k, H, _ptr(rows), _stream(stream)))
+    return rows
+
+
+def moe_nvfp4_combine(y, w, inv, k: int, out=None, x=None, x_next=None, stream=None):
+    """out [T, H] bf16 = bf16(sum_j w[t, j] * y[inv[t*k+j]]), y f32 [T*k, H] in expert order."""
+    import torch
+    if not isinstance(w, torch.Tensor) or w.dim() != 2:
+        raise ValueError("w must be a 2-D torch tensor [T, k]")
+    T = int(w.shape[0])
+    if not isinstance(y, torch.Tensor) or y.dim() != 2:
+        raise ValueError("y must be a 2-D torch tensor [T*k, H]")
+    H = int(y.shape[1])
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=y.device)
+    need = [("y", y, torch.float32, (T * k, H)), ("w", w, torch.float32, (T, k)), ("inv", inv, torch.int32, (T * k,)),
+            ("out", out, torch.bfloat16, (T, H))]
+    if x_next is not None:
+        need += [("x", x, torch.bfloat16, (T, H)), ("x_next", x_next, torch.bfloat16, (T, H))]
+    for args in need:
+        _need(*args, device=False)
+    for args in need:
+        _need(*args)
+    _check(lib().moe_nvfp4_combine(_ptr(y), _ptr(w), _ptr(inv), T, k, H, _ptr(x if x_next is not None else None),
+                                   _ptr(out), _ptr(x_next), _stream(stream)))
+    return out
+
+
+def moe_nvfp4_ep_plan(counts_all, rank: int, recv_rows: int, layout: int = _abi.EP_EXPERT_MAJOR, stream=None):
+    """From counts_all [G, E] int32 (row s = rank s's routed rows per expert): dst_off [E] and
+    recv_ids [recv_rows] (int32 CUDA tensors), as include/moe_nvfp4.h describes."""
+    import torch
+    if not isinstance(counts_all, torch.Tensor) or counts_all.dim() != 2:
+        raise ValueError("counts_all must be a 2-D torch tensor [G, E]")
+    G, E = (int(v) for v in counts_all.shape)
+    _need("counts_all", counts_all, torch.int32, (G, E))
+    dst_off = torch.empty(E, dtype=torch.int32, device=counts_all.device)
+    recv_ids = torch.empty(max(int(recv_rows), 1), dtype=torch.int32, device=counts_all.device)
+    _check(lib().moe_nvfp4_ep_plan(_ptr(counts_all), G, E, rank, layout, _ptr(dst_off), _ptr(recv_ids),
+                                   int(recv_rows), _stream(stream)))
+    return dst_off, recv_ids[:int(recv_rows)]
+
+
+def _route_need(route: dict, T: int, k: int, E: int):
+    import torch
+    return [("ids", route["ids"], torch.int32, (T, k)), ("w", route["w"], torch.float32, (T, k)),
+            ("perm", route["perm"], torch.int32, (T * k,)), ("inv", route["inv"], torch.int32, (T * k,)),
+            ("offsets", route["offsets"], torch.int32, (E + 1,))]
+
+
+def moe_nvfp4_ep_dispatch(x, route: dict, dst_off, recv_x_ptrs, capacity_rows: int, stream=None) -> None:
+    """Stores this rank's routed rows (x [T, H] bf16, route = moe_nvfp4_route(...)) into their
+    owners' receive buffers: recv_x_ptrs holds G device addresses (ints) valid in this process,
+    each of capacity_rows rows."""
+    import torch
+    T, k = (int(v) for v in route["ids"].shape)
+    E = int(dst_off.shape[0])
+    H = int(x.shape[1])
+    G = len(recv_x_ptrs)
+    need = [("x", x, torch.bfloat16, (T, H)), ("dst_off", dst_off, torch.int32, (E,))] + _route_need(route, T, k, E)
+    for args in need:
+        _need(*args, device=False)
+    for args in need:
+        _need(*args)
+    ptrs = (ctypes.c_void_p * G)(*[int(p) for p in recv_x_ptrs])
+    _check(lib().moe_nvfp4_ep_dispatch(_ptr(x), T, k, H, E, _ptr(route["ids"]), _ptr(route["perm"]),
+                                       _ptr(route["offsets"]), _ptr(dst_off), G, ptrs, int(capacity_rows),
+                                       _stream(stream)))
+
+
+def moe_nvfp4_ep_combine(route: dict, dst_off, recv_y_ptrs, hidden: int, capacity_rows: int, out=None, x=None,
+                         x_next=None, stream=None):
+    """out [T, H] bf16 = the layer's combine of the routed rows' expert outputs, read from their
+    owners' f32 output buffers (recv_y_ptrs: G device addresses valid in this process, each of
+    capacity_rows rows)."""
+    import torch
+    T, k = (int(v) for v in route["ids"].shape)
+    E = int(dst_off.shape[0])
+    H = int(hidden)
+    G = len(recv_y_ptrs)
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=dst_off.device)
+    need = [("dst_off", dst_off, torch.int32, (E,)), ("out", out, torch.bfloat16, (T, H))] + _route_need(route, T, k, E)
+    if x_next is not None:
+        need += [("x", x, torch.bfloat16, (T, H)), ("x_next", x_next, torch.bfloat16, (T, H))]
+    for args in need:
+        _need(*args, device=False)
+    for args in need:
+        _need(*args)
+    ptrs = (ctypes.c_void_p * G)(*[int(p) for p in recv_y_ptrs])
+    _check(lib().moe_nvfp4_ep_combine(_ptr(x if x_next is not None else None), T, k, H, E, _ptr(route["ids"]),
+                                      _ptr(route["w"]), _ptr(route["inv"]), _ptr(route["offsets"]), _ptr(dst_off),
+                                      G, ptrs, int(capacity_rows), _ptr(out), _ptr(x_next), _stream(stream)))
+    return out
+
+
+def moe_nvfp4_ep_buffer_create(nbytes: int):
+    """(device address, 64-byte IPC handle) of a new peer-visible buffer on the current device."""
+    p = ctypes.c_void_p()
+    h = (ctypes.c_uint8 * _abi.EP_HANDLE_BYTES)()
+    _check(lib().moe_nvfp4_ep_buffer_create(int(nbytes), ctypes.byref(p), h))
+    return int(p.value), bytes(h)
+
+
+def moe_nvfp4_ep_buffer_open(handle: bytes) -> int:
+    """Device address, in this process, of another process's buffer."""
+    if len(handle) != _abi.EP_HANDLE_BYTES:
+        raise ValueError(f"an ep buffer handle has {_abi.EP_HANDLE_BYTES} bytes")
+    p = ctypes.c_void_p()
+    h = (ctypes.c_uint8 * _abi.EP_HANDLE_BYTES).from_buffer_copy(handle)
+    _check(lib().moe_nvfp4_ep_buffer_open(h, ctypes.byref(p)))
+    return int(p.value)
+
+
+def moe_nvfp4_ep_buffer_close(peer_ptr: int) -> None:
+    _check(lib().moe_nvfp4_ep_buffer_close(ctypes.c_void_p(int(peer_ptr))))
+
+
+def moe_nvfp4_ep_buffer_destroy(dev_ptr: int) -> None:
+    _check(lib().moe_nvfp4_ep_buffer_destroy(ctypes.c_void_p(int(dev_ptr))))
 
 
 def moe_nvfp4_encode(w, dst, dst_stride: int, codes_off: int, scales_off: int, global_off: int,

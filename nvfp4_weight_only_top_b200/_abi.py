@@ -25,6 +25,10 @@ PATH_AUTO = 0
 PATH_DECODE = 1
 PATH_PREFILL = 2
 
+EP_EXPERT_MAJOR = 0
+EP_SOURCE_MAJOR = 1
+EP_HANDLE_BYTES = 64
+
 
 class Bank(ctypes.Structure):
     """moe_nvfp4_bank."""
@@ -77,6 +81,18 @@ SIGNATURES = {
     "moe_nvfp4_rows_forward": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i32, _vp, _vp]),
     "moe_nvfp4_rows_stats": (ctypes.c_int, [_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i64)]),
     "moe_nvfp4_rows_destroy": (ctypes.c_int, [_vp]),
+    "moe_nvfp4_experts": (ctypes.c_int, [_vp, _vp, _i64, _BANKP, _vp, _vp, _sz, _i32, _vp]),
+    "moe_nvfp4_experts_workspace_bytes": (ctypes.c_size_t, [_i64, _i32, _i32, _i32, _i32]),
+    "moe_nvfp4_ep_plan": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _i64, _vp]),
+    "moe_nvfp4_ep_dispatch": (ctypes.c_int, [_vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _i64, _vp]),
+    "moe_nvfp4_ep_combine": (ctypes.c_int, [_vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i64,
+                                            _vp, _vp, _vp]),
+    "moe_nvfp4_gather_rows": (ctypes.c_int, [_vp, _vp, _i64, _i32, _i32, _vp, _vp]),
+    "moe_nvfp4_combine": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp]),
+    "moe_nvfp4_ep_buffer_create": (ctypes.c_int, [_u64, ctypes.POINTER(_vp), _vp]),
+    "moe_nvfp4_ep_buffer_open": (ctypes.c_int, [_vp, ctypes.POINTER(_vp)]),
+    "moe_nvfp4_ep_buffer_close": (ctypes.c_int, [_vp]),
+    "moe_nvfp4_ep_buffer_destroy": (ctypes.c_int, [_vp]),
     "moe_nvfp4_last_error": (ctypes.c_char_p, []),
     "moe_nvfp4_device_status": (ctypes.c_int, []),
     "moe_nvfp4_last_launch_count": (ctypes.c_int, []),

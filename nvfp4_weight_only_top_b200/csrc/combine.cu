@@ -55,6 +55,21 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   }
 }
 
+// Experts-only calls: y_rows[r] = y[inv[r]] (the expert output of row r, which the expert
+// kernels wrote at its place in expert order), zero for padding rows (id < 0).
+__global__ void __launch_bounds__(256) unpermute_kernel(const float* __restrict__ y, const int32_t* __restrict__ inv,
+                                                        const int32_t* __restrict__ ids, int64_t R, int H,
+                                                        float* __restrict__ y_rows) {
+  const int per_row = H / 4;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= R * per_row) return;
+  const int64_t r = idx / per_row;
+  const int c = (int)(idx - r * per_row) * 4;
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (ids[r] >= 0) v = *reinterpret_cast<const float4*>(y + (size_t)inv[r] * H + c);
+  *reinterpret_cast<float4*>(y_rows + (size_t)r * H + c) = v;
+}
+
 }  // namespace
 
 int launch_combine(const float* y, const float* w, const int32_t* inv, int64_t T, int k, int H,
@@ -62,6 +77,14 @@ int launch_combine(const float* y, const float* w, const int32_t* inv, int64_t T
   const int64_t n = T * (H / 8);
   const int blocks = (int)((n + 255) / 256);
   combine_kernel<<<blocks, 256, 0, s>>>(y, w, inv, T, k, H, x, out, x_next);
+  const cudaError_t err = cudaGetLastError();
+  return err == cudaSuccess ? 1 : -(int)err;
+}
+
+int launch_unpermute(const float* y, const int32_t* inv, const int32_t* ids, int64_t R, int H, float* y_rows,
+                     cudaStream_t s) {
+  const int64_t n = R * (H / 4);
+  unpermute_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(y, inv, ids, R, H, y_rows);
   const cudaError_t err = cudaGetLastError();
   return err == cudaSuccess ? 1 : -(int)err;
 }

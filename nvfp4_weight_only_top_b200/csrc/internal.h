@@ -41,6 +41,11 @@ inline int64_t max_groups(int64_t R, int E, int group_rows) {
 int launch_route(const float* logits, int64_t T, int E, int k, const RouteBufs& b,
                  cudaStream_t s);
 
+// Routing of rows whose expert ids are given (k = 1, weights 1): ids [R] of the caller; ids
+// outside [0, E) mark padding rows, placed after all expert rows and in no group.  chunk_counts
+// must hold route_chunks(R) * (E + 1) ints.  Returns the number of kernels launched.
+int launch_route_ids(const int32_t* rows, int64_t R, int E, const RouteBufs& b, cudaStream_t s);
+
 struct BankView {
   const uint8_t* base;
   uint64_t stride;
@@ -68,6 +73,9 @@ int launch_rows_down(const BankView& bank, const float* h, const RouteBufs& rb, 
 int launch_combine(const float* y, const float* w, const int32_t* inv, int64_t T, int k, int H,
                    const uint16_t* x, uint16_t* out, uint16_t* x_next, cudaStream_t s);
 
+// y_rows [R, H] f32 = y[inv[r]] for rows with ids[r] >= 0, zero for the others.
+int launch_unpermute(const float* y, const int32_t* inv, const int32_t* ids, int64_t R, int H, float* y_rows,
+                     cudaStream_t s);
 size_t decode_smem_bytes(int K, int xrows, bool gateup);
 
 // Decode of larger batches on the router's groups (up to 8 routed rows of one expert, group_rows
@@ -146,6 +154,20 @@ int launch_w4a4_gateup(const BankView& bank, const float* act_scales, const uint
 int launch_w4a4_down(const BankView& bank, const float* act_scales, const uint8_t* h_codes, const uint8_t* h_scales,
                      int64_t R, const RouteBufs& rb, float* y, unsigned* tile_ctr, int num_sms, cudaStream_t s);
 
+// Expert parallelism over peer memory (ep.cu).  Ranks G <= kEpMaxRanks; the plan writes dst_off [E]
+// and recv_ids [recv_rows]; dispatch and combine take G peer pointers (host array).
+constexpr int kEpMaxRanks = 64;
+size_t ep_plan_smem_bytes(int G, int E);
+int launch_ep_plan(const int32_t* C, int G, int E, int rank, int layout, int32_t* dst_off, int32_t* recv_ids,
+                   int64_t recv_rows, cudaStream_t s);
+bool ep_move_supported(int H);
+int launch_ep_dispatch(const uint16_t* x, int64_t R, int k, int H, const int32_t* ids, const int32_t* perm,
+                       const int32_t* offsets, const int32_t* dst_off, int El, int64_t cap, void* const* recv, int G,
+                       int num_sms, cudaStream_t s);
+int launch_ep_combine(int64_t T, int k, int H, const int32_t* ids, const float* w, const int32_t* inv,
+                      const int32_t* offsets, const int32_t* dst_off, int El, int64_t cap, const float* const* ys,
+                      int G, const uint16_t* x, uint16_t* out, uint16_t* x_next, cudaStream_t s);
+
 // Tiled tensor map over a byte tensor of the given rank (dims innermost first, strides in bytes
 // of dims 1.., box sizes); 0 or a negative cudaError_t.
 int make_tensor_map(CUtensorMap* map, int rank, const void* base, const uint64_t* dims, const uint64_t* strides,
@@ -164,6 +186,7 @@ cudaError_t set_smem_limit(const void* kernel, int bytes);
 // C-ABI bridge (moe_nvfp4.cu): status and message of the calling host thread, the current
 // device (sm_100 check, SM count).
 int api_fail(int code, const char* msg);
+void api_set_launches(int n);          // moe_nvfp4_last_launch_count of the calling thread
 int api_cuda_fail(int err, const char* what);
 int api_device(int* dev, int* sms);
 

@@ -113,7 +113,9 @@ struct WsLayout {
 
 size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-WsLayout ws_layout(int64_t T, int E, int k, int H, int I, int path) {
+// given_ids: the routing of an experts-only call (rows with given expert ids), whose chunk
+// counts carry a padding bin and exist for every R.
+WsLayout ws_layout(int64_t T, int E, int k, int H, int I, int path, bool given_ids = false) {
   (void)path;
   WsLayout L{};
   const size_t R = (size_t)T * k;
@@ -133,7 +135,8 @@ WsLayout ws_layout(int64_t T, int E, int k, int H, int I, int path) {
   L.ngroups = take(4);
   L.singles = take((size_t)E * 16);
   L.nsingles = take(4);
-  L.chunk_counts = take(T > moe::kRouteChunk ? (size_t)moe::route_chunks(T) * E * 4 : 0);
+  L.chunk_counts = take(given_ids ? (size_t)moe::route_chunks(T) * (E + 1) * 4
+                                  : T > moe::kRouteChunk ? (size_t)moe::route_chunks(T) * E * 4 : 0);
   L.bar = take(2 * sizeof(unsigned));        // tile counters of the tensor-core path
   L.h = take(R * (size_t)I * 4);
   L.y = take(R * (size_t)H * 4);
@@ -515,6 +518,115 @@ int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
   return MOE_NVFP4_OK;
 }
 
+// Experts-only call: y_rows[r] = expert ids[r] applied to x_rows[r] (no router, no weights, no
+// combine), for expert parallelism, where a rank runs its own experts on the rows other ranks
+// sent it.  The same expert kernels as the layer: the ids router (k = 1) places the rows in
+// expert order, the tensor-core or the grouped/row kernels compute y in that order, and the
+// unpermute kernel writes each row's result back at its own index.
+int experts_impl(const void* x_rows, const int32_t* ids, int64_t R, const moe_nvfp4_bank* bank, float* y_rows,
+                 void* workspace, size_t workspace_bytes, int32_t path, void* stream) {
+  t_last_launches = 0;
+  int rc = check_bank(bank);
+  if (rc) return rc;
+  const int E = bank->num_experts, H = bank->hidden, I = bank->intermediate;
+  if ((rc = check_k_T(R, E, 1))) return rc;
+  if (path < MOE_NVFP4_PATH_AUTO || path > MOE_NVFP4_PATH_PREFILL)
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "path %d unknown", path);
+  int dev;
+  DeviceInfo info;
+  if ((rc = current_device(&dev, &info))) return rc;
+  if (R == 0) return MOE_NVFP4_OK;
+  if (!x_rows || !ids || !y_rows) return fail(MOE_NVFP4_ERR_INVALID_ARG, "x_rows, ids and y_rows must not be NULL");
+  if (!aligned(x_rows, 16) || !aligned(y_rows, 16) || !aligned(ids, 4))
+    return fail(MOE_NVFP4_ERR_INVALID_ARG, "x_rows and y_rows must be 16-byte aligned, ids 4-byte aligned");
+  const int use = resolve_path(path, R, 1, E, H, I);
+  if (use == MOE_NVFP4_PATH_PREFILL && !moe::prefill_supported(H, I))
+    return fail(MOE_NVFP4_ERR_UNSUPPORTED, "prefill path needs H %% 256 == 0 and I %% 256 == 0 (H=%d, I=%d)", H, I);
+  const int xrows = (int)(R < 8 ? R : 8);
+  if (use != MOE_NVFP4_PATH_PREFILL &&
+      (moe::decode_smem_bytes(H, xrows, true) == 0 || moe::decode_smem_bytes(I, xrows, false) == 0 ||
+       (int)moe::decode_smem_bytes(H, xrows, true) > info.smem_optin))
+    return fail(MOE_NVFP4_ERR_UNSUPPORTED, "H=%d / I=%d exceed the decode kernel's shared memory", H, I);
+  const WsLayout L = ws_layout(R, E, 1, H, I, use, true);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  if (ws) {
+    if (workspace_bytes < L.total)
+      return fail(MOE_NVFP4_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes,
+                  L.total);
+    if (!aligned(ws, 256)) return fail(MOE_NVFP4_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  } else if ((rc = ensure_workspace(dev, L.total, s, &ws))) {
+    return rc;
+  }
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  moe::RouteBufs rb = route_bufs(w8, L);
+  const moe::BankView bv = view_of(bank);
+  const uint16_t* xb = static_cast<const uint16_t*>(x_rows);
+  float* h = reinterpret_cast<float*>(w8 + L.h);
+  float* y = reinterpret_cast<float*>(w8 + L.y);
+  int launches = 0;
+  if (use == MOE_NVFP4_PATH_PREFILL) {
+    rb.group_rows = moe::kPrefillRows;
+    unsigned* tile_ctr = reinterpret_cast<unsigned*>(w8 + L.bar);
+    const cudaError_t e = cudaMemsetAsync(tile_ctr, 0, 2 * sizeof(unsigned), s);
+    if (e != cudaSuccess) return cuda_fail(e, "clear tile counters");
+    prof_before(MOE_NVFP4_KERNEL_ROUTE, s);
+    if ((rc = after_launch(moe::launch_route_ids(ids, R, E, rb, s), s, "ids route", &launches))) return rc;
+    void* xp = w8 + L.y;
+    void* hb = w8 + L.h;
+    float* colscale = reinterpret_cast<float*>(w8 + L.h + up256((size_t)R * I * 2));
+    prof_before(MOE_NVFP4_KERNEL_PREFILL_GATHER, s);
+    if ((rc = after_launch(moe::launch_gather_f16(xb, rb.perm, 1, R, H, xp, colscale, s), s, "gather", &launches)))
+      return rc;
+    const int pairs = prefill_pair_kernel() ? moe::prefill2_pairs(info.sms) : 0;
+    prof_before(MOE_NVFP4_KERNEL_PREFILL_GATEUP, s);
+    rc = pairs > 0 ? moe::launch_prefill2_gateup(bv, xp, colscale, R, rb, hb, pairs, s)
+                   : moe::launch_prefill_gateup(bv, xp, colscale, R, rb, hb, tile_ctr, info.sms, s);
+    if ((rc = after_launch(rc, s, "prefill gate/up", &launches))) return rc;
+    prof_before(MOE_NVFP4_KERNEL_PREFILL_DOWN, s);
+    rc = pairs > 0 ? moe::launch_prefill2_down(bv, hb, R, rb, y, pairs, s)
+                   : moe::launch_prefill_down(bv, hb, R, rb, y, tile_ctr + 1, info.sms, s);
+    if ((rc = after_launch(rc, s, "prefill down", &launches))) return rc;
+  } else if (moe::grouped_supported(H, I) && decode_kernel_choice() != kDecodeRows) {
+    rb.group_rows = 8;
+    rb.split_singles = 0;
+    rb.expert_major = 1;
+    prof_before(MOE_NVFP4_KERNEL_ROUTE, s);
+    if ((rc = after_launch(moe::launch_route_ids(ids, R, E, rb, s), s, "ids route", &launches))) return rc;
+    prof_before(MOE_NVFP4_KERNEL_DECODE_GATEUP, s);
+    if ((rc = after_launch(moe::launch_grouped_gateup(bv, xb, 1, rb, h, info.sms, s), s, "grouped gate/up",
+                           &launches)))
+      return rc;
+    prof_before(MOE_NVFP4_KERNEL_DECODE_DOWN, s);
+    if ((rc = after_launch(moe::launch_grouped_down(bv, h, rb, y, info.sms, s), s, "grouped down", &launches)))
+      return rc;
+  } else {
+    const bool rows = moe::rows_supported(H, true) && moe::rows_supported(I, false);
+    const bool multi = !rows || R > 1;       // groups of two or more rows exist only then
+    rb.split_singles = rows ? 1 : 0;
+    prof_before(MOE_NVFP4_KERNEL_ROUTE, s);
+    if ((rc = after_launch(moe::launch_route_ids(ids, R, E, rb, s), s, "ids route", &launches))) return rc;
+    prof_before(MOE_NVFP4_KERNEL_DECODE_GATEUP, s);
+    if (rows && (rc = after_launch(moe::launch_rows_gateup(bv, xb, 1, rb, h, info.sms, s), s, "rows gate/up",
+                                   &launches)))
+      return rc;
+    if (multi && (rc = after_launch(moe::launch_decode_gateup(bv, xb, 1, rb, xrows, h, info.sms, s), s, "decode gate/up",
+                           &launches)))
+      return rc;
+    prof_before(MOE_NVFP4_KERNEL_DECODE_DOWN, s);
+    if (rows && (rc = after_launch(moe::launch_rows_down(bv, h, rb, y, info.sms, s), s, "rows down", &launches)))
+      return rc;
+    if (multi && (rc = after_launch(moe::launch_decode_down(bv, h, rb, xrows, y, info.sms, s), s, "decode down",
+                                    &launches)))
+      return rc;
+  }
+  prof_before(MOE_NVFP4_KERNEL_COMBINE, s);
+  if ((rc = after_launch(moe::launch_unpermute(y, rb.inv, rb.ids, R, H, y_rows, s), s, "unpermute", &launches)))
+    return rc;
+  t_last_launches = launches;
+  return MOE_NVFP4_OK;
+}
+
 int ensure_stage(void** p, size_t* have, size_t need) {
   if (*have >= need) return MOE_NVFP4_OK;
   if (*p) cudaFree(*p);
@@ -655,6 +767,8 @@ cudaError_t set_smem_limit(const void* kernel, int bytes) {
 }
 
 int api_fail(int code, const char* msg) { return fail(code, "%s", msg); }
+
+void api_set_launches(int n) { t_last_launches = n; }
 
 int api_cuda_fail(int err, const char* what) { return cuda_fail((cudaError_t)err, what); }
 
@@ -929,6 +1043,16 @@ int moe_nvfp4_route(const float* logits_dev, int64_t T, int32_t E, int32_t k, in
 size_t moe_nvfp4_workspace_bytes(int64_t T, int32_t E, int32_t k, int32_t H, int32_t I, int32_t path) {
   if (T < 0 || E < 1 || E > 1024 || k < 1 || k > 32 || k > E || H < 128 || I < 128) return 0;
   return ws_layout(T, E, k, H, I, resolve_path(path, T, k, E, H, I)).total;
+}
+
+int moe_nvfp4_experts(const void* x_rows_dev, const int32_t* expert_ids_dev, int64_t R, const moe_nvfp4_bank* bank,
+                      float* y_rows_dev, void* workspace_dev, size_t workspace_bytes, int32_t path, void* stream) {
+  return experts_impl(x_rows_dev, expert_ids_dev, R, bank, y_rows_dev, workspace_dev, workspace_bytes, path, stream);
+}
+
+size_t moe_nvfp4_experts_workspace_bytes(int64_t R, int32_t E, int32_t H, int32_t I, int32_t path) {
+  if (R < 0 || E < 1 || E > 1024 || H < 128 || I < 128) return 0;
+  return ws_layout(R, E, 1, H, I, resolve_path(path, R, 1, E, H, I), true).total;
 }
 
 const char* moe_nvfp4_last_error(void) { return t_last_error.c_str(); }

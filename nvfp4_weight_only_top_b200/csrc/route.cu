@@ -199,6 +199,73 @@ __global__ void __launch_bounds__(32) route_scatter_kernel(int64_t T, int E, int
   }
 }
 
+// Rows with given expert ids (k = 1), step 1: this chunk's rows per bin, bins 0 .. E-1 for the
+// experts and bin E for rows whose id lies outside [0, E) (padding rows).
+__global__ void __launch_bounds__(256) ids_count_kernel(const int32_t* __restrict__ rows, int64_t R, int E,
+                                                        RouteBufs b) {
+  __shared__ int cnt[kMaxE + 1];
+  const int64_t r0 = (int64_t)blockIdx.x * kRouteChunk;
+  const int nr = (int)(R - r0 < kRouteChunk ? R - r0 : kRouteChunk);
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < nr; i += blockDim.x) {
+    const int id = rows[r0 + i];
+    const bool ok = id >= 0 && id < E;
+    b.ids[r0 + i] = ok ? id : -1;
+    b.w[r0 + i] = 1.0f;
+    atomicAdd(&cnt[ok ? id : E], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e <= E; e += blockDim.x)
+    b.chunk_counts[(size_t)blockIdx.x * (E + 1) + e] = cnt[e];
+}
+
+// Step 2 (one CTA): per-bin prefix over chunks, then counts, offsets and groups of the experts;
+// the padding bin's chunk prefixes are left in chunk_counts and its rows go after all expert
+// rows (offsets[E] is the number of expert rows).
+__global__ void __launch_bounds__(1024) ids_scan_kernel(int nchunks, int E, RouteBufs b) {
+  __shared__ int cnt[kMaxE], tmp[kMaxE], tmp1[kMaxE], tmp2[kMaxE], warp_tmp[32];
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    int run = 0;
+    for (int c = 0; c < nchunks; ++c) {
+      int* p = b.chunk_counts + (size_t)c * (E + 1) + e;
+      const int v = *p;
+      *p = run;
+      run += v;
+    }
+    if (e < E) cnt[e] = run;
+  }
+  __syncthreads();
+  finish_counts(cnt, tmp, tmp1, tmp2, warp_tmp, E, b.group_rows, b);
+}
+
+// Step 3: stable placement of the chunk's rows, expert rows by expert, padding rows at the end.
+__global__ void __launch_bounds__(32) ids_scatter_kernel(int64_t R, int E, RouteBufs b) {
+  __shared__ int run[kMaxE + 1];
+  const int lane = threadIdx.x;
+  const int64_t r0 = (int64_t)blockIdx.x * kRouteChunk;
+  const int nr = (int)(R - r0 < kRouteChunk ? R - r0 : kRouteChunk);
+  for (int e = lane; e <= E; e += 32)
+    run[e] = b.offsets[e] + b.chunk_counts[(size_t)blockIdx.x * (E + 1) + e];
+  __syncwarp();
+  for (int i = 0; i < nr; i += 32) {
+    // one row per lane, placed in row order: lanes with the same bin take consecutive slots
+    const int64_t r = r0 + i + lane;
+    const bool have = i + lane < nr;
+    const int id = have ? b.ids[r] : 0;
+    const int bin = id < 0 ? E : id;
+    for (int l = 0; l < 32; ++l) {
+      if (lane == l && have) {
+        const int pos = run[bin];
+        run[bin] = pos + 1;
+        b.perm[pos] = (int32_t)r;
+        b.inv[r] = pos;
+      }
+      __syncwarp();
+    }
+  }
+}
+
 }  // namespace
 
 int launch_route(const float* logits, int64_t T, int E, int k, const RouteBufs& b,
@@ -212,6 +279,15 @@ int launch_route(const float* logits, int64_t T, int E, int k, const RouteBufs& 
   route_chunk_kernel<<<nch, 256, 0, s>>>(logits, T, E, k, b);
   route_scan_kernel<<<1, 1024, 0, s>>>(nch, E, b);
   route_scatter_kernel<<<nch, 32, 0, s>>>(T, E, k, b);
+  const cudaError_t err = cudaGetLastError();
+  return err == cudaSuccess ? 3 : -(int)err;
+}
+
+int launch_route_ids(const int32_t* rows, int64_t R, int E, const RouteBufs& b, cudaStream_t s) {
+  const int nch = route_chunks(R);
+  ids_count_kernel<<<nch, 256, 0, s>>>(rows, R, E, b);
+  ids_scan_kernel<<<1, 1024, 0, s>>>(nch, E, b);
+  ids_scatter_kernel<<<nch, 32, 0, s>>>(R, E, b);
   const cudaError_t err = cudaGetLastError();
   return err == cudaSuccess ? 3 : -(int)err;
 }
