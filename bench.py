@@ -610,6 +610,101 @@ def measure_w4a4(cfg, steps: int, warm: int) -> dict:
             "gpu_launches": launches * reps * gsteps}
 
 
+NVLINK_GBS = 770.0      # measured peer copy per direction per GPU on this machine's B200s (NVLink 5)
+
+
+def measure_ep(cfg, G: int = 8, steps: int = 10, warm: int = 3) -> dict:
+    """Expert parallelism over G ranks (each rank the workload's T tokens, E/G experts), emulated
+    on one GPU: every rank's buffers live on this device and the peer pointers are local, so the
+    dispatch and combine kernels move the rows through HBM here instead of NVLink.  Times rank
+    0's step (dispatch of its routed rows, its experts on the rows it receives, its combine) with
+    CUDA events; the other ranks' dispatches and experts run once, untimed, so that rank 0
+    receives and reads back real data.  Reports each kernel against the HBM peak and the time
+    the same bytes would take over NVLink at the measured peer-copy bandwidth."""
+    import torch
+    import nvfp4_weight_only_top_b200 as moe
+    from nvfp4_weight_only_top_b200 import ep
+    from moe_inputs import device as mdev
+    lay = cfg.layout
+    s = torch.cuda.Stream()
+    torch.cuda.set_stream(s)
+    buf = mdev.bank_tensor(lay, cfg.seed, 0)
+    bank = moe.make_bank(buf.data_ptr(), lay.E, lay.H, lay.I, lay.record_stride, lay.codes_off, lay.scales_off,
+                         lay.global_off, 0)
+    H, k, T = cfg.H, cfg.k, cfg.T
+    xs, routes = [], []
+    for r in range(G):
+        xs.append(torch.from_numpy(moe_inputs.make_x(cfg, seed=cfg.seed + r).view(np.int16)).view(
+            torch.bfloat16).cuda())
+        lg = torch.from_numpy(moe_inputs.make_logits(cfg, seed=cfg.seed + r)).cuda()
+        routes.append(moe.moe_nvfp4_route(lg, k))
+    C = torch.stack([rt["counts"] for rt in routes]).contiguous()
+    plans = [ep.plan(C.cpu().numpy(), r) for r in range(G)]
+    cap = max(plans[0]["recv_totals"])
+    recv_x = [torch.empty((cap, H), dtype=torch.bfloat16, device="cuda") for _ in range(G)]
+    recv_y = [torch.empty((cap, H), dtype=torch.float32, device="cuda") for _ in range(G)]
+    xp, yp = [t.data_ptr() for t in recv_x], [t.data_ptr() for t in recv_y]
+    plan_dev = [moe.moe_nvfp4_ep_plan(C, r, plans[r]["recv_total"], moe.EP_EXPERT_MAJOR) for r in range(G)]
+    shards = [ep.shard_bank(bank, r, G) for r in range(G)]
+    Rr = [p["recv_total"] for p in plans]
+    wsb = [torch.empty(moe.moe_nvfp4_experts_workspace_bytes(Rr[r], cfg.E // G, H, cfg.I), dtype=torch.uint8,
+                       device="cuda") for r in range(G)]
+    for r in range(G):
+        moe.moe_nvfp4_ep_dispatch(xs[r], routes[r], plan_dev[r][0], xp, cap)
+    for r in range(G):
+        moe.moe_nvfp4_experts(recv_x[r][:Rr[r]], plan_dev[r][1], shards[r], y_rows=recv_y[r][:Rr[r]],
+                              workspace=wsb[r], sorted_ids=True)
+    out = torch.empty_like(xs[0])
+
+    def step():
+        moe.moe_nvfp4_ep_dispatch(xs[0], routes[0], plan_dev[0][0], xp, cap)
+        ev[1].record(s)
+        moe.moe_nvfp4_experts(recv_x[0][:Rr[0]], plan_dev[0][1], shards[0], y_rows=recv_y[0][:Rr[0]],
+                              workspace=wsb[0], sorted_ids=True)
+        ev[2].record(s)
+        moe.moe_nvfp4_ep_combine(routes[0], plan_dev[0][0], yp, H, cap, out=out)
+
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for _ in range(warm):
+        ev[0].record(s)
+        step()
+        ev[3].record(s)
+    torch.cuda.synchronize()
+    parts = np.zeros(3)
+    total = 0.0
+    moe.moe_nvfp4_profile_begin()
+    for _ in range(steps):
+        ev[0].record(s)
+        step()
+        ev[3].record(s)
+        torch.cuda.synchronize()
+        parts += [ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]), ev[2].elapsed_time(ev[3])]
+        total += ev[0].elapsed_time(ev[3])
+    prof = moe.moe_nvfp4_profile_end()
+    assert moe.moe_nvfp4_device_status() == 0
+    parts /= steps
+    ms = total / steps
+    hbm, tf_burst, tf_sus, peak_kind = load_peaks()
+    R = T * k
+    disp_bytes = 2.0 * R * H * 2                     # each routed row read once and stored once
+    comb_bytes = R * H * 4.0 + T * H * 2.0           # every result row read, the output written
+    remote = (G - 1) / G                             # share of rows whose owner is another GPU
+    flops = 2.0 * Rr[0] * 3 * H * cfg.I
+    return {"metric": "MoE-layer tok/s per GPU (expert parallel, emulated on one GPU)", "value": T / (ms / 1000.0),
+            "unit": "tok/s", "ms_per_step": ms, "steps": steps, "warmup": warm, "dtype": "bf16",
+            "config": dict(workload_config(cfg), parallelism=f"ep{G} emulated on 1 GPU", tokens_per_rank=T,
+                           experts_per_rank=cfg.E // G, rows_received=Rr[0]),
+            "kernels_ms": {"dispatch": parts[0], "experts": parts[1], "combine": parts[2]},
+            "experts_kernels_ms": {k_: v[0] / steps for k_, v in prof.items()},
+            "dispatch": {"bytes": disp_bytes, "GB/s": disp_bytes / parts[0] / 1e6, "hbm_frac": disp_bytes / parts[0]
+                         / 1e6 / hbm, "nvlink_ms": remote * R * H * 2 / (NVLINK_GBS * 1e6)},
+            "combine": {"bytes": comb_bytes, "GB/s": comb_bytes / parts[2] / 1e6, "hbm_frac": comb_bytes / parts[2]
+                        / 1e6 / hbm, "nvlink_ms": remote * R * H * 4 / (NVLINK_GBS * 1e6)},
+            "experts_tflops": flops / (parts[1] / 1000.0) / 1e12,
+            "experts_tflops_frac": flops / (parts[1] / 1000.0) / 1e12 / tf_burst,
+            "peaks": {"hbm_gbs": hbm, "bf16_tflops": tf_burst, "kind": peak_kind, "nvlink_gbs": NVLINK_GBS}}
+
+
 def measure_encoder(experts: int = 16, reps: int = 5) -> dict:
     """NVFP4 encoding of `experts` full-size BF16 experts (gate and up [2560, 5120], down
     [5120, 2560]) into bank records; HBM-bound.  The algorithmic minimum is one read of the BF16
@@ -787,6 +882,8 @@ def main():
     if (not args.config or args.config == "prefill_t8192") and rank == 0:
         cfg = moe_inputs.CONFIGS["prefill_t8192"]
         variants["w4a4_prefill_t8192"] = measure_w4a4(cfg, MIN_STEPS["prefill_t8192"] * 2, 3)
+        torch.cuda.empty_cache()
+        variants["ep8_prefill_t8192"] = measure_ep(cfg, 8, MIN_STEPS["prefill_t8192"], 3)
         torch.cuda.empty_cache()
     comps = {}
     if not args.config and rank == 0:

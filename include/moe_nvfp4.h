@@ -223,11 +223,15 @@ int moe_nvfp4_route(const float* logits_dev, int64_t T, int32_t E, int32_t k, in
  * layer (path as in moe_nvfp4_forward_ex with T = R, k = 1): for a row, the result is the one
  * the layer computes for that row and expert on the same path.  workspace_dev: NULL for the
  * internal workspace, else at least moe_nvfp4_experts_workspace_bytes(...) bytes, 256-byte
- * aligned.  R = 0 returns OK.
+ * aligned.  R = 0 returns OK.  flags: 0, or MOE_NVFP4_EXPERTS_SORTED when the caller knows the
+ * ids are non-decreasing and all in [0, E) (rows already in expert order, as an expert-major
+ * receive buffer holds them): the results are then written in place, saving one pass over y
+ * (with unsorted ids the flag leaves rows in the wrong places, within y_rows).
  */
+#define MOE_NVFP4_EXPERTS_SORTED 1
 int moe_nvfp4_experts(const void* x_rows_dev, const int32_t* expert_ids_dev, int64_t R,
                       const moe_nvfp4_bank* bank, float* y_rows_dev, void* workspace_dev,
-                      size_t workspace_bytes, int32_t path, void* stream);
+                      size_t workspace_bytes, int32_t path, int32_t flags, void* stream);
 size_t moe_nvfp4_experts_workspace_bytes(int64_t R, int32_t E, int32_t H, int32_t I,
                                          int32_t path);
 

@@ -207,9 +207,10 @@ def moe_nvfp4_route(logits, k: int, stream=None) -> dict:
 
 
 def moe_nvfp4_experts(x_rows, expert_ids, bank: Bank, y_rows=None, workspace=None, path: int = PATH_AUTO,
-                      stream=None):
+                      sorted_ids: bool = False, stream=None):
     """y_rows [R, H] f32 = expert expert_ids[r] applied to x_rows[r] (bf16 [R, H]); ids outside
-    [0, E) are padding rows (zero output)."""
+    [0, E) are padding rows (zero output).  sorted_ids: the caller knows the ids are
+    non-decreasing and all valid (MOE_NVFP4_EXPERTS_SORTED)."""
     import torch
     if not isinstance(x_rows, torch.Tensor) or x_rows.dim() != 2:
         raise ValueError("x_rows must be a 2-D torch tensor [R, H]")
@@ -226,7 +227,8 @@ def moe_nvfp4_experts(x_rows, expert_ids, bank: Bank, y_rows=None, workspace=Non
         _need(*args)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().moe_nvfp4_experts(_ptr(x_rows), _ptr(expert_ids), R, ctypes.byref(bank), _ptr(y_rows),
-                                   _ptr(workspace), ws_bytes, path, _stream(stream)))
+                                   _ptr(workspace), ws_bytes, path, _abi.EXPERTS_SORTED if sorted_ids else 0,
+                                   _stream(stream)))
     return y_rows
 
 

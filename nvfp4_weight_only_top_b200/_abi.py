@@ -28,6 +28,7 @@ PATH_PREFILL = 2
 EP_EXPERT_MAJOR = 0
 EP_SOURCE_MAJOR = 1
 EP_HANDLE_BYTES = 64
+EXPERTS_SORTED = 1
 
 
 class Bank(ctypes.Structure):
@@ -81,7 +82,7 @@ SIGNATURES = {
     "moe_nvfp4_rows_forward": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i32, _vp, _vp]),
     "moe_nvfp4_rows_stats": (ctypes.c_int, [_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i64)]),
     "moe_nvfp4_rows_destroy": (ctypes.c_int, [_vp]),
-    "moe_nvfp4_experts": (ctypes.c_int, [_vp, _vp, _i64, _BANKP, _vp, _vp, _sz, _i32, _vp]),
+    "moe_nvfp4_experts": (ctypes.c_int, [_vp, _vp, _i64, _BANKP, _vp, _vp, _sz, _i32, _i32, _vp]),
     "moe_nvfp4_experts_workspace_bytes": (ctypes.c_size_t, [_i64, _i32, _i32, _i32, _i32]),
     "moe_nvfp4_ep_plan": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _i64, _vp]),
     "moe_nvfp4_ep_dispatch": (ctypes.c_int, [_vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _i64, _vp]),

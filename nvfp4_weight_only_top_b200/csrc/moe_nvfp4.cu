@@ -524,7 +524,7 @@ int forward_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
 // expert order, the tensor-core or the grouped/row kernels compute y in that order, and the
 // unpermute kernel writes each row's result back at its own index.
 int experts_impl(const void* x_rows, const int32_t* ids, int64_t R, const moe_nvfp4_bank* bank, float* y_rows,
-                 void* workspace, size_t workspace_bytes, int32_t path, void* stream) {
+                 void* workspace, size_t workspace_bytes, int32_t path, int32_t flags, void* stream) {
   t_last_launches = 0;
   int rc = check_bank(bank);
   if (rc) return rc;
@@ -532,6 +532,8 @@ int experts_impl(const void* x_rows, const int32_t* ids, int64_t R, const moe_nv
   if ((rc = check_k_T(R, E, 1))) return rc;
   if (path < MOE_NVFP4_PATH_AUTO || path > MOE_NVFP4_PATH_PREFILL)
     return fail(MOE_NVFP4_ERR_INVALID_ARG, "path %d unknown", path);
+  if (flags & ~MOE_NVFP4_EXPERTS_SORTED) return fail(MOE_NVFP4_ERR_INVALID_ARG, "flags 0x%x unknown", flags);
+  const bool sorted = (flags & MOE_NVFP4_EXPERTS_SORTED) != 0;
   int dev;
   DeviceInfo info;
   if ((rc = current_device(&dev, &info))) return rc;
@@ -563,7 +565,9 @@ int experts_impl(const void* x_rows, const int32_t* ids, int64_t R, const moe_nv
   const moe::BankView bv = view_of(bank);
   const uint16_t* xb = static_cast<const uint16_t*>(x_rows);
   float* h = reinterpret_cast<float*>(w8 + L.h);
-  float* y = reinterpret_cast<float*>(w8 + L.y);
+  // Rows already in expert order: the router's permutation is the identity, so the down
+  // kernels write each row's result in place and no unpermute follows.
+  float* y = sorted ? y_rows : reinterpret_cast<float*>(w8 + L.y);
   int launches = 0;
   if (use == MOE_NVFP4_PATH_PREFILL) {
     rb.group_rows = moe::kPrefillRows;
@@ -620,9 +624,11 @@ int experts_impl(const void* x_rows, const int32_t* ids, int64_t R, const moe_nv
                                     &launches)))
       return rc;
   }
-  prof_before(MOE_NVFP4_KERNEL_COMBINE, s);
-  if ((rc = after_launch(moe::launch_unpermute(y, rb.inv, rb.ids, R, H, y_rows, s), s, "unpermute", &launches)))
-    return rc;
+  if (!sorted) {
+    prof_before(MOE_NVFP4_KERNEL_COMBINE, s);
+    if ((rc = after_launch(moe::launch_unpermute(y, rb.inv, rb.ids, R, H, y_rows, s), s, "unpermute", &launches)))
+      return rc;
+  }
   t_last_launches = launches;
   return MOE_NVFP4_OK;
 }
@@ -1046,8 +1052,10 @@ size_t moe_nvfp4_workspace_bytes(int64_t T, int32_t E, int32_t k, int32_t H, int
 }
 
 int moe_nvfp4_experts(const void* x_rows_dev, const int32_t* expert_ids_dev, int64_t R, const moe_nvfp4_bank* bank,
-                      float* y_rows_dev, void* workspace_dev, size_t workspace_bytes, int32_t path, void* stream) {
-  return experts_impl(x_rows_dev, expert_ids_dev, R, bank, y_rows_dev, workspace_dev, workspace_bytes, path, stream);
+                      float* y_rows_dev, void* workspace_dev, size_t workspace_bytes, int32_t path, int32_t flags,
+                      void* stream) {
+  return experts_impl(x_rows_dev, expert_ids_dev, R, bank, y_rows_dev, workspace_dev, workspace_bytes, path, flags,
+                      stream);
 }
 
 size_t moe_nvfp4_experts_workspace_bytes(int64_t R, int32_t E, int32_t H, int32_t I, int32_t path) {

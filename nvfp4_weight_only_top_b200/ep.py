@@ -116,9 +116,9 @@ class CudaOps:
         from . import moe_nvfp4_ep_plan
         return moe_nvfp4_ep_plan(counts_all, rank, recv_rows, layout)
 
-    def experts(self, rows, ids, shard, y=None, path=_abi.PATH_AUTO):
+    def experts(self, rows, ids, shard, y=None, path=_abi.PATH_AUTO, sorted_ids=False):
         from . import moe_nvfp4_experts
-        return moe_nvfp4_experts(rows, ids, shard, y_rows=y, path=path)
+        return moe_nvfp4_experts(rows, ids, shard, y_rows=y, path=path, sorted_ids=sorted_ids)
 
     def combine(self, y, w, inv, k, x=None, x_next=None):
         from . import moe_nvfp4_combine
@@ -273,7 +273,7 @@ class ExpertParallel:
         dst_off, ids = self.ops.recv_plan(C, self.rank, Rr, _abi.EP_EXPERT_MAJOR)
         self.ops.dispatch(x, r, dst_off, self.recv_x_ptrs, self.capacity)
         self._barrier()                  # every row has reached its owner
-        self.ops.experts(self._recv_x[:Rr], ids, self.shard, y=self._recv_y[:Rr], path=self.path)
+        self.ops.experts(self._recv_x[:Rr], ids, self.shard, y=self._recv_y[:Rr], path=self.path, sorted_ids=True)
         self._barrier()                  # every owner's results are ready
         return self.ops.peer_combine(r, dst_off, self.recv_y_ptrs, self.H, self.capacity, x=x, x_next=x_next)
 

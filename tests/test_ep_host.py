@@ -116,7 +116,7 @@ class OracleOps:
         assert pl["recv_total"] == recv_rows
         return torch.from_numpy(pl[f"dst_off_{key}"]), torch.from_numpy(pl[f"recv_ids_{key}"])
 
-    def experts(self, rows, ids, shard, y=None, path=0):
+    def experts(self, rows, ids, shard, y=None, path=0, sorted_ids=False):
         import torch
         first = int(shard.base_dev or 0) // int(shard.record_stride)
         out = np.zeros(tuple(rows.shape))

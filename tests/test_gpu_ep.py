@@ -68,6 +68,22 @@ def test_experts_empty_and_single_row():
         assert_layer_close(y.cpu().numpy().astype(np.float64), ref, f"single row, expert {e}")
 
 
+@pytest.mark.parametrize("path", [1, 2])
+def test_experts_sorted_flag_writes_in_place_bitwise(path):
+    """Rows in expert order with MOE_NVFP4_EXPERTS_SORTED: the same results as without it."""
+    import torch
+    moe = _moe()
+    cfg = moe_inputs.LayerConfig(name="experts_sorted", E=16, k=1, H=512, I=256, T=260, seed=5)
+    buf, bank = device_bank(cfg)
+    x = bf16_tensor(moe_inputs.make_x(cfg))
+    ids = torch.from_numpy(np.sort(np.random.default_rng(1).integers(0, 16, 260)).astype(np.int32)).cuda()
+    ids[:30] = 0                                          # a long first segment
+    a = moe.moe_nvfp4_experts(x, ids, bank, path=path)
+    b = moe.moe_nvfp4_experts(x, ids, bank, path=path, sorted_ids=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
 @pytest.mark.parametrize("path,T", [(2, 300), (1, 40)])
 def test_layer_equals_gather_experts_combine_bitwise(path, T):
     """The layer = its router, the gather of the routed rows, the experts on them and the
@@ -150,7 +166,8 @@ def _emulated_peer_step(moe, ep, bank, cfg, ranks, path):
         moe.moe_nvfp4_ep_dispatch(x, routes[s], dsts[s], xp, cap)
     for d in range(G):
         Rr = plans[d]["recv_total"]
-        moe.moe_nvfp4_experts(recv_x[d][:Rr], ids[d], ep.shard_bank(bank, d, G), y_rows=recv_y[d][:Rr], path=path)
+        moe.moe_nvfp4_experts(recv_x[d][:Rr], ids[d], ep.shard_bank(bank, d, G), y_rows=recv_y[d][:Rr], path=path,
+                              sorted_ids=True)
     outs, nexts = [], []
     for s, (x, _, _, _) in enumerate(ranks):
         nx = torch.empty_like(x)
