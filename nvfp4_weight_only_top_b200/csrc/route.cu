@@ -54,6 +54,51 @@ __device__ int block_scan_excl(int* a, int n, int* warp_tmp) {
   return total;
 }
 
+// Stable placement of rows r0 .. r0+n-1 (n <= 32, one per lane, bins from bin_of) by one warp:
+// lanes with the same bin take consecutive slots in lane order, from run[bin] on, and the
+// lowest lane of each bin advances run[bin] for the next call.
+template <typename BinOf>
+__device__ __forceinline__ void place32(int64_t r0, int n, int lane, int* run, const RouteBufs& b, BinOf bin_of) {
+  const bool have = lane < n;
+  const unsigned act = __ballot_sync(kFull, have);
+  if (have) {
+    const int64_t r = r0 + lane;
+    const int bin = bin_of(r);
+    const unsigned peers = __match_any_sync(act, bin);
+    const unsigned below = peers & ((1u << lane) - 1u);
+    const int pos = run[bin] + __popc(below);
+    b.perm[pos] = (int32_t)r;
+    b.inv[r] = pos;
+    __syncwarp(act);
+    if (below == 0u) run[bin] += __popc(peers);
+  }
+  __syncwarp();
+}
+
+// Per-bin exclusive prefix over chunks, in place in chunk_counts ([nchunks][stride]); returns
+// bin e's total.  Loads go out 16 at a time so that their latencies overlap.
+__device__ __forceinline__ int chunk_prefix(int32_t* cc, int nchunks, int stride, int e) {
+  int run = 0;
+  int c = 0;
+  for (; c + 16 <= nchunks; c += 16) {
+    int v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = cc[(size_t)(c + i) * stride + e];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      cc[(size_t)(c + i) * stride + e] = run;
+      run += v[i];
+    }
+  }
+  for (; c < nchunks; ++c) {
+    int* p = cc + (size_t)c * stride + e;
+    const int v = *p;
+    *p = run;
+    run += v;
+  }
+  return run;
+}
+
 // From per-expert counts in shared memory: offsets and the two group lists.  An expert's rows
 // are cut into groups of group_rows; when split_singles is set, a last group of a single row
 // goes to the one-row list instead.  All full groups (exactly group_rows rows) come first, in
@@ -98,7 +143,7 @@ __device__ void finish_counts(int* cnt, int* tmp, int* tmp1, int* tmp2, int* war
 }
 
 // Single-CTA routing for T <= kRouteChunk: router, histogram, scan, groups, stable scatter.
-__global__ void __launch_bounds__(512) route_small_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(1024) route_small_kernel(const float* __restrict__ logits,
                                                           int T, int E, int k, RouteBufs b) {
   __shared__ int cnt[kMaxE], tmp[kMaxE], tmp1[kMaxE], tmp2[kMaxE], run[kMaxE], warp_tmp[32];
   __shared__ int sids[kRouteChunk * 32];
@@ -122,21 +167,14 @@ __global__ void __launch_bounds__(512) route_small_kernel(const float* __restric
   for (int e = threadIdx.x; e < E; e += blockDim.x) run[e] = cnt[e];   // cnt now = offsets
   __syncthreads();
   if (wid == 0) {
-    for (int t = 0; t < T; ++t) {
-      if (lane < k) {
-        const int r = t * k + lane, e = sids[r];
-        const int pos = run[e];
-        run[e] = pos + 1;
-        b.perm[pos] = r;
-        b.inv[r] = pos;
-      }
-      __syncwarp();
-    }
+    const int R = T * k;
+    for (int r0 = 0; r0 < R; r0 += 32)
+      place32(r0, min(32, R - r0), lane, run, b, [&](int64_t r) { return sids[r]; });
   }
 }
 
 // Multi-CTA routing, step 1: route the chunk's tokens and count its rows per expert.
-__global__ void __launch_bounds__(256) route_chunk_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(512) route_chunk_kernel(const float* __restrict__ logits,
                                                           int64_t T, int E, int k, RouteBufs b) {
   __shared__ int cnt[kMaxE];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -163,16 +201,7 @@ __global__ void __launch_bounds__(256) route_chunk_kernel(const float* __restric
 // Multi-CTA routing, step 2 (one CTA): per-expert prefix over chunks, counts, offsets, groups.
 __global__ void __launch_bounds__(1024) route_scan_kernel(int nchunks, int E, RouteBufs b) {
   __shared__ int cnt[kMaxE], tmp[kMaxE], tmp1[kMaxE], tmp2[kMaxE], warp_tmp[32];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = 0;
-    for (int c = 0; c < nchunks; ++c) {
-      int* p = b.chunk_counts + (size_t)c * E + e;
-      const int v = *p;
-      *p = run;
-      run += v;
-    }
-    cnt[e] = run;
-  }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = chunk_prefix(b.chunk_counts, nchunks, E, e);
   __syncthreads();
   finish_counts(cnt, tmp, tmp1, tmp2, warp_tmp, E, b.group_rows, b);
 }
@@ -186,17 +215,9 @@ __global__ void __launch_bounds__(32) route_scatter_kernel(int64_t T, int E, int
   for (int e = lane; e < E; e += 32)
     run[e] = b.offsets[e] + b.chunk_counts[(size_t)blockIdx.x * E + e];
   __syncwarp();
-  for (int i = 0; i < nt; ++i) {
-    if (lane < k) {
-      const int64_t r = (t0 + i) * k + lane;
-      const int e = b.ids[r];
-      const int pos = run[e];
-      run[e] = pos + 1;
-      b.perm[pos] = (int32_t)r;
-      b.inv[r] = pos;
-    }
-    __syncwarp();
-  }
+  const int64_t r_begin = t0 * k, n = (int64_t)nt * k;
+  for (int64_t i = 0; i < n; i += 32)
+    place32(r_begin + i, (int)min((int64_t)32, n - i), lane, run, b, [&](int64_t r) { return b.ids[r]; });
 }
 
 // Rows with given expert ids (k = 1), step 1: this chunk's rows per bin, bins 0 .. E-1 for the
@@ -226,13 +247,7 @@ __global__ void __launch_bounds__(256) ids_count_kernel(const int32_t* __restric
 __global__ void __launch_bounds__(1024) ids_scan_kernel(int nchunks, int E, RouteBufs b) {
   __shared__ int cnt[kMaxE], tmp[kMaxE], tmp1[kMaxE], tmp2[kMaxE], warp_tmp[32];
   for (int e = threadIdx.x; e <= E; e += blockDim.x) {
-    int run = 0;
-    for (int c = 0; c < nchunks; ++c) {
-      int* p = b.chunk_counts + (size_t)c * (E + 1) + e;
-      const int v = *p;
-      *p = run;
-      run += v;
-    }
+    const int run = chunk_prefix(b.chunk_counts, nchunks, E + 1, e);
     if (e < E) cnt[e] = run;
   }
   __syncthreads();
@@ -248,22 +263,11 @@ __global__ void __launch_bounds__(32) ids_scatter_kernel(int64_t R, int E, Route
   for (int e = lane; e <= E; e += 32)
     run[e] = b.offsets[e] + b.chunk_counts[(size_t)blockIdx.x * (E + 1) + e];
   __syncwarp();
-  for (int i = 0; i < nr; i += 32) {
-    // one row per lane, placed in row order: lanes with the same bin take consecutive slots
-    const int64_t r = r0 + i + lane;
-    const bool have = i + lane < nr;
-    const int id = have ? b.ids[r] : 0;
-    const int bin = id < 0 ? E : id;
-    for (int l = 0; l < 32; ++l) {
-      if (lane == l && have) {
-        const int pos = run[bin];
-        run[bin] = pos + 1;
-        b.perm[pos] = (int32_t)r;
-        b.inv[r] = pos;
-      }
-      __syncwarp();
-    }
-  }
+  for (int i = 0; i < nr; i += 32)
+    place32(r0 + i, min(32, nr - i), lane, run, b, [&](int64_t r) {
+      const int id = b.ids[r];
+      return id < 0 ? E : id;
+    });
 }
 
 }  // namespace
@@ -271,12 +275,12 @@ __global__ void __launch_bounds__(32) ids_scatter_kernel(int64_t R, int E, Route
 int launch_route(const float* logits, int64_t T, int E, int k, const RouteBufs& b,
                  cudaStream_t s) {
   if (T <= kRouteChunk) {
-    route_small_kernel<<<1, 512, 0, s>>>(logits, (int)T, E, k, b);
+    route_small_kernel<<<1, 1024, 0, s>>>(logits, (int)T, E, k, b);
     const cudaError_t err = cudaGetLastError();
     return err == cudaSuccess ? 1 : -(int)err;
   }
   const int nch = route_chunks(T);
-  route_chunk_kernel<<<nch, 256, 0, s>>>(logits, T, E, k, b);
+  route_chunk_kernel<<<nch, 512, 0, s>>>(logits, T, E, k, b);
   route_scan_kernel<<<1, 1024, 0, s>>>(nch, E, b);
   route_scatter_kernel<<<nch, 32, 0, s>>>(T, E, k, b);
   const cudaError_t err = cudaGetLastError();
