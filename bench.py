@@ -686,7 +686,7 @@ def measure_ep(cfg, G: int = 8, steps: int = 10, warm: int = 3) -> dict:
     ms = total / steps
     hbm, tf_burst, tf_sus, peak_kind = load_peaks()
     R = T * k
-    disp_bytes = 2.0 * R * H * 2                     # each routed row read once and stored once
+    disp_bytes = T * H * 2.0 + R * H * 2.0           # x read once (its k copies come from L2), rows stored
     comb_bytes = R * H * 4.0 + T * H * 2.0           # every result row read, the output written
     remote = (G - 1) / G                             # share of rows whose owner is another GPU
     flops = 2.0 * Rr[0] * 3 * H * cfg.I
