@@ -54,7 +54,8 @@ def parse():
                     help="one workload only (default: decode_t1 as the headline, then every other "
                          "full-size workload in the same line)")
     ap.add_argument("--ncu-case", default=None, choices=["decode_t1_e16", "decode_t8_e16", "decode_t16_e16", "decode_t64_e16",
-                                                        "prefill_t4096_e16", "decode_t64z_e64", "w4a4_t4096_e16"],
+                                                        "prefill_t4096_e16", "decode_t64z_e64", "w4a4_t4096_e16",
+                                                        "ep8_t2048_e64"],
                     help="plain layer calls on a small bank for ncu captures (no timing, no graph)")
     ap.add_argument("--calls", type=int, default=4, help="layer calls of --ncu-case")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -613,25 +614,19 @@ def measure_w4a4(cfg, steps: int, warm: int) -> dict:
 NVLINK_GBS = 770.0      # measured peer copy per direction per GPU on this machine's B200s (NVLink 5)
 
 
-def measure_ep(cfg, G: int = 8, steps: int = 10, warm: int = 3) -> dict:
-    """Expert parallelism over G ranks (each rank the workload's T tokens, E/G experts), emulated
-    on one GPU: every rank's buffers live on this device and the peer pointers are local, so the
-    dispatch and combine kernels move the rows through HBM here instead of NVLink.  Times rank
-    0's step (dispatch of its routed rows, its experts on the rows it receives, its combine) with
-    CUDA events; the other ranks' dispatches and experts run once, untimed, so that rank 0
-    receives and reads back real data.  Reports each kernel against the HBM peak and the time
-    the same bytes would take over NVLink at the measured peer-copy bandwidth."""
+def ep_emulation(cfg, G: int):
+    """G expert-parallel ranks of cfg emulated on this GPU (each rank cfg.T tokens of its own, E/G
+    experts): routes every rank, plans, dispatches every rank's rows and runs every rank's experts
+    once, so that any rank's step can then be repeated on real data.  Returns the state."""
     import torch
     import nvfp4_weight_only_top_b200 as moe
     from nvfp4_weight_only_top_b200 import ep
     from moe_inputs import device as mdev
     lay = cfg.layout
-    s = torch.cuda.Stream()
-    torch.cuda.set_stream(s)
     buf = mdev.bank_tensor(lay, cfg.seed, 0)
     bank = moe.make_bank(buf.data_ptr(), lay.E, lay.H, lay.I, lay.record_stride, lay.codes_off, lay.scales_off,
                          lay.global_off, 0)
-    H, k, T = cfg.H, cfg.k, cfg.T
+    H, k = cfg.H, cfg.k
     xs, routes = [], []
     for r in range(G):
         xs.append(torch.from_numpy(moe_inputs.make_x(cfg, seed=cfg.seed + r).view(np.int16)).view(
@@ -643,26 +638,59 @@ def measure_ep(cfg, G: int = 8, steps: int = 10, warm: int = 3) -> dict:
     cap = max(plans[0]["recv_totals"])
     recv_x = [torch.empty((cap, H), dtype=torch.bfloat16, device="cuda") for _ in range(G)]
     recv_y = [torch.empty((cap, H), dtype=torch.float32, device="cuda") for _ in range(G)]
-    xp, yp = [t.data_ptr() for t in recv_x], [t.data_ptr() for t in recv_y]
-    plan_dev = [moe.moe_nvfp4_ep_plan(C, r, plans[r]["recv_total"], moe.EP_EXPERT_MAJOR) for r in range(G)]
-    shards = [ep.shard_bank(bank, r, G) for r in range(G)]
-    Rr = [p["recv_total"] for p in plans]
-    wsb = [torch.empty(moe.moe_nvfp4_experts_workspace_bytes(Rr[r], cfg.E // G, H, cfg.I), dtype=torch.uint8,
-                       device="cuda") for r in range(G)]
+    st = dict(buf=buf, bank=bank, xs=xs, routes=routes, C=C, plans=plans, cap=cap, recv_x=recv_x, recv_y=recv_y,
+              xp=[t.data_ptr() for t in recv_x], yp=[t.data_ptr() for t in recv_y],
+              plan_dev=[moe.moe_nvfp4_ep_plan(C, r, plans[r]["recv_total"], moe.EP_EXPERT_MAJOR) for r in range(G)],
+              shards=[ep.shard_bank(bank, r, G) for r in range(G)], Rr=[p["recv_total"] for p in plans])
+    st["wsb"] = [torch.empty(moe.moe_nvfp4_experts_workspace_bytes(st["Rr"][r], cfg.E // G, H, cfg.I),
+                             dtype=torch.uint8, device="cuda") for r in range(G)]
     for r in range(G):
-        moe.moe_nvfp4_ep_dispatch(xs[r], routes[r], plan_dev[r][0], xp, cap)
+        ep_dispatch(st, r)
     for r in range(G):
-        moe.moe_nvfp4_experts(recv_x[r][:Rr[r]], plan_dev[r][1], shards[r], y_rows=recv_y[r][:Rr[r]],
-                              workspace=wsb[r], sorted_ids=True)
-    out = torch.empty_like(xs[0])
+        ep_experts(st, r)
+    return st
+
+
+def ep_dispatch(st, r):
+    import nvfp4_weight_only_top_b200 as moe
+    moe.moe_nvfp4_ep_dispatch(st["xs"][r], st["routes"][r], st["plan_dev"][r][0], st["xp"], st["cap"])
+
+
+def ep_experts(st, r):
+    import nvfp4_weight_only_top_b200 as moe
+    Rr = st["Rr"][r]
+    moe.moe_nvfp4_experts(st["recv_x"][r][:Rr], st["plan_dev"][r][1], st["shards"][r], y_rows=st["recv_y"][r][:Rr],
+                          workspace=st["wsb"][r], sorted_ids=True)
+
+
+def ep_combine(st, r, out):
+    import nvfp4_weight_only_top_b200 as moe
+    moe.moe_nvfp4_ep_combine(st["routes"][r], st["plan_dev"][r][0], st["yp"], out.shape[1], st["cap"], out=out)
+
+
+def measure_ep(cfg, G: int = 8, steps: int = 10, warm: int = 3) -> dict:
+    """Expert parallelism over G ranks (each rank the workload's T tokens, E/G experts), emulated
+    on one GPU: every rank's buffers live on this device and the peer pointers are local, so the
+    dispatch and combine kernels move the rows through HBM here instead of NVLink.  Times rank
+    0's step (dispatch of its routed rows, its experts on the rows it receives, its combine) with
+    CUDA events; the other ranks' dispatches and experts run once, untimed, so that rank 0
+    receives and reads back real data.  Reports each kernel against the HBM peak and the time
+    the same bytes would take over NVLink at the measured peer-copy bandwidth."""
+    import torch
+    import nvfp4_weight_only_top_b200 as moe
+    s = torch.cuda.Stream()
+    torch.cuda.set_stream(s)
+    H, k, T = cfg.H, cfg.k, cfg.T
+    st = ep_emulation(cfg, G)
+    Rr = st["Rr"]
+    out = torch.empty_like(st["xs"][0])
 
     def step():
-        moe.moe_nvfp4_ep_dispatch(xs[0], routes[0], plan_dev[0][0], xp, cap)
+        ep_dispatch(st, 0)
         ev[1].record(s)
-        moe.moe_nvfp4_experts(recv_x[0][:Rr[0]], plan_dev[0][1], shards[0], y_rows=recv_y[0][:Rr[0]],
-                              workspace=wsb[0], sorted_ids=True)
+        ep_experts(st, 0)
         ev[2].record(s)
-        moe.moe_nvfp4_ep_combine(routes[0], plan_dev[0][0], yp, H, cap, out=out)
+        ep_combine(st, 0, out)
 
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     for _ in range(warm):
@@ -686,7 +714,7 @@ def measure_ep(cfg, G: int = 8, steps: int = 10, warm: int = 3) -> dict:
     ms = total / steps
     hbm, tf_burst, tf_sus, peak_kind = load_peaks()
     R = T * k
-    disp_bytes = T * H * 2.0 + R * H * 2.0           # x read once (its k copies come from L2), rows stored
+    disp_bytes = T * H * 2.0 + R * H * 2.0           # each token row read once and stored k times
     comb_bytes = R * H * 4.0 + T * H * 2.0           # every result row read, the output written
     remote = (G - 1) / G                             # share of rows whose owner is another GPU
     flops = 2.0 * Rr[0] * 3 * H * cfg.I
@@ -816,13 +844,28 @@ def ncu_case(case: str, calls: int) -> None:
     decode_t8_e16 (T=8, the few-token kernel), decode_t16_e16 and decode_t64_e16 (T=16 and 64, the
     grouped kernels), prefill_t4096_e16 (T=4096, tensor-core path);
     decode_t64z_e64: T=64 with Zipf routing over 64 resident experts (1.4 GB);
-    w4a4_t4096_e16: T=4096 on the W4A4 path (NVFP4 activations).
+    w4a4_t4096_e16: T=4096 on the W4A4 path (NVFP4 activations);
+    ep8_t2048_e64: expert parallelism over 8 ranks emulated on this GPU, 2048 tokens per rank, 64
+    experts (8 per rank): rank 0's dispatch and combine kernels.
     """
     import torch
     import nvfp4_weight_only_top_b200 as moe
     from moe_inputs import device as mdev
     T, path = NCU_CASES[case]
     E, k, H, I = (64 if case.endswith("e64") else 16), 8, 5120, 2560
+    if path == "ep":
+        # expert parallelism over 8 ranks emulated on this GPU: every rank's rows are dispatched
+        # and its experts run once in the set-up; then rank 0's dispatch and combine, `calls` times
+        cfg = moe_inputs.LayerConfig(case, E, k, H, I, T)
+        st = ep_emulation(cfg, 8)
+        out = torch.empty_like(st["xs"][0])
+        for _ in range(calls):
+            ep_dispatch(st, 0)
+            ep_combine(st, 0, out)
+        torch.cuda.synchronize()
+        assert moe.moe_nvfp4_device_status() == 0
+        print(f"{case}: {calls} calls ok")
+        return
     lay = moe_inputs.record_layout(E, H, I)
     buf = mdev.bank_tensor(lay, 0, 0)
     bank = moe.make_bank(buf.data_ptr(), E, H, I, lay.record_stride, lay.codes_off, lay.scales_off,
@@ -848,7 +891,7 @@ def ncu_case(case: str, calls: int) -> None:
 NCU_CASES = {"decode_t1_e16": (1, "decode"), "decode_t8_e16": (8, "decode"), "decode_t16_e16": (16, "decode"),
              "decode_t64_e16": (64, "decode"),
              "prefill_t4096_e16": (4096, "prefill"), "decode_t64z_e64": (64, "decode"),
-             "w4a4_t4096_e16": (4096, "w4a4")}
+             "w4a4_t4096_e16": (4096, "w4a4"), "ep8_t2048_e64": (2048, "ep")}
 
 
 def main():

@@ -271,15 +271,16 @@ int moe_nvfp4_ep_plan(const int32_t* counts_all_dev, int32_t ranks, int32_t num_
 
 /*
  * Stores every routed row of this rank (x_dev [T, H] BF16; routed row r = t*k+j) into the
- * receive buffer of the owner of ids[r], at row dst_off[g] + (inv[r] - offsets[g]) of an
- * EXPERT_MAJOR plan.  recv_x_ptrs_host: host array of G device pointers valid in this process
- * (this rank's own buffer, the others opened with moe_nvfp4_ep_buffer_open), each 16-byte
- * aligned.  ids, perm and offsets are moe_nvfp4_route's for this rank's tokens.
+ * receive buffer of the owner of g = ids[r], at row dst_off[g] + (inv[r] - offsets[g]) of an
+ * EXPERT_MAJOR plan; each token's row is read once and stored k times.  recv_x_ptrs_host: host
+ * array of G device pointers valid in this process (this rank's own buffer, the others opened
+ * with moe_nvfp4_ep_buffer_open), each 16-byte aligned.  ids, inv and offsets are
+ * moe_nvfp4_route's for this rank's tokens.
  * capacity_rows: rows every receive buffer holds; a row whose place falls outside
  * [0, capacity_rows) is not stored (a plan from counts that do not match the routing).
  */
 int moe_nvfp4_ep_dispatch(const void* x_dev, int64_t T, int32_t k, int32_t hidden,
-                          int32_t num_experts, const int32_t* ids_dev, const int32_t* perm_dev,
+                          int32_t num_experts, const int32_t* ids_dev, const int32_t* inv_dev,
                           const int32_t* offsets_dev, const int32_t* dst_off_dev, int32_t ranks,
                           void* const* recv_x_ptrs_host, int64_t capacity_rows, void* stream);
 

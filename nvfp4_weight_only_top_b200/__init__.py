@@ -315,7 +315,7 @@ def moe_nvfp4_ep_dispatch(x, route: dict, dst_off, recv_x_ptrs, capacity_rows: i
     for args in need:
         _need(*args)
     ptrs = (ctypes.c_void_p * G)(*[int(p) for p in recv_x_ptrs])
-    _check(lib().moe_nvfp4_ep_dispatch(_ptr(x), T, k, H, E, _ptr(route["ids"]), _ptr(route["perm"]),
+    _check(lib().moe_nvfp4_ep_dispatch(_ptr(x), T, k, H, E, _ptr(route["ids"]), _ptr(route["inv"]),
                                        _ptr(route["offsets"]), _ptr(dst_off), G, ptrs, int(capacity_rows),
                                        _stream(stream)))
 

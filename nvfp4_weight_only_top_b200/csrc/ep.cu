@@ -5,10 +5,10 @@
 //   plan      from the count matrix C[s][g] (rows rank s routes to global expert g, gathered
 //             from every rank) the place of this rank's rows in every receiver's buffer and the
 //             local expert id of every row this rank receives;
-//   dispatch  gathers this rank's routed rows and stores each straight into its expert owner's
-//             receive buffer (a peer pointer), expert-major there: for local expert e, the rows
-//             of rank 0, then of rank 1, ...; the receiver's expert kernels then read them in
-//             place;
+//   dispatch  reads each token's row once and stores it straight into the receive buffer of the
+//             owner of each of its k experts (a peer pointer), expert-major there: for local
+//             expert e, the rows of rank 0, then of rank 1, ...; the receiver's expert kernels
+//             then read them in place;
 //   combine   reads each routed row's expert output back from the owner's output buffer (peer
 //             loads) and forms out[t] = bf16(sum_j w[t, j] * y[t, j]) with the layer's own f32
 //             accumulation order.
@@ -119,35 +119,41 @@ struct PeerPtrs {
   void* p[kEpMaxRanks];
 };
 
-// One CTA per routed row in turn (grid-stride over the permuted order p): row x[perm[p] / k]
-// goes to its owner's receive buffer at dst_off[g] + (p - offsets[g]).  Each thread loads its
-// vectors of the row first, then stores them, so that a row's loads are in flight together.
-__global__ void __launch_bounds__(kMoveThreads) ep_dispatch_kernel(const uint16_t* __restrict__ x, int64_t R, int k,
+// One CTA per token in turn (grid-stride over tokens): the token's row of x is read once into
+// registers and stored to the owner of each of its k experts, routed row r = t*k+j going to row
+// dst_off[g] + (inv[r] - offsets[g]) of that owner's receive buffer.
+__global__ void __launch_bounds__(kMoveThreads) ep_dispatch_kernel(const uint16_t* __restrict__ x, int64_t T, int k,
                                                                    int H, const int32_t* __restrict__ ids,
-                                                                   const int32_t* __restrict__ perm,
+                                                                   const int32_t* __restrict__ inv,
                                                                    const int32_t* __restrict__ offsets,
                                                                    const int32_t* __restrict__ dst_off, int El,
                                                                    int64_t cap, PeerPtrs recv) {
   const int nv = H / 8;
-  for (int64_t p = blockIdx.x; p < R; p += gridDim.x) {
-    const int r = perm[p];
-    const int g = ids[r];
-    const int d = g / El;
-    const int64_t pos = (int64_t)dst_off[g] + (p - offsets[g]);
-    if (pos < 0 || pos >= cap) continue;          // a plan that does not fit: store nothing
-    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(r / k) * H);
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(recv.p[d]) + (size_t)pos * H);
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
     uint4 v[kMaxVec];
 #pragma unroll
     for (int i = 0; i < kMaxVec; ++i)
       if (threadIdx.x + i * kMoveThreads < nv) v[i] = src[threadIdx.x + i * kMoveThreads];
+    for (int j = 0; j < k; ++j) {
+      const int64_t r = t * k + j;
+      const int g = ids[r];
+      const int d = g / El;
+      const int64_t pos = (int64_t)dst_off[g] + (inv[r] - offsets[g]);
+      if (pos < 0 || pos >= cap) continue;          // a plan that does not fit: store nothing
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(recv.p[d]) + (size_t)pos * H);
 #pragma unroll
-    for (int i = 0; i < kMaxVec; ++i)
-      if (threadIdx.x + i * kMoveThreads < nv) dst[threadIdx.x + i * kMoveThreads] = v[i];
+      for (int i = 0; i < kMaxVec; ++i)
+        if (threadIdx.x + i * kMoveThreads < nv) dst[threadIdx.x + i * kMoveThreads] = v[i];
+    }
   }
-  // Order this thread's stores (to peers) before anything the stream does after the kernel, at
-  // system scope: the barrier that follows the dispatch then publishes them to their owners.
-  __threadfence_system();
+  // Order the CTA's stores (to peers) before anything the stream does after the kernel, at system
+  // scope: the barrier that follows the dispatch then publishes them to their owners.  The CTA
+  // barrier orders every thread's stores before thread 0's fence, which is cumulative; one fence
+  // per CTA instead of one per thread (a system-scope fence in every thread was this kernel's
+  // largest stall).
+  __syncthreads();
+  if (threadIdx.x == 0) __threadfence_system();
 }
 
 // out[t] = bf16(sum_j w[t, j] * y_owner(t, j)), j = 0 .. k-1 in order with fmaf, as the layer's
@@ -217,13 +223,13 @@ int launch_ep_plan(const int32_t* C, int G, int E, int rank, int layout, int32_t
 
 bool ep_move_supported(int H) { return H % 8 == 0 && H / 8 <= kMaxVec * kMoveThreads; }
 
-int launch_ep_dispatch(const uint16_t* x, int64_t R, int k, int H, const int32_t* ids, const int32_t* perm,
+int launch_ep_dispatch(const uint16_t* x, int64_t T, int k, int H, const int32_t* ids, const int32_t* inv,
                        const int32_t* offsets, const int32_t* dst_off, int El, int64_t cap, void* const* recv, int G,
                        int num_sms, cudaStream_t s) {
   PeerPtrs pp{};
   for (int d = 0; d < G; ++d) pp.p[d] = recv[d];
-  const int64_t blocks = R < (int64_t)num_sms * 16 ? R : (int64_t)num_sms * 16;
-  ep_dispatch_kernel<<<(unsigned)blocks, kMoveThreads, 0, s>>>(x, R, k, H, ids, perm, offsets, dst_off, El, cap, pp);
+  const int64_t blocks = T < (int64_t)num_sms * 16 ? T : (int64_t)num_sms * 16;
+  ep_dispatch_kernel<<<(unsigned)blocks, kMoveThreads, 0, s>>>(x, T, k, H, ids, inv, offsets, dst_off, El, cap, pp);
   const cudaError_t err = cudaGetLastError();
   return err == cudaSuccess ? 1 : -(int)err;
 }
@@ -288,7 +294,7 @@ int moe_nvfp4_ep_plan(const int32_t* counts_all_dev, int32_t ranks, int32_t num_
 }
 
 int moe_nvfp4_ep_dispatch(const void* x_dev, int64_t T, int32_t k, int32_t hidden, int32_t num_experts,
-                          const int32_t* ids_dev, const int32_t* perm_dev, const int32_t* offsets_dev,
+                          const int32_t* ids_dev, const int32_t* inv_dev, const int32_t* offsets_dev,
                           const int32_t* dst_off_dev, int32_t ranks, void* const* recv_x_ptrs_host,
                           int64_t capacity_rows, void* stream) {
   moe::api_set_launches(0);
@@ -301,7 +307,7 @@ int moe_nvfp4_ep_dispatch(const void* x_dev, int64_t T, int32_t k, int32_t hidde
   int dev, sms;
   if ((rc = moe::api_device(&dev, &sms))) return rc;
   if (T == 0) return MOE_NVFP4_OK;
-  if (!x_dev || !ids_dev || !perm_dev || !offsets_dev || !dst_off_dev || !recv_x_ptrs_host)
+  if (!x_dev || !ids_dev || !inv_dev || !offsets_dev || !dst_off_dev || !recv_x_ptrs_host)
     return moe::api_fail(MOE_NVFP4_ERR_INVALID_ARG, "a pointer argument is NULL");
   if (!al(x_dev, 16)) return moe::api_fail(MOE_NVFP4_ERR_INVALID_ARG, "x must be 16-byte aligned");
   if (capacity_rows < 0) return moe::api_fail(MOE_NVFP4_ERR_INVALID_ARG, "capacity_rows is negative");
@@ -309,7 +315,7 @@ int moe_nvfp4_ep_dispatch(const void* x_dev, int64_t T, int32_t k, int32_t hidde
     if (!recv_x_ptrs_host[d] || !al(recv_x_ptrs_host[d], 16))
       return moe::api_fail(MOE_NVFP4_ERR_INVALID_ARG, "every receive buffer must be non-NULL and 16-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return done(moe::launch_ep_dispatch(static_cast<const uint16_t*>(x_dev), T * k, k, hidden, ids_dev, perm_dev,
+  return done(moe::launch_ep_dispatch(static_cast<const uint16_t*>(x_dev), T, k, hidden, ids_dev, inv_dev,
                                       offsets_dev, dst_off_dev, num_experts / ranks, capacity_rows, recv_x_ptrs_host,
                                       ranks, sms, s),
               "ep dispatch");

@@ -20,17 +20,29 @@ struct RouteBufs {
   int32_t* ngroups;    // [1]
   int4* singles;       // [max_groups]: (expert, permuted row, 1, 0): one-row groups
   int32_t* nsingles;   // [1]
-  int32_t* chunk_counts;  // [nchunks, E] (multi-CTA routing only)
+  int32_t* chunk_counts;  // [nchunks, E]: kRouteChunk tokens per chunk (T > kRouteChunk), or
+                          // kSmallTok tokens per chunk (T <= kRouteChunk)
+  unsigned* done;         // [1]: CTAs of the one-launch router that finished (reset by its last)
   int group_rows;      // rows per group (decode token tile)
   int split_singles;   // 1: one-row groups go to `singles`; 0: they stay in `groups`
   int expert_major;    // 1: each expert's groups are listed together (full, then its partial);
                        // 0: all full groups first, then the partial ones
 };
 
-// Tokens per routing chunk in the multi-CTA router; one CTA routes T <= this on its own.
+// Tokens per routing chunk in the multi-launch router, used for T > kRouteChunk; up to
+// kRouteChunk tokens are routed in one launch, by one CTA up to kOneCtaTokens, else kSmallTok
+// tokens (one per warp) per CTA.
 constexpr int kRouteChunk = 64;
+constexpr int kSmallTok = 8;
+// Up to this many tokens one CTA routes them alone (measured faster than the one-launch
+// multi-CTA router below about 32 tokens, which pays for a memset and the last-CTA hand-off).
+constexpr int kOneCtaTokens = 32;
 
 inline int route_chunks(int64_t T) { return (int)((T + kRouteChunk - 1) / kRouteChunk); }
+// Ints of RouteBufs::chunk_counts the router needs for T tokens and E experts.
+inline size_t route_chunk_ints(int64_t T, int E) {
+  return T > kRouteChunk ? (size_t)route_chunks(T) * E : (size_t)((T + kSmallTok - 1) / kSmallTok) * E;
+}
 inline int64_t max_groups(int64_t R, int E, int group_rows) {
   int64_t g = (R + group_rows - 1) / group_rows + E;
   return g < R ? g : R;
@@ -161,7 +173,7 @@ size_t ep_plan_smem_bytes(int G, int E);
 int launch_ep_plan(const int32_t* C, int G, int E, int rank, int layout, int32_t* dst_off, int32_t* recv_ids,
                    int64_t recv_rows, cudaStream_t s);
 bool ep_move_supported(int H);
-int launch_ep_dispatch(const uint16_t* x, int64_t R, int k, int H, const int32_t* ids, const int32_t* perm,
+int launch_ep_dispatch(const uint16_t* x, int64_t T, int k, int H, const int32_t* ids, const int32_t* inv,
                        const int32_t* offsets, const int32_t* dst_off, int El, int64_t cap, void* const* recv, int G,
                        int num_sms, cudaStream_t s);
 int launch_ep_combine(int64_t T, int k, int H, const int32_t* ids, const float* w, const int32_t* inv,

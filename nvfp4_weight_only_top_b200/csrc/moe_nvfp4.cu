@@ -108,7 +108,7 @@ int current_device(int* dev, DeviceInfo* info) {
 
 // Sizes of the workspace sub-buffers, each 256-byte aligned.
 struct WsLayout {
-  size_t ids, w, counts, offsets, perm, inv, groups, ngroups, singles, nsingles, chunk_counts, bar, h, y, total;
+  size_t ids, w, counts, offsets, perm, inv, groups, ngroups, singles, nsingles, chunk_counts, done, bar, h, y, total;
 };
 
 size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -135,8 +135,8 @@ WsLayout ws_layout(int64_t T, int E, int k, int H, int I, int path, bool given_i
   L.ngroups = take(4);
   L.singles = take((size_t)E * 16);
   L.nsingles = take(4);
-  L.chunk_counts = take(given_ids ? (size_t)moe::route_chunks(T) * (E + 1) * 4
-                                  : T > moe::kRouteChunk ? (size_t)moe::route_chunks(T) * E * 4 : 0);
+  L.chunk_counts = take(given_ids ? (size_t)moe::route_chunks(T) * (E + 1) * 4 : moe::route_chunk_ints(T, E) * 4);
+  L.done = take(4);
   L.bar = take(2 * sizeof(unsigned));        // tile counters of the tensor-core path
   L.h = take(R * (size_t)I * 4);
   L.y = take(R * (size_t)H * 4);
@@ -304,6 +304,7 @@ moe::RouteBufs route_bufs(uint8_t* ws, const WsLayout& L) {
   b.singles = reinterpret_cast<int4*>(ws + L.singles);
   b.nsingles = reinterpret_cast<int32_t*>(ws + L.nsingles);
   b.chunk_counts = reinterpret_cast<int32_t*>(ws + L.chunk_counts);
+  b.done = reinterpret_cast<unsigned*>(ws + L.done);
   b.group_rows = 8;
   b.split_singles = 0;
   b.expert_major = 0;

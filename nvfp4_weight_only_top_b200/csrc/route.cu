@@ -16,44 +16,6 @@ namespace {
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
-// Exclusive scan of n ints in shared memory (in place) by the whole block; returns the total.
-__device__ int block_scan_excl(int* a, int n, int* warp_tmp) {
-  const int tid = threadIdx.x, nt = blockDim.x;
-  const int per = (n + nt - 1) / nt;
-  const int lo = tid * per, hi = min(n, lo + per);
-  int s = 0;
-  for (int i = lo; i < hi; ++i) s += a[i];
-  // inclusive warp scan of s
-  const int lane = tid & 31, wid = tid >> 5, nw = (nt + 31) >> 5;
-  int v = s;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int o = __shfl_up_sync(kFull, v, off);
-    if (lane >= off) v += o;
-  }
-  if (lane == 31) warp_tmp[wid] = v;
-  __syncthreads();
-  if (wid == 0) {
-    int t = lane < nw ? warp_tmp[lane] : 0;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(kFull, t, off);
-      if (lane >= off) t += o;
-    }
-    if (lane < nw) warp_tmp[lane] = t;  // inclusive prefix over warps
-  }
-  __syncthreads();
-  int run = v - s + (wid > 0 ? warp_tmp[wid - 1] : 0);  // exclusive prefix of this thread
-  const int total = warp_tmp[nw - 1];
-  for (int i = lo; i < hi; ++i) {
-    const int c = a[i];
-    a[i] = run;
-    run += c;
-  }
-  __syncthreads();
-  return total;
-}
-
 // Stable placement of rows r0 .. r0+n-1 (n <= 32, one per lane, bins from bin_of) by one warp:
 // lanes with the same bin take consecutive slots in lane order, from run[bin] on, and the
 // lowest lane of each bin advances run[bin] for the next call.
@@ -99,6 +61,46 @@ __device__ __forceinline__ int chunk_prefix(int32_t* cc, int nchunks, int stride
   return run;
 }
 
+// Exclusive prefix sums of four arrays of n ints in shared memory, in place, by one warp (each
+// lane a contiguous run, then a shuffle scan of the runs' sums); the four totals go to tot[0..3].
+__device__ __forceinline__ void warp_scan4_excl(int* a0, int* a1, int* a2, int* a3, int n, int* tot) {
+  const int lane = threadIdx.x & 31, per = (n + 31) / 32;
+  const int lo = min(n, lane * per), hi = min(n, lo + per);
+  int s[4] = {0, 0, 0, 0};
+  for (int i = lo; i < hi; ++i) {
+    s[0] += a0[i];
+    s[1] += a1[i];
+    s[2] += a2[i];
+    s[3] += a3[i];
+  }
+  int inc[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int v = __shfl_up_sync(kFull, inc[j], o);
+      if (lane >= o) inc[j] += v;
+    }
+  int run[4] = {inc[0] - s[0], inc[1] - s[1], inc[2] - s[2], inc[3] - s[3]};
+  for (int i = lo; i < hi; ++i) {
+    int v = a0[i];
+    a0[i] = run[0];
+    run[0] += v;
+    v = a1[i];
+    a1[i] = run[1];
+    run[1] += v;
+    v = a2[i];
+    a2[i] = run[2];
+    run[2] += v;
+    v = a3[i];
+    a3[i] = run[3];
+    run[3] += v;
+  }
+  if (lane == 31)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tot[j] = inc[j];
+}
+
 // From per-expert counts in shared memory: offsets and the two group lists.  An expert's rows
 // are cut into groups of group_rows; when split_singles is set, a last group of a single row
 // goes to the one-row list instead.  All full groups (exactly group_rows rows) come first, in
@@ -119,10 +121,11 @@ __device__ void finish_counts(int* cnt, int* tmp, int* tmp1, int* tmp2, int* war
     tmp1[e] = single;
   }
   __syncthreads();
-  const int nf = block_scan_excl(tmp, E, warp_tmp);         // tmp: first full group of e
-  const int np = block_scan_excl(tmp2, E, warp_tmp);        // tmp2: its partial group, after the full ones
-  const int ns = block_scan_excl(tmp1, E, warp_tmp);        // tmp1: its one-row group slot
-  const int R = block_scan_excl(cnt, E, warp_tmp);          // cnt -> offsets (in place)
+  // tmp: first full group of e; tmp2: its partial group, after the full ones; tmp1: its one-row
+  // group slot; cnt -> offsets (in place)
+  if (threadIdx.x < 32) warp_scan4_excl(tmp, tmp2, tmp1, cnt, E, warp_tmp);
+  __syncthreads();
+  const int nf = warp_tmp[0], np = warp_tmp[1], ns = warp_tmp[2], R = warp_tmp[3];
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     b.offsets[e] = cnt[e];
     const int c = b.counts[e];
@@ -142,11 +145,11 @@ __device__ void finish_counts(int* cnt, int* tmp, int* tmp1, int* tmp2, int* war
   }
 }
 
-// Single-CTA routing for T <= kRouteChunk: router, histogram, scan, groups, stable scatter.
-__global__ void __launch_bounds__(1024) route_small_kernel(const float* __restrict__ logits,
-                                                          int T, int E, int k, RouteBufs b) {
+// Single-CTA routing for T <= kOneCtaTokens: router, histogram, scan, groups, stable placement.
+__global__ void __launch_bounds__(1024) route_one_cta_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                             RouteBufs b) {
   __shared__ int cnt[kMaxE], tmp[kMaxE], tmp1[kMaxE], tmp2[kMaxE], run[kMaxE], warp_tmp[32];
-  __shared__ int sids[kRouteChunk * 32];
+  __shared__ int sids[kOneCtaTokens * 32];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
@@ -171,6 +174,55 @@ __global__ void __launch_bounds__(1024) route_small_kernel(const float* __restri
     for (int r0 = 0; r0 < R; r0 += 32)
       place32(r0, min(32, R - r0), lane, run, b, [&](int64_t r) { return sids[r]; });
   }
+}
+
+// Routing of T <= kRouteChunk tokens in one launch: CTA c routes tokens kSmallTok c .. (one per
+// warp) and counts its rows per expert; the last CTA to finish (a counter in the workspace, zero
+// at launch) takes every CTA's counts, forms counts, offsets and groups, and places the rows, one
+// warp per CTA's rows, each from its own running positions.
+__global__ void __launch_bounds__(32 * kSmallTok) route_small_kernel(const float* __restrict__ logits, int T, int E,
+                                                                     int k, RouteBufs b) {
+  __shared__ int cnt[kMaxE], tmp[kMaxE], tmp1[kMaxE], tmp2[kMaxE], warp_tmp[32];
+  __shared__ int s_last;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int nch = gridDim.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int t = blockIdx.x * kSmallTok + wid;
+  if (t < T) {
+    int id;
+    float w;
+    route_row(logits + (size_t)t * E, E, k, lane, id, w);
+    if (lane < k) {
+      b.ids[t * k + lane] = id;
+      b.w[t * k + lane] = w;
+      atomicAdd(&cnt[id], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) b.chunk_counts[(size_t)blockIdx.x * E + e] = cnt[e];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();                                   // this CTA's ids and counts before the count
+    s_last = atomicAdd(b.done, 1u) == (unsigned)(nch - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();                                     // every CTA's ids and counts after the count
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = chunk_prefix(b.chunk_counts, nch, E, e);
+  __syncthreads();
+  finish_counts(cnt, tmp, tmp1, tmp2, warp_tmp, E, b.group_rows, b);
+  __syncthreads();                                     // cnt = offsets
+  // running position of chunk c's next row of expert e, in place in chunk_counts
+  for (int i = threadIdx.x; i < nch * E; i += blockDim.x) b.chunk_counts[i] += cnt[i % E];
+  __syncthreads();
+  for (int c = wid; c < nch; c += kSmallTok) {
+    const int r_begin = c * kSmallTok * k, r_end = min(T, (c + 1) * kSmallTok) * k;
+    for (int r0 = r_begin; r0 < r_end; r0 += 32)
+      place32(r0, min(32, r_end - r0), lane, b.chunk_counts + (size_t)c * E, b,
+              [&](int64_t r) { return __ldcg(b.ids + r); });
+  }
+  if (threadIdx.x == 0) *b.done = 0;                   // for the next call on this workspace
 }
 
 // Multi-CTA routing, step 1: route the chunk's tokens and count its rows per expert.
@@ -274,9 +326,16 @@ __global__ void __launch_bounds__(32) ids_scatter_kernel(int64_t R, int E, Route
 
 int launch_route(const float* logits, int64_t T, int E, int k, const RouteBufs& b,
                  cudaStream_t s) {
-  if (T <= kRouteChunk) {
-    route_small_kernel<<<1, 1024, 0, s>>>(logits, (int)T, E, k, b);
+  if (T <= kOneCtaTokens) {
+    route_one_cta_kernel<<<1, 1024, 0, s>>>(logits, (int)T, E, k, b);
     const cudaError_t err = cudaGetLastError();
+    return err == cudaSuccess ? 1 : -(int)err;
+  }
+  if (T <= kRouteChunk) {
+    cudaError_t err = cudaMemsetAsync(b.done, 0, sizeof(unsigned), s);
+    if (err != cudaSuccess) return -(int)err;
+    route_small_kernel<<<(unsigned)((T + kSmallTok - 1) / kSmallTok), 32 * kSmallTok, 0, s>>>(logits, (int)T, E, k, b);
+    err = cudaGetLastError();
     return err == cudaSuccess ? 1 : -(int)err;
   }
   const int nch = route_chunks(T);
