@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(kMoveThreads) ep_dispatch_kernel(const uint16_
                                                                    const int32_t* __restrict__ inv,
                                                                    const int32_t* __restrict__ offsets,
                                                                    const int32_t* __restrict__ dst_off, int El,
-                                                                   int64_t cap, PeerPtrs recv) {
+                                                                   int E, int64_t cap, PeerPtrs recv) {
   const int nv = H / 8;
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(kMoveThreads) ep_dispatch_kernel(const uint16_
     for (int j = 0; j < k; ++j) {
       const int64_t r = t * k + j;
       const int g = ids[r];
+      if ((unsigned)g >= (unsigned)E) continue;     // not an expert id: store nothing
       const int d = g / El;
       const int64_t pos = (int64_t)dst_off[g] + (inv[r] - offsets[g]);
       if (pos < 0 || pos >= cap) continue;          // a plan that does not fit: store nothing
@@ -163,8 +164,8 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(int64_t T, int k, int H
                                                          const float* __restrict__ w,
                                                          const int32_t* __restrict__ inv,
                                                          const int32_t* __restrict__ offsets,
-                                                         const int32_t* __restrict__ dst_off, int El, int64_t cap,
-                                                         PeerPtrs ys,
+                                                         const int32_t* __restrict__ dst_off, int El, int E,
+                                                         int64_t cap, PeerPtrs ys,
                                                          const uint16_t* __restrict__ x, uint16_t* __restrict__ out,
                                                          uint16_t* __restrict__ x_next) {
   const int per_row = H / 8;
@@ -176,6 +177,7 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(int64_t T, int k, int H
   for (int j = 0; j < k; ++j) {
     const int64_t r = t * k + j;
     const int g = ids[r];
+    if ((unsigned)g >= (unsigned)E) continue;     // not an expert id: the row adds nothing
     const int d = g / El;
     const int64_t pos = (int64_t)dst_off[g] + (inv[r] - offsets[g]);
     if (pos < 0 || pos >= cap) continue;          // a plan that does not fit: the row adds nothing
@@ -229,7 +231,8 @@ int launch_ep_dispatch(const uint16_t* x, int64_t T, int k, int H, const int32_t
   PeerPtrs pp{};
   for (int d = 0; d < G; ++d) pp.p[d] = recv[d];
   const int64_t blocks = T < (int64_t)num_sms * 16 ? T : (int64_t)num_sms * 16;
-  ep_dispatch_kernel<<<(unsigned)blocks, kMoveThreads, 0, s>>>(x, T, k, H, ids, inv, offsets, dst_off, El, cap, pp);
+  ep_dispatch_kernel<<<(unsigned)blocks, kMoveThreads, 0, s>>>(x, T, k, H, ids, inv, offsets, dst_off, El, El * G, cap,
+                                                               pp);
   const cudaError_t err = cudaGetLastError();
   return err == cudaSuccess ? 1 : -(int)err;
 }
@@ -240,8 +243,8 @@ int launch_ep_combine(int64_t T, int k, int H, const int32_t* ids, const float* 
   PeerPtrs pp{};
   for (int d = 0; d < G; ++d) pp.p[d] = const_cast<float*>(ys[d]);
   const int64_t n = T * (H / 8);
-  ep_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(T, k, H, ids, w, inv, offsets, dst_off, El, cap, pp,
-                                                                 x, out, x_next);
+  ep_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(T, k, H, ids, w, inv, offsets, dst_off, El, El * G,
+                                                                 cap, pp, x, out, x_next);
   const cudaError_t err = cudaGetLastError();
   return err == cudaSuccess ? 1 : -(int)err;
 }

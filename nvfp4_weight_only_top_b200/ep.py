@@ -186,26 +186,53 @@ class ExpertParallel:
 
     # -- peer buffers ------------------------------------------------------------------------
     def _make_buffers(self) -> None:
+        """Creates this rank's receive buffers and maps every peer's.  Every rank learns whether all
+        of them succeeded (an all-gather of the outcome) and all raise together if one failed, so
+        that no rank is left waiting in a later collective."""
         import torch.distributed as dist
-        from . import moe_nvfp4_ep_buffer_create, moe_nvfp4_ep_buffer_open
+        from . import (moe_nvfp4_ep_buffer_close, moe_nvfp4_ep_buffer_create, moe_nvfp4_ep_buffer_destroy,
+                       moe_nvfp4_ep_buffer_open)
         cap, H = self.capacity, self.H
-        px, hx = moe_nvfp4_ep_buffer_create(cap * H * 2)
-        py, hy = moe_nvfp4_ep_buffer_create(cap * H * 4)
-        self._own = [px, py]
+        err = None
+        mine = None
+        try:
+            px, hx = moe_nvfp4_ep_buffer_create(cap * H * 2)
+            self._own.append(px)
+            py, hy = moe_nvfp4_ep_buffer_create(cap * H * 4)
+            self._own.append(py)
+            mine = (hx, hy)
+        except Exception as exc:            # reported to every rank below
+            err = repr(exc)
         handles = [None] * self.world
-        dist.all_gather_object(handles, (hx, hy), group=self.group)
+        dist.all_gather_object(handles, mine, group=self.group)
         xs, ys = [], []
-        for d, (hxd, hyd) in enumerate(handles):
-            if d == self.rank:
-                xs.append(px)
-                ys.append(py)
-            else:
-                a = moe_nvfp4_ep_buffer_open(hxd)
-                self._opened.append(a)
-                b = moe_nvfp4_ep_buffer_open(hyd)
-                self._opened.append(b)
-                xs.append(a)
-                ys.append(b)
+        if all(h is not None for h in handles):
+            try:
+                for d, (hxd, hyd) in enumerate(handles):
+                    if d == self.rank:
+                        xs.append(px)
+                        ys.append(py)
+                        continue
+                    a = moe_nvfp4_ep_buffer_open(hxd)
+                    self._opened.append(a)
+                    b = moe_nvfp4_ep_buffer_open(hyd)
+                    self._opened.append(b)
+                    xs.append(a)
+                    ys.append(b)
+            except Exception as exc:
+                err = repr(exc)
+        outcome = [None] * self.world
+        dist.all_gather_object(outcome, err, group=self.group)
+        failed = {d: e for d, e in enumerate(outcome) if e is not None}
+        if failed or any(h is None for h in handles):
+            for p in self._opened:
+                moe_nvfp4_ep_buffer_close(p)
+            self._opened = []
+            dist.barrier(group=self.group)          # no peer still maps this rank's buffers
+            for p in self._own:
+                moe_nvfp4_ep_buffer_destroy(p)
+            self._own = []
+            raise RuntimeError(f"expert-parallel buffers could not be set up: {failed}")
         self.recv_x_ptrs, self.recv_y_ptrs = xs, ys
         self._recv_x = _view(px, (cap, H), _bf16(), self.device)
         self._recv_y = _view(py, (cap, H), _f32(), self.device)

@@ -206,3 +206,53 @@ def test_collective_step_reproduces_the_layer_gloo(case):
         assert scale is not None, err
         assert shape_ok
         assert err <= 1e-12 * max(scale, 1.0), (rank, err, scale)
+
+
+def _ep_setup_rank_main(rank, ws, port, q):
+    """Rank 0 creates its buffers, rank 1 fails to: both must raise together, rank 0 freeing its
+    own buffers, instead of leaving one rank waiting in a later collective."""
+    import sys
+    os.environ.update({"WORLD_SIZE": str(ws), "RANK": str(rank), "MASTER_ADDR": "127.0.0.1",
+                       "MASTER_PORT": str(port)})
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch.distributed as dist
+    import nvfp4_weight_only_top_b200 as moe
+    from nvfp4_weight_only_top_b200 import ep as ep_mod
+    freed, made = [], []
+    if rank == 0:
+        def create(nbytes):
+            made.append(4096 * (1 + len(made)))
+            return made[-1], bytes(64)
+        moe.moe_nvfp4_ep_buffer_create = create
+    else:
+        def fail(nbytes):
+            raise moe.MoeError(-3, "out of memory")
+        moe.moe_nvfp4_ep_buffer_create = fail
+    moe.moe_nvfp4_ep_buffer_destroy = lambda p: freed.append(p)
+    moe.moe_nvfp4_ep_buffer_open = lambda h: (_ for _ in ()).throw(AssertionError("no handle to open"))
+    dist.init_process_group("gloo", rank=rank, world_size=ws, timeout=datetime.timedelta(seconds=60))
+    bank = moe.make_bank(0, 8, 32, 32, 4096, [0, 0, 0], [0, 0, 0], [0, 0, 0])
+    try:
+        ep_mod.ExpertParallel(bank, 2, transport="peer", capacity_rows=16, ops=OracleOps(None, 8))
+        q.put((rank, "no error", freed))
+    except RuntimeError as exc:
+        q.put((rank, str(exc), freed))
+    dist.destroy_process_group()
+
+
+def test_peer_buffer_setup_fails_on_every_rank_together_gloo():
+    ws, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_ep_setup_rank_main, args=(r, ws, port, q)) for r in range(ws)]
+    for p in procs:
+        p.start()
+    got = sorted(q.get(timeout=120) for _ in range(ws))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (r0, msg0, freed0), (r1, msg1, freed1) = got
+    assert "could not be set up" in msg0 and "could not be set up" in msg1
+    assert "out of memory" in msg0                     # rank 0 names rank 1's failure
+    assert freed0 == [4096, 8192] and freed1 == []      # rank 0 freed both of its buffers
