@@ -123,8 +123,8 @@ constexpr int kPrefillRows = 256;
 bool prefill_supported(int H, int I);
 // xp [R, H] bf16 = x[perm[r] / k] for every routed row r (expert order).
 int launch_gather(const uint16_t* x, const int32_t* perm, int k, int64_t R, int H, void* xp, cudaStream_t s);
-// xp [R, H] f16 = x[perm[r] / k] 2^s_r (s_r the row's prescale), colscale[r] = 2^-s_r.
-int launch_gather_f16(const uint16_t* x, const int32_t* perm, int k, int64_t R, int H, void* xp, float* colscale,
+// xp [T k, H] f16: row inv[t k + j] = x[t] 2^s_t (s_t the token's prescale), colscale there = 2^-s_t.
+int launch_gather_f16(const uint16_t* x, const int32_t* inv, int k, int64_t T, int H, void* xp, float* colscale,
                       cudaStream_t s);
 // hb [R, I] bf16 = silu(xp Wg^T gg) * (xp Wu^T gu); with colscale, xp holds prescaled f16 rows
 // (F16 MMA operands) whose results are multiplied by colscale[r], else bf16 rows.

@@ -366,7 +366,7 @@ int prefill_impl(const void* x, const float* logits, int64_t T, const moe_nvfp4_
   // that undo it sit in the unused second half of the h region (h is bf16 [R, I] there).
   float* colscale = reinterpret_cast<float*>(w8 + L.h + up256((size_t)R * I * 2));
   prof_before(MOE_NVFP4_KERNEL_PREFILL_GATHER, s);
-  if ((rc = after_launch(moe::launch_gather_f16(static_cast<const uint16_t*>(x), rb.perm, k, R, H, xp, colscale, s), s,
+  if ((rc = after_launch(moe::launch_gather_f16(static_cast<const uint16_t*>(x), rb.inv, k, T, H, xp, colscale, s), s,
                          "gather", &launches)))
     return rc;
   const int pairs = prefill_pair_kernel() ? moe::prefill2_pairs(info.sms) : 0;
@@ -581,7 +581,7 @@ int experts_impl(const void* x_rows, const int32_t* ids, int64_t R, const moe_nv
     void* hb = w8 + L.h;
     float* colscale = reinterpret_cast<float*>(w8 + L.h + up256((size_t)R * I * 2));
     prof_before(MOE_NVFP4_KERNEL_PREFILL_GATHER, s);
-    if ((rc = after_launch(moe::launch_gather_f16(xb, rb.perm, 1, R, H, xp, colscale, s), s, "gather", &launches)))
+    if ((rc = after_launch(moe::launch_gather_f16(xb, rb.inv, 1, R, H, xp, colscale, s), s, "gather", &launches)))
       return rc;
     const int pairs = prefill_pair_kernel() ? moe::prefill2_pairs(info.sms) : 0;
     prof_before(MOE_NVFP4_KERNEL_PREFILL_GATEUP, s);

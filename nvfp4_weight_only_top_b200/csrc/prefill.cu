@@ -456,16 +456,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Gathers the routed rows of x (bf16 [T, H]) in expert order into xp as f16 [R, H], each row
 // times the exact power of two 2^s that puts its largest magnitude in [2^9, 2^10) (the decode
 // kernels' prescale; every BF16 value down to 2^-23 of the row's maximum is exact in f16), and
-// writes colscale[r] = 2^-s.  One CTA of 128 threads per routed row: the maximum first, then the
-// conversion.
+// writes colscale[p] = 2^-s.  One CTA of 128 threads per token: its row is read and converted
+// once (the maximum first), then stored at the place inv[t*k + j] of each of its k routed rows.
 constexpr int kGatherThreads = 128;
 constexpr int kGatherPer = 8;          // 16-byte chunks per thread (H <= 8192)
 __global__ void __launch_bounds__(kGatherThreads) gather_f16_kernel(const uint16_t* __restrict__ x,
-                                                                   const int32_t* __restrict__ perm, int k, int H,
+                                                                   const int32_t* __restrict__ inv, int k, int H,
                                                                    uint16_t* __restrict__ xp,
                                                                    float* __restrict__ colscale) {
-  const int64_t r = blockIdx.x;
-  const int t = perm[r] / k;
+  const int64_t t = blockIdx.x;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
   const int n8 = H / 8;
   uint4 v[kGatherPer];
@@ -485,7 +484,6 @@ __global__ void __launch_bounds__(kGatherThreads) gather_f16_kernel(const uint16
   m = max(max(s_m[0], s_m[1]), max(s_m[2], s_m[3]));
   const int sh = prescale_shift_bf16(m);
   const float f = exp2_int(sh);
-  uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * H);
 #pragma unroll
   for (int i = 0; i < kGatherPer; ++i) {
     const int c = (int)threadIdx.x + i * kGatherThreads;
@@ -494,10 +492,20 @@ __global__ void __launch_bounds__(kGatherThreads) gather_f16_kernel(const uint16
       uint32_t o[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) o[j] = pack_f16x2(bf16_bits_to_f32(w[j] & 0xFFFFu) * f, bf16_bits_to_f32(w[j] >> 16) * f);
-      dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
+      v[i] = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
-  if (threadIdx.x == 0) colscale[r] = exp2_int(-sh);
+  // the token's row goes to the place of each of its k routed rows
+  for (int j = 0; j < k; ++j) {
+    const int64_t p = inv[t * k + j];
+    uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)p * H);
+#pragma unroll
+    for (int i = 0; i < kGatherPer; ++i) {
+      const int c = (int)threadIdx.x + i * kGatherThreads;
+      if (c < n8) dst[c] = v[i];
+    }
+    if (threadIdx.x == 0) colscale[p] = exp2_int(-sh);
+  }
 }
 
 // Gathers the routed rows of x (bf16 [T, H]) in expert order into xp (bf16 [R, H]).
@@ -601,10 +609,10 @@ int make_tensor_map(CUtensorMap* map, int rank, const void* base, const uint64_t
 
 bool prefill_supported(int H, int I) { return H % 256 == 0 && I % 256 == 0; }
 
-int launch_gather_f16(const uint16_t* x, const int32_t* perm, int k, int64_t R, int H, void* xp, float* colscale,
+int launch_gather_f16(const uint16_t* x, const int32_t* inv, int k, int64_t T, int H, void* xp, float* colscale,
                       cudaStream_t s) {
   if (H / 8 > kGatherPer * kGatherThreads) return -(int)cudaErrorInvalidValue;
-  gather_f16_kernel<<<(unsigned)R, kGatherThreads, 0, s>>>(x, perm, k, H, static_cast<uint16_t*>(xp), colscale);
+  gather_f16_kernel<<<(unsigned)T, kGatherThreads, 0, s>>>(x, inv, k, H, static_cast<uint16_t*>(xp), colscale);
   const cudaError_t err = cudaGetLastError();
   return err == cudaSuccess ? 1 : -(int)err;
 }
