@@ -273,3 +273,44 @@ def test_ep_calls_reject_bad_arguments():
     with pytest.raises(ValueError):                         # ids of the wrong length
         moe.moe_nvfp4_experts(torch.zeros((4, 512), dtype=torch.bfloat16, device="cuda"),
                               torch.zeros(3, dtype=torch.int32, device="cuda"), bank)
+
+
+def test_expert_parallel_layer_world_size_one_matches_layer():
+    """ExpertParallel itself (the host orchestration, the IPC receive buffers, NCCL counts and
+    barriers) in a one-rank NCCL process group on one GPU, both transports, two steps each: equal
+    bit for bit to the single-GPU layer on the same expert kernels."""
+    import os
+    import socket
+    import subprocess
+    import sys
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    code = (
+        "import datetime, numpy as np, torch, torch.distributed as dist, moe_inputs\n"
+        "import nvfp4_weight_only_top_b200 as moe\n"
+        "from nvfp4_weight_only_top_b200.ep import ExpertParallel\n"
+        "from gpu_helpers import device_bank, bf16_tensor, bits_of\n"
+        "torch.cuda.set_device(0)\n"
+        "dist.init_process_group('nccl', rank=0, world_size=1, timeout=datetime.timedelta(seconds=120))\n"
+        "cfg = moe_inputs.LayerConfig('ep1', 16, 4, 512, 256, 300, 1, 'normal', seed=4)\n"
+        "buf, bank = device_bank(cfg)\n"
+        "x = bf16_tensor(moe_inputs.make_x(cfg))\n"
+        "lg = torch.from_numpy(moe_inputs.make_logits(cfg)).cuda()\n"
+        "want = moe.moe_nvfp4_forward_ex(x, lg, bank, cfg.k, path=moe.PATH_PREFILL)\n"
+        "for transport in ('peer', 'collective'):\n"
+        "    layer = ExpertParallel(bank, cfg.k, transport=transport, capacity_rows=cfg.T * cfg.k, path=moe.PATH_PREFILL)\n"
+        "    for step in range(2):\n"
+        "        out = layer.forward(x, lg)\n"
+        "        torch.cuda.synchronize()\n"
+        "        assert moe.moe_nvfp4_device_status() == 0\n"
+        "        assert np.array_equal(bits_of(out), bits_of(want)), (transport, step)\n"
+        "    layer.close()\n"
+        "dist.destroy_process_group()\n"
+        "print('ep world 1 ok')\n")
+    here = os.path.dirname(os.path.abspath(__file__))
+    env = dict(os.environ, MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK="0", WORLD_SIZE="1",
+               NCCL_NVLS_ENABLE="0",
+               PYTHONPATH=os.pathsep.join([here, os.path.dirname(here), os.environ.get("PYTHONPATH", "")]))
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and "ep world 1 ok" in r.stdout, r.stdout[-2000:] + r.stderr[-2000:]
