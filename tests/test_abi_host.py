@@ -255,3 +255,96 @@ def test_w4a4_binding_checks_scales_and_taps():
         moe.moe_nvfp4_forward_w4a4(x, lg, bank, _cpu((16,), torch.float32), 2, out=out)
     with pytest.raises(ValueError, match="act_scales has dtype"):
         moe.moe_nvfp4_forward_w4a4(x, lg, bank, _cpu((16, 2), torch.float16), 2, out=out)
+
+
+# ---- experts-only call and expert parallelism: host validation (nothing reaches a device)
+
+def _vp(v):
+    return ctypes.c_void_p(v)
+
+
+def test_experts_call_rejects_bad_arguments_on_the_host():
+    lib = moe.lib()
+    b = _bank()
+    call = lambda R=4, path=0, flags=0, bank=b: lib.moe_nvfp4_experts(        # noqa: E731
+        _vp(0x20000), _vp(0x30000), R, ctypes.byref(bank) if bank is not None else None, _vp(0x40000), None, 0, path,
+        flags, None)
+    assert call(bank=None) == _abi.ERR_INVALID_ARG
+    assert call(R=-1) == _abi.ERR_INVALID_ARG
+    assert call(path=7) == _abi.ERR_INVALID_ARG
+    assert call(flags=2) == _abi.ERR_INVALID_ARG
+    assert "flags" in moe.moe_nvfp4_last_error()
+    assert call(bank=_bank(hidden=200)) == _abi.ERR_UNSUPPORTED
+
+
+def test_experts_workspace_bytes():
+    f = moe.moe_nvfp4_experts_workspace_bytes
+    assert f(-1, 16, 512, 256) == 0 and f(8, 0, 512, 256) == 0 and f(8, 16, 64, 256) == 0
+    small, big = f(8, 16, 512, 256), f(4096, 16, 512, 256)
+    assert 0 < small < big
+    # the h and y regions alone: R x (I + H) x 4 bytes
+    assert big >= 4096 * (256 + 512) * 4
+
+
+@pytest.mark.parametrize("G,E,rank,layout,rows,code", [
+    (0, 8, 0, 0, 0, _abi.ERR_INVALID_ARG),     # no ranks
+    (65, 130, 0, 0, 0, _abi.ERR_INVALID_ARG),  # more ranks than the kernels take
+    (3, 8, 0, 0, 0, _abi.ERR_INVALID_ARG),     # experts do not split evenly
+    (2, 8, 2, 0, 0, _abi.ERR_INVALID_ARG),     # rank outside 0..G-1
+    (2, 8, 0, 2, 0, _abi.ERR_INVALID_ARG),     # unknown layout
+    (2, 8, 0, 0, -1, _abi.ERR_INVALID_ARG),    # negative row count
+])
+def test_ep_plan_rejects_bad_arguments(G, E, rank, layout, rows, code):
+    lib = moe.lib()
+    assert lib.moe_nvfp4_ep_plan(_vp(0x1000), G, E, rank, layout, _vp(0x2000), _vp(0x3000), rows, None) == code
+
+
+def test_ep_dispatch_and_combine_reject_bad_arguments():
+    lib = moe.lib()
+    ptrs = (ctypes.c_void_p * 2)(0x50000, 0x60000)
+    disp = lambda T=4, k=2, H=512, E=8, G=2, cap=16: lib.moe_nvfp4_ep_dispatch(     # noqa: E731
+        _vp(0x20000), T, k, H, E, _vp(0x1000), _vp(0x2000), _vp(0x3000), _vp(0x4000), G, ptrs, cap, None)
+    assert disp(k=0) == _abi.ERR_INVALID_ARG
+    assert disp(k=9) == _abi.ERR_INVALID_ARG        # k > E
+    assert disp(T=-1) == _abi.ERR_INVALID_ARG
+    assert disp(E=9) == _abi.ERR_INVALID_ARG        # 9 experts over 2 ranks
+    assert disp(H=12) == _abi.ERR_UNSUPPORTED       # not a multiple of 8
+    assert disp(H=8200) == _abi.ERR_UNSUPPORTED     # above 8192
+    comb = lambda T=4, k=2, H=512, E=8, G=2, cap=16: lib.moe_nvfp4_ep_combine(      # noqa: E731
+        _vp(0x20000), T, k, H, E, _vp(0x1000), _vp(0x2000), _vp(0x3000), _vp(0x4000), _vp(0x5000), G, ptrs, cap,
+        _vp(0x70000), None, None)
+    assert comb(k=0) == _abi.ERR_INVALID_ARG
+    assert comb(G=0) == _abi.ERR_INVALID_ARG
+    assert comb(H=12) == _abi.ERR_UNSUPPORTED
+
+
+def test_gather_rows_combine_and_buffers_reject_bad_arguments():
+    lib = moe.lib()
+    assert lib.moe_nvfp4_gather_rows(_vp(0x20000), _vp(0x1000), 4, 0, 512, _vp(0x30000), None) == _abi.ERR_INVALID_ARG
+    assert lib.moe_nvfp4_gather_rows(_vp(0x20000), _vp(0x1000), 4, 2, 500, _vp(0x30000), None) == \
+        _abi.ERR_UNSUPPORTED
+    assert lib.moe_nvfp4_combine(_vp(0x1000), _vp(0x2000), _vp(0x3000), -1, 2, 512, None, _vp(0x4000), None,
+                                 None) == _abi.ERR_INVALID_ARG
+    p = ctypes.c_void_p()
+    h = (ctypes.c_uint8 * 64)()
+    assert lib.moe_nvfp4_ep_buffer_create(0, ctypes.byref(p), h) == _abi.ERR_INVALID_ARG
+    assert lib.moe_nvfp4_ep_buffer_open(None, ctypes.byref(p)) == _abi.ERR_INVALID_ARG
+    assert lib.moe_nvfp4_ep_buffer_close(None) == _abi.OK          # closing nothing is a no-op
+    assert lib.moe_nvfp4_ep_buffer_destroy(None) == _abi.OK
+
+
+def test_ep_bindings_check_tensors_before_devices():
+    import torch
+    b = _bank(num_experts=8, hidden=256)
+    with pytest.raises(ValueError):          # ids of the wrong dtype
+        moe.moe_nvfp4_experts(torch.zeros((4, 256), dtype=torch.bfloat16), torch.zeros(4, dtype=torch.int64), b)
+    with pytest.raises(ValueError):          # y rows of the wrong width
+        moe.moe_nvfp4_experts(torch.zeros((4, 256), dtype=torch.bfloat16), torch.zeros(4, dtype=torch.int32), b,
+                              y_rows=torch.zeros((4, 128), dtype=torch.float32))
+    with pytest.raises(ValueError):          # counts of the wrong dtype
+        moe.moe_nvfp4_ep_plan(torch.zeros((2, 8), dtype=torch.int64), 0, 0)
+    with pytest.raises(ValueError):          # perm of the wrong length
+        moe.moe_nvfp4_gather_rows(torch.zeros((4, 256), dtype=torch.bfloat16), torch.zeros(7, dtype=torch.int32), 2,
+                                  rows=torch.zeros((8, 256), dtype=torch.bfloat16))
+    with pytest.raises(ValueError):          # an ep buffer handle has 64 bytes
+        moe.moe_nvfp4_ep_buffer_open(b"short")

@@ -314,3 +314,24 @@ def test_expert_parallel_layer_world_size_one_matches_layer():
                PYTHONPATH=os.pathsep.join([here, os.path.dirname(here), os.environ.get("PYTHONPATH", "")]))
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0 and "ep world 1 ok" in r.stdout, r.stdout[-2000:] + r.stderr[-2000:]
+
+
+@pytest.mark.parametrize("path", [1, 2])
+def test_experts_caller_workspace_matches_internal_bitwise(path):
+    """A caller workspace of exactly moe_nvfp4_experts_workspace_bytes gives the same result as the
+    internal one; one byte less is refused before anything runs."""
+    import torch
+    moe = _moe()
+    cfg = moe_inputs.LayerConfig(name="experts_ws", E=16, k=1, H=512, I=256, T=200, seed=6)
+    buf, bank = device_bank(cfg)
+    x = bf16_tensor(moe_inputs.make_x(cfg))
+    ids = torch.from_numpy(np.random.default_rng(2).integers(-1, 16, 200).astype(np.int32)).cuda()
+    n = moe.moe_nvfp4_experts_workspace_bytes(200, 16, 512, 256, path)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    a = moe.moe_nvfp4_experts(x, ids, bank, path=path)
+    b = moe.moe_nvfp4_experts(x, ids, bank, path=path, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_nvfp4_experts(x, ids, bank, path=path, workspace=ws[:n - 1])
+    assert ei.value.code == -4
