@@ -236,10 +236,11 @@ size_t moe_nvfp4_experts_workspace_bytes(int64_t R, int32_t E, int32_t H, int32_
                                          int32_t path);
 
 /*
- * Expert parallelism (EP) over G ranks, one process per GPU.  Source: the pages' servers run the
- * model with expert parallelism over eight GPUs (page "Running Beam-1.0 (501B) on workstation
- * GPUs", the serving configurations; page "Beam 1.0 501B-A23B, streaming pack, NVFP4 experts /
- * MLX 8-bit residents", the eight-GPU server line).  The layer is the one of moe_nvfp4_forward;
+ * Expert parallelism (EP) over G ranks, one process per GPU.  Source: the official deployment of
+ * the model runs tensor and expert parallelism over eight GPUs (page "Beam 1.0 501B", the
+ * model-information page's introduction: TP8/EP8); the workstation recipe uses tensor
+ * parallelism over four (page "Running Beam-1.0 (501B) on workstation GPUs", its serving
+ * command).  The layer is the one of moe_nvfp4_forward;
  * EP only changes where each expert runs.  Rank d holds global experts d*El .. d*El+El-1
  * (El = E / G) as a bank of El records (a moe_nvfp4_bank whose base points at record d*El of the
  * full bank layout) and routes its own tokens over all E with moe_nvfp4_route (ids, w, counts,

@@ -12,9 +12,10 @@
 //   combine   reads each routed row's expert output back from the owner's output buffer (peer
 //             loads) and forms out[t] = bf16(sum_j w[t, j] * y[t, j]) with the layer's own f32
 //             accumulation order.
-// The pages' servers run the model with tensor and expert parallelism over eight GPUs (page
-// "Running Beam-1.0 (501B) on workstation GPUs", the serving configurations; page "Beam 1.0
-// 501B-A23B, streaming pack, NVFP4 experts / MLX 8-bit residents", the eight-GPU server line).
+// The official deployment of the model runs tensor and expert parallelism over eight GPUs (page
+// "Beam 1.0 501B", the model-information page's introduction: TP8/EP8); the workstation recipe
+// uses tensor parallelism over four (page "Running Beam-1.0 (501B) on workstation GPUs", its
+// serving command).
 #include <cuda_runtime.h>
 
 #include <cstring>

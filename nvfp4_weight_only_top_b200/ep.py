@@ -1,8 +1,9 @@
 """Expert parallelism (EP) of the MoE layer over G GPUs, one process per GPU.
 
-The pages' servers run the model with expert parallelism over eight GPUs (page "Running
-Beam-1.0 (501B) on workstation GPUs", the serving configurations; page "Beam 1.0 501B-A23B,
-streaming pack, NVFP4 experts / MLX 8-bit residents", the eight-GPU server line).  EP changes
+The pages' servers split the model over several GPUs: the official deployment uses tensor and
+expert parallelism over eight GPUs (page "Beam 1.0 501B", the model-information page's
+introduction: TP8/EP8) and the workstation recipe tensor parallelism over four (page "Running
+Beam-1.0 (501B) on workstation GPUs", its serving command).  EP changes
 where each expert runs, not what the layer computes: rank d holds global experts d*El ..
 d*El+El-1 (El = E / G) and routes its own tokens over all E experts; every routed row travels
 to its expert's owner, is run there, and its result travels back to be combined.
