@@ -256,3 +256,29 @@ def test_peer_buffer_setup_fails_on_every_rank_together_gloo():
     assert "could not be set up" in msg0 and "could not be set up" in msg1
     assert "out of memory" in msg0                     # rank 0 names rank 1's failure
     assert freed0 == [4096, 8192] and freed1 == []      # rank 0 freed both of its buffers
+
+
+def test_plan_invariants_on_random_count_matrices():
+    """For many random count matrices: every owner's receive buffer is filled exactly once (the
+    places of all ranks' rows tile [0, recv_total) without overlap), the two layouts hold the same
+    rows, and the receive ids count each local expert's rows."""
+    rng = np.random.default_rng(11)
+    for _ in range(200):
+        G = int(rng.integers(1, 9))
+        El = int(rng.integers(1, 6))
+        E = G * El
+        C = rng.integers(0, 7, size=(G, E)) * (rng.random((G, E)) < 0.7)
+        plans = [ep.plan(C, s) for s in range(G)]
+        for key in ("expert_major", "source_major"):
+            for d in range(G):
+                cover = np.zeros(plans[d]["recv_total"], dtype=np.int64)
+                for s in range(G):
+                    for g in range(d * El, (d + 1) * El):
+                        o = plans[s][f"dst_off_{key}"][g]
+                        cover[o:o + C[s, g]] += 1
+                assert np.all(cover == 1), (G, El, key, d)
+                ids = plans[d][f"recv_ids_{key}"]
+                assert np.array_equal(np.bincount(ids, minlength=El), C[:, d * El:(d + 1) * El].sum(axis=0))
+        for s in range(G):
+            assert sum(plans[s]["send"]) == C[s].sum()
+            assert plans[s]["recv_total"] == plans[0]["recv_totals"][s]
