@@ -59,6 +59,10 @@ def parse():
                     help="plain layer calls on a small bank for ncu captures (no timing, no graph)")
     ap.add_argument("--calls", type=int, default=4, help="layer calls of --ncu-case")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--parallel", default="replicas", choices=["replicas", "ep"],
+                    help="replicas (default): every rank runs the whole layer on its own tokens; ep: expert "
+                         "parallelism over the job's ranks (peer transport), one workload (--config, default "
+                         "prefill_t8192)")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=20.0,
                     help="seconds of oracle work for the reference arm / CPU baseline")
@@ -733,6 +737,64 @@ def measure_ep(cfg, G: int = 8, steps: int = 10, warm: int = 3) -> dict:
             "peaks": {"hbm_gbs": hbm, "bf16_tflops": tf_burst, "kind": peak_kind, "nvlink_gbs": NVLINK_GBS}}
 
 
+def run_ep(args, ws, rank, local) -> None:
+    """--parallel ep: the layer with expert parallelism over the job's ranks, one per GPU (rank d
+    owns experts d E/N .. (d+1) E/N - 1 and routes its own T tokens over all E; peer transport).
+    Each step is ExpertParallel.forward, which synchronises with the host once (the gathered
+    counts); timed with CUDA events between barriers, max over ranks; value = all ranks' tokens /
+    that time.  With one process a one-rank process group is made."""
+    import socket
+    import torch
+    import torch.distributed as dist
+    import nvfp4_weight_only_top_b200 as moe
+    from nvfp4_weight_only_top_b200.ep import ExpertParallel
+    from moe_inputs import device as mdev
+    if not dist.is_initialized():
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", str(port))
+        import datetime
+        dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    name = args.config or "prefill_t8192"
+    cfg = moe_inputs.CONFIGS[name]
+    if cfg.layers != 1 or cfg.E % ws:
+        raise SystemExit(f"--parallel ep takes a one-layer workload whose experts split over {ws} ranks")
+    lay = cfg.layout
+    buf = mdev.bank_tensor(lay, cfg.seed, 0)        # the full layout; a rank reads only its experts
+    bank = moe.make_bank(buf.data_ptr(), lay.E, lay.H, lay.I, lay.record_stride, lay.codes_off, lay.scales_off,
+                         lay.global_off, 0)
+    x = torch.from_numpy(moe_inputs.make_x(cfg, seed=cfg.seed + rank).view(np.int16)).view(torch.bfloat16).cuda()
+    lg = torch.from_numpy(moe_inputs.make_logits(cfg, seed=cfg.seed + rank)).cuda()
+    layer = ExpertParallel(bank, cfg.k, transport="peer", capacity_rows=cfg.T * cfg.k * min(ws, 4))
+    steps = args.steps if args.steps is not None else 20
+    warm = args.warmup if args.warmup is not None else 3
+    for _ in range(warm):
+        layer.forward(x, lg)
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        out = layer.forward(x, lg)
+    e1.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms = max_over_ranks(ws, e0.elapsed_time(e1) / steps)
+    assert moe.moe_nvfp4_device_status() == 0 and out.shape == x.shape
+    layer.close()
+    if rank == 0:
+        print(json.dumps({"metric": f"MoE-layer tok/s, expert parallel over {ws} GPU(s) (peer transport)",
+                          "value": cfg.T * ws / (ms / 1000.0), "unit": "tok/s", "n_gpus": ws, "steps": steps,
+                          "warmup": warm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                          "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                          "config": dict(workload_config(cfg), parallelism=f"ep{ws}", tokens_per_rank=cfg.T,
+                                         experts_per_rank=cfg.E // ws)}), flush=True)
+    dist.destroy_process_group()
+
+
 def measure_encoder(experts: int = 16, reps: int = 5) -> dict:
     """NVFP4 encoding of `experts` full-size BF16 experts (gate and up [2560, 5120], down
     [5120, 2560]) into bank records; HBM-bound.  The algorithmic minimum is one read of the BF16
@@ -905,6 +967,9 @@ def main():
     import torch
 
     ws, rank, local = dist_init()
+    if args.parallel == "ep":
+        run_ep(args, ws, rank, local)
+        return
     names = [args.config] if args.config else FULL_RUN
     recs = {}
     for name in names:
