@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(kPlanThreads) ep_plan_kernel(const int32_t* __
   extern __shared__ int sm[];
   int* tot = sm;            // [E]: rows of expert g over all ranks
   int* seg = sm + E;        // [El * G]: this rank's receive segments in buffer order -> their starts
-  __shared__ int lane_sum[32];
+  __shared__ int s_total;      // rows sent to this rank
   const int El = E / G, nseg = El * G;
   for (int i = threadIdx.x; i < nseg; i += blockDim.x) {
     int e, s;
@@ -76,10 +76,10 @@ __global__ void __launch_bounds__(kPlanThreads) ep_plan_kernel(const int32_t* __
       seg[i] = run;
       run += v;
     }
-    if (lane == 31) lane_sum[0] = incl;            // rows sent here in total
+    if (lane == 31) s_total = incl;
   }
   __syncthreads();
-  const int total = lane_sum[0];
+  const int total = s_total;
   if (blockIdx.x == 0) {
     for (int g = threadIdx.x; g < E; g += blockDim.x) {
       const int d = g / El, e = g - d * El;
@@ -213,11 +213,11 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(int64_t T, int k, int H
 
 }  // namespace
 
-size_t ep_plan_smem_bytes(int G, int E) { return (size_t)(E + E) * sizeof(int); }
+size_t ep_plan_smem_bytes(int E) { return (size_t)(E + E) * sizeof(int); }   // tot[E] and seg[El * G = E]
 
 int launch_ep_plan(const int32_t* C, int G, int E, int rank, int layout, int32_t* dst_off, int32_t* recv_ids,
                    int64_t recv_rows, cudaStream_t s) {
-  const size_t smem = ep_plan_smem_bytes(G, E);
+  const size_t smem = ep_plan_smem_bytes(E);
   const int64_t ctas = recv_rows > 0 ? (recv_rows + kPlanRowsPerCta - 1) / kPlanRowsPerCta : 1;
   ep_plan_kernel<<<(unsigned)ctas, kPlanThreads, smem, s>>>(C, G, E, rank, layout, dst_off, recv_ids, recv_rows);
   const cudaError_t err = cudaGetLastError();

@@ -169,7 +169,7 @@ int launch_w4a4_down(const BankView& bank, const float* act_scales, const uint8_
 // Expert parallelism over peer memory (ep.cu).  Ranks G <= kEpMaxRanks; the plan writes dst_off [E]
 // and recv_ids [recv_rows]; dispatch and combine take G peer pointers (host array).
 constexpr int kEpMaxRanks = 64;
-size_t ep_plan_smem_bytes(int G, int E);
+size_t ep_plan_smem_bytes(int E);
 int launch_ep_plan(const int32_t* C, int G, int E, int rank, int layout, int32_t* dst_off, int32_t* recv_ids,
                    int64_t recv_rows, cudaStream_t s);
 bool ep_move_supported(int H);
